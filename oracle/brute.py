@@ -1,0 +1,34 @@
+"""Second, independent CPU implementation of the LoRA delta -- TEST INFRASTRUCTURE ONLY.
+
+numpy fp64 matrix products per adapter group: for every adapter i, gather the rows of the
+tokens that name it and evaluate ``y0 + s_i * (x_g @ A_i^T) @ B_i^T``.  This groups tokens
+by adapter (the grouping SGMV performs, "Compress then Serve" review thread, rebuttal on
+Punica) and uses library matrix products, so it shares neither loop structure nor
+summation order with ``lora_oracle.c``.
+"""
+from __future__ import annotations
+
+from typing import Sequence
+
+import numpy as np
+
+from workloads import to_float64
+
+
+def lora_delta(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray,
+               A: Sequence[np.ndarray], B: Sequence[np.ndarray], scales: Sequence[float],
+               y_offset: int = 0, o: int = None) -> np.ndarray:
+    ids = np.asarray(ids)
+    if ((ids < -1) | (ids >= len(A))).any():
+        raise ValueError("adapter id out of range")
+    if o is None:
+        o = y0.shape[1] - y_offset
+    xd = to_float64(x, dtype)
+    out = to_float64(y0, dtype)[:, y_offset:y_offset + o].copy()
+    for i in np.unique(ids[ids >= 0]):
+        rows = np.nonzero(ids == i)[0]
+        Ai = to_float64(A[i], dtype)
+        Bi = to_float64(B[i], dtype)
+        s = float(np.float32(scales[i]))
+        out[rows] += s * ((xd[rows] @ Ai.T) @ Bi.T)
+    return out

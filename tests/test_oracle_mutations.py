@@ -1,0 +1,73 @@
+"""The pins must catch plausible slips in the oracle.
+
+Each case copies the oracle's C source to a temporary directory, plants one mistake by a
+text substitution, builds that copy with gcc and runs the pin tests against it: at least
+one pin has to fail.  The committed oracle is never modified and no GPU is involved.
+"""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "lora_oracle.c")
+
+MUTATIONS = {
+    "transposed_A": ("acc += xrow[j] * widen(A[i], dtype, (int64_t)k * h + j)",
+                     "acc += xrow[j] * widen(A[i], dtype, (int64_t)j * r + k)"),
+    "transposed_B": ("widen(B[i], dtype, n * r + k) * v[k]", "widen(B[i], dtype, (int64_t)k * o + n) * v[k]"),
+    "dropped_y0": ("yr[n] = widen(y0, dtype, t * ldy + y_offset + n);\n            int32_t i",
+                   "yr[n] = 0.0;\n            int32_t i"),
+    "scale_squared": ("yr[n] += scales[i] * acc;\n            }\n        }\n        free(v);",
+                      "yr[n] += scales[i] * scales[i] * acc;\n            }\n        }\n        free(v);"),
+    "scale_dropped": ("yr[n] += scales[i] * acc;\n            }\n        }\n        free(v);",
+                      "yr[n] += acc;\n            }\n        }\n        free(v);"),
+    "neighbour_id": ("int32_t i = ids[t];\n            if (i < 0)\n                continue;\n            int32_t r",
+                     "int32_t i = ids[(t + 1) % T];\n            if (i < 0)\n                continue;\n            int32_t r"),
+    "rank_off_by_one": ("for (int32_t k = 0; k < r; ++k) {\n                double acc = 0.0;\n                for (int64_t j = 0; j < h; ++j)\n                    acc += xrow[j]",
+                        "for (int32_t k = 0; k < r - 1; ++k) {\n                double acc = 0.0;\n                for (int64_t j = 0; j < h; ++j)\n                    acc += xrow[j]"),
+    "unstable_segments": ("for (int64_t t = 0; t < T; ++t)\n        if (ids[t] >= 0)\n            perm[next[ids[t]]++]",
+                          "for (int64_t t = T - 1; t >= 0; --t)\n        if (ids[t] >= 0)\n            perm[next[ids[t]]++]"),
+    "offset_ignored": ("widen(y0, dtype, t * ldy + y_offset + n);\n            int32_t i",
+                       "widen(y0, dtype, t * ldy + n);\n            int32_t i"),
+}
+
+PIN_TESTS = [
+    lambda: [pins.test_loop_matches_grouped_matrix_products(n, d)
+             for n in ("tiny_sgmv", "multirank_decode") for d in (False, True)],
+    lambda: pins.test_single_adapter_equals_merged_weight("tiny_sgmv"),
+    lambda: [pins.test_selection_matrices_closed_form("f32", *s) for s in [(8, 8, 8), (24, 8, 16)]],
+    pins.test_rank_one_closed_form,
+    lambda: pins.test_zero_B_or_zero_scale_leaves_y_unchanged("B"),
+    pins.test_delta_linear_in_scale,
+    pins.test_mixed_ranks_equal_per_adapter_runs,
+    pins.test_output_slice_offset,
+    pins.test_exhaustive_tiny_against_outer_products,
+    lambda: [pins.test_segments_equal_stable_argsort(s) for s in (1, 2)],
+]
+
+
+@pytest.mark.parametrize("mut", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(mut, tmp_path):
+    old, new = MUTATIONS[mut]
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation anchor not unique: %s" % mut
+    path = tmp_path / "mut.c"
+    path.write_text(src.replace(old, new))
+    so = str(tmp_path / ("libmut_%s.so" % mut))
+    subprocess.check_call(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c99", "-o", so, str(path)])
+    saved = oracle._load()
+    oracle._lib = oracle.bind(so)
+    failures = 0
+    try:
+        for pin in PIN_TESTS:
+            try:
+                pin()
+            except (AssertionError, oracle.OracleError, ValueError):
+                failures += 1
+    finally:
+        oracle._lib = saved
+    assert failures > 0, "no pin caught the planted mistake %s" % mut

@@ -1,0 +1,330 @@
+"""Pins for the CPU oracle: closed forms, invariants and brute force that the LoRA
+definition and the pages fix.  None of these re-types the oracle's loop; each is chosen so
+that a plausible slip in the oracle (a dropped term, a transposed operand, a wrong index, the
+scale on the wrong step) fails at least one of them.
+
+Definition pinned: per token, y = y0 + s_i * B_i (A_i x) with i the token's adapter
+("TGI Multi-LoRA" page, "Technical Foundation: LoRA"; "Compress then Serve" review thread,
+add_lora_slice pseudocode: A with scale 1 into an fp32 buffer, then B with the scale into a
+slice of y).
+"""
+import itertools
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.brute as brute
+import workloads
+from workloads import accounting, bf16_bits_to_f32, f32_to_bf16_bits, to_float64
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _adapters(p, n):
+    return [p.A(i) for i in range(n)], [p.B(i) for i in range(n)]
+
+
+SMALL = {
+    "tiny_sgmv": {},
+    "decode_bgmv": dict(shapes=[("q", 512, 384, 0)]),
+    "multirank_decode": dict(T=96, n=24, shapes=[("q", 256, 320, 0)]),
+    "prefill_sgmv": dict(n=3, seg_len=130, shapes=[("up", 256, 448, 0)]),
+    "many_adapter_qkvo": dict(T=64, n=50, shapes=[("q", 256, 256, 0), ("k", 256, 64, 0),
+                                                  ("v", 256, 64, 0), ("o", 256, 256, 1)]),
+}
+
+
+@pytest.mark.parametrize("name", workloads.WORKLOAD_NAMES)
+@pytest.mark.parametrize("delta_only", [False, True])
+def test_loop_matches_grouped_matrix_products(name, delta_only):
+    wl = workloads.generate(name, delta_only=delta_only, **SMALL[name])
+    for p in wl.projections:
+        A, B = _adapters(p, wl.n)
+        ref = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+        alt = brute.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+        scale = max(np.abs(alt).max(), 1e-30)
+        assert np.abs(ref - alt).max() <= 1e-12 * scale
+
+
+@pytest.mark.parametrize("name", ["tiny_sgmv", "decode_bgmv"])
+def test_single_adapter_equals_merged_weight(name):
+    """A batch whose tokens all use adapter 0 equals y0 + x (W_delta)^T with the merged
+    weight W_delta = s * B A formed first (o x h), the LoRA merge of the definition."""
+    over = {} if name == "tiny_sgmv" else dict(shapes=[("q", 384, 256, 0)], T=12)
+    wl = workloads.generate(name, **over)
+    p = wl.projections[0]
+    ids = np.zeros(wl.T, dtype=np.int32)
+    A, B = _adapters(p, wl.n)
+    ref = oracle.lora_delta(wl.dtype, p.x, p.y0, ids, A, B, p.scales)
+    s = float(p.scales[0])
+    dW = s * (to_float64(B[0], wl.dtype) @ to_float64(A[0], wl.dtype))
+    merged = to_float64(p.y0, wl.dtype) + to_float64(p.x, wl.dtype) @ dW.T
+    assert np.allclose(ref, merged, rtol=0, atol=1e-12 * np.abs(merged).max())
+
+
+def _int_store(a, dtype):
+    a = np.asarray(a, dtype=np.float32)
+    return f32_to_bf16_bits(a) if dtype == "bf16" else a
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("h,r,o", [(8, 8, 8), (24, 8, 16), (16, 4, 40)])
+def test_selection_matrices_closed_form(dtype, h, r, o):
+    """A_i selects coordinates pa (A[k, pa[k]] = 1), B_i selects rank slots pb
+    (B[n, pb[n]] = 1): the delta is exactly s * x[t, pa[pb[n]]].  A transposed or mis-indexed
+    operand selects different coordinates."""
+    rng = np.random.default_rng(7)
+    T = 5
+    pa = rng.permutation(h)[:r]
+    pb = rng.integers(0, r, size=o)
+    A = np.zeros((r, h), np.float32)
+    A[np.arange(r), pa] = 1
+    B = np.zeros((o, r), np.float32)
+    B[np.arange(o), pb] = 1
+    x = rng.integers(-8, 9, size=(T, h)).astype(np.float32)
+    y0 = rng.integers(-8, 9, size=(T, o)).astype(np.float32)
+    s = 0.5
+    ids = np.zeros(T, np.int32)
+    ref = oracle.lora_delta(dtype, _int_store(x, dtype), _int_store(y0, dtype), ids,
+                            [_int_store(A, dtype)], [_int_store(B, dtype)], [s])
+    want = y0.astype(np.float64) + s * x[:, pa[pb]].astype(np.float64)
+    assert np.array_equal(ref, want)
+
+
+def test_rank_one_closed_form():
+    """All rows of A equal u and all columns of B equal w: delta = s * r * (u . x) * w."""
+    rng = np.random.default_rng(11)
+    T, h, r, o = 6, 32, 5, 12
+    u = rng.integers(-3, 4, size=h).astype(np.float32)
+    w = rng.integers(-3, 4, size=o).astype(np.float32)
+    A = np.tile(u, (r, 1))
+    B = np.tile(w[:, None], (1, r))
+    x = rng.integers(-4, 5, size=(T, h)).astype(np.float32)
+    y0 = rng.integers(-4, 5, size=(T, o)).astype(np.float32)
+    s = 0.25
+    ref = oracle.lora_delta("f32", x, y0, np.zeros(T, np.int32), [A], [B], [s])
+    want = y0 + s * r * (x @ u)[:, None] * w[None, :]
+    assert np.array_equal(ref, want.astype(np.float64))
+
+
+@pytest.mark.parametrize("which", ["B", "s"])
+def test_zero_B_or_zero_scale_leaves_y_unchanged(which):
+    wl = workloads.generate("multirank_decode", **SMALL["multirank_decode"])
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    sc = np.array(p.scales)
+    if which == "B":
+        B = [np.zeros_like(b) for b in B]
+    else:
+        sc = np.zeros_like(sc)
+    ref = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, sc)
+    assert np.array_equal(ref, to_float64(p.y0, wl.dtype))
+
+
+def test_delta_linear_in_scale():
+    """Doubling s doubles the delta exactly (a power-of-two scale is exact in fp64); a
+    scale applied twice, or to both steps, breaks this."""
+    wl = workloads.generate("multirank_decode", delta_only=True, **SMALL["multirank_decode"])
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    d1 = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    d2 = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, 2 * p.scales)
+    assert np.array_equal(d2, 2 * d1)
+    assert np.abs(d1).max() > 0
+
+
+def test_token_permutation_permutes_output():
+    wl = workloads.generate("many_adapter_qkvo", **SMALL["many_adapter_qkvo"])
+    p = wl.projections[1]
+    A, B = _adapters(p, wl.n)
+    ref = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    perm = np.random.default_rng(3).permutation(wl.T)
+    ref_p = oracle.lora_delta(wl.dtype, p.x[perm], p.y0[perm], wl.ids[perm], A, B, p.scales)
+    assert np.array_equal(ref_p, ref[perm])
+
+
+def test_mixed_ranks_equal_per_adapter_runs():
+    """The multi-rank batch equals, row for row, batches that each carry one adapter
+    (all other tokens without adapter)."""
+    wl = workloads.generate("multirank_decode", **SMALL["multirank_decode"])
+    p = wl.projections[0]
+    assert len(set(p.ranks.tolist())) > 1
+    A, B = _adapters(p, wl.n)
+    ref = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    for i in np.unique(wl.ids):
+        ids_i = np.where(wl.ids == i, wl.ids, -1).astype(np.int32)
+        one = oracle.lora_delta(wl.dtype, p.x, p.y0, ids_i, A, B, p.scales)
+        rows = wl.ids == i
+        assert np.array_equal(one[rows], ref[rows])
+        assert np.array_equal(one[~rows], to_float64(p.y0, wl.dtype)[~rows])
+
+
+def test_zero_padding_rank_changes_nothing():
+    wl = workloads.generate("multirank_decode", **SMALL["multirank_decode"])
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    R = int(p.ranks.max())
+    Ap = [np.concatenate([a, np.zeros((R - a.shape[0], a.shape[1]), a.dtype)]) for a in A]
+    Bp = [np.concatenate([b, np.zeros((b.shape[0], R - b.shape[1]), b.dtype)], axis=1) for b in B]
+    ref = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    pad = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, Ap, Bp, p.scales)
+    assert np.array_equal(ref, pad)
+
+
+def test_no_adapter_rows_and_bad_ids():
+    wl = workloads.generate("tiny_sgmv")
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    ids = wl.ids.copy()
+    ids[::3] = -1
+    ref = oracle.lora_delta(wl.dtype, p.x, p.y0, ids, A, B, p.scales)
+    assert np.array_equal(ref[ids < 0], p.y0[ids < 0].astype(np.float64))
+    for bad in (wl.n, -2):
+        ids2 = wl.ids.copy()
+        ids2[1] = bad
+        with pytest.raises(oracle.OracleError):
+            oracle.lora_delta(wl.dtype, p.x, p.y0, ids2, A, B, p.scales)
+        with pytest.raises(oracle.OracleError):
+            oracle.build_segments(ids2, wl.n)
+
+
+def test_output_slice_offset():
+    """The delta lands in columns [y_offset, y_offset + o) of a wider y (the fused-output
+    slice of the pseudocode); the oracle reads y0 only there."""
+    wl = workloads.generate("tiny_sgmv")
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    wide = np.random.default_rng(5).standard_normal((wl.T, 3 * p.o)).astype(np.float32)
+    wide[:, 96:96 + p.o] = p.y0
+    ref_off = oracle.lora_delta(wl.dtype, p.x, wide, wl.ids, A, B, p.scales, y_offset=96, o=p.o)
+    ref = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    assert np.array_equal(ref_off, ref)
+
+
+def test_exhaustive_tiny_against_outer_products():
+    """T = 3 tokens, two adapters of ranks 2 and 3 plus "no adapter": every one of the
+    3**3 id assignments, integer inputs, compared exactly with W_i = s_i * sum_k
+    outer(B_i[:, k], A_i[k, :]) in rational arithmetic."""
+    rng = np.random.default_rng(13)
+    T, h, o = 3, 4, 5
+    ranks = [2, 3]
+    A = [rng.integers(-3, 4, size=(r, h)).astype(np.float32) for r in ranks]
+    B = [rng.integers(-3, 4, size=(o, r)).astype(np.float32) for r in ranks]
+    s = [Fraction(1, 2), Fraction(3, 1)]
+    x = rng.integers(-3, 4, size=(T, h)).astype(np.float32)
+    y0 = rng.integers(-3, 4, size=(T, o)).astype(np.float32)
+    W = []
+    for i in range(2):
+        Wi = [[Fraction(0)] * h for _ in range(o)]
+        for k in range(ranks[i]):
+            for n_ in range(o):
+                for j in range(h):
+                    Wi[n_][j] += s[i] * int(B[i][n_, k]) * int(A[i][k, j])
+        W.append(Wi)
+    for combo in itertools.product([-1, 0, 1], repeat=T):
+        ids = np.array(combo, np.int32)
+        ref = oracle.lora_delta("f32", x, y0, ids, A, B, [float(v) for v in s])
+        for t in range(T):
+            for n_ in range(o):
+                want = Fraction(int(y0[t, n_]))
+                if ids[t] >= 0:
+                    want += sum(W[ids[t]][n_][j] * int(x[t, j]) for j in range(h))
+                assert Fraction(ref[t, n_]) == want
+
+
+def test_shrink_and_expand_steps():
+    """Shrink alone against a library product; expand alone against a library product on a
+    given fp32 intermediate; shrink then expand (fp32 intermediate) against the delta."""
+    wl = workloads.generate("multirank_decode", **SMALL["multirank_decode"])
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    R = int(p.ranks.max())
+    v = oracle.lora_shrink(wl.dtype, p.x, wl.ids, A, ldv=R)
+    xd = to_float64(p.x, wl.dtype)
+    for t in range(wl.T):
+        i = wl.ids[t]
+        r = p.ranks[i]
+        want = to_float64(A[i], wl.dtype) @ xd[t]
+        assert np.allclose(v[t, :r], want, rtol=0, atol=1e-12 * max(1.0, np.abs(want).max()))
+        assert not v[t, r:].any()
+    v32 = workloads.random_intermediate(wl.T, R, seed=9)
+    e = oracle.lora_expand(wl.dtype, v32, p.y0, wl.ids, B, p.scales)
+    y0d = to_float64(p.y0, wl.dtype)
+    for t in range(wl.T):
+        i = wl.ids[t]
+        r = p.ranks[i]
+        want = y0d[t] + float(p.scales[i]) * (to_float64(B[i], wl.dtype) @ v32[t, :r].astype(np.float64))
+        assert np.allclose(e[t], want, rtol=0, atol=1e-12 * np.abs(want).max())
+    full = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    composed = oracle.lora_expand(wl.dtype, v.astype(np.float32), p.y0, wl.ids, B, p.scales)
+    assert np.abs(composed - full).max() <= 1e-6 * np.abs(full).max()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_segments_equal_stable_argsort(seed):
+    rng = np.random.default_rng(seed)
+    n = [1, 7, 1000][seed]
+    T = [0, 33, 4096][seed]
+    ids = rng.integers(-1, n, size=T).astype(np.int32)
+    perm, seg_ptr, seg_adapter = oracle.build_segments(ids, n)
+    valid = np.nonzero(ids >= 0)[0]
+    order = valid[np.argsort(ids[valid], kind="stable")]
+    assert np.array_equal(perm, order)
+    uniq, counts = np.unique(ids[valid], return_counts=True)
+    assert np.array_equal(seg_adapter, uniq)
+    assert np.array_equal(seg_ptr, np.concatenate([[0], np.cumsum(counts)]).astype(np.int32))
+
+
+def test_segments_of_workloads():
+    for name in ("decode_bgmv", "multirank_decode", "many_adapter_qkvo"):
+        wl = workloads.generate(name, shapes=[("q", 8, 8, 0)])
+        perm, seg_ptr, seg_adapter = oracle.build_segments(wl.ids, wl.n)
+        for s in range(len(seg_adapter)):
+            toks = perm[seg_ptr[s]:seg_ptr[s + 1]]
+            assert (wl.ids[toks] == seg_adapter[s]).all()
+            assert (np.diff(toks) > 0).all()
+        assert (np.diff(seg_adapter) > 0).all()
+
+
+def test_page_size_figures_pin_byte_accounting():
+    g = json.load(open(os.path.join(HERE, "golden", "page_sizes.json")))
+    m = g["mistral7b"]
+    shapes = {"q": (m["hidden"], m["hidden"]), "k": (m["hidden"], m["kv_out"]),
+              "v": (m["hidden"], m["kv_out"]), "o": (m["hidden"], m["hidden"])}
+    b = accounting.adapter_bytes([shapes[p] for p in g["reading_projections"]],
+                                 g["reading_rank"], m["layers"], 2)
+    assert round(b / 1e6, 1) == g["adapter_mb"]
+    assert b / (g["base_gb"] * 1e9) < g["adapter_over_base_below"]
+    inc = g["n_adapters_for_vram_claim"] * g["adapter_mb"] / (g["base_gb"] * 1e3)
+    assert abs(inc - g["vram_increase_roughly"]) < 0.005
+
+
+def test_workload_byte_accounting_counts_distinct_adapters():
+    wl = workloads.generate("decode_bgmv", shapes=[("q", 64, 32, 0)])
+    d = np.unique(wl.ids)
+    e = 2
+    want = wl.T * 64 * e + 2 * wl.T * 32 * e + len(d) * 16 * (64 + 32) * e
+    assert accounting.workload_bytes(wl) == want
+
+
+def test_recipe_is_deterministic_and_rounded():
+    a = workloads.generate("decode_bgmv", shapes=[("q", 64, 32, 0)])
+    b = workloads.generate("decode_bgmv", shapes=[("q", 64, 32, 0)])
+    assert np.array_equal(a.ids, b.ids)
+    assert np.array_equal(a.projections[0].A_flat, b.projections[0].A_flat)
+    x32 = bf16_bits_to_f32(a.projections[0].x)
+    assert np.array_equal(f32_to_bf16_bits(x32), a.projections[0].x)
+    # variance vs std reading of N(0, 1/4096): std 1/64 vs 1/4096
+    s_var = np.std(bf16_bits_to_f32(a.projections[0].A_flat))
+    c = workloads.generate("decode_bgmv", shapes=[("q", 64, 32, 0)], reading="std")
+    s_std = np.std(bf16_bits_to_f32(c.projections[0].A_flat))
+    assert 0.8 / 64 < s_var < 1.2 / 64 and 0.8 / 4096 < s_std < 1.2 / 4096
+    z = workloads.generate("multirank_decode", shapes=[("q", 8, 8, 0)])
+    counts = np.bincount(z.ids, minlength=z.n)
+    assert counts[0] == counts.max() and set(z.projections[0].ranks) <= {8, 16, 32, 64}
+    pf = workloads.generate("prefill_sgmv", shapes=[("up", 8, 8, 0)])
+    assert np.array_equal(pf.ids, np.repeat(np.arange(8), 512))

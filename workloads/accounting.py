@@ -1,0 +1,56 @@
+"""Byte and FLOP accounting for the LoRA delta (measurement bookkeeping, no method arithmetic).
+
+Algorithmic bytes of one call over one projection:
+
+* x read once:                 T_valid * h * e
+* y read and written:          2 * T_valid * o * e
+* each distinct touched adapter's weights, once: r_i * (h + o) * e
+
+The rank-space intermediate, the ids and the segment table are not counted.  ``e`` is the
+element size (2 for bf16, 4 for fp32).  T_valid counts tokens whose id names an adapter.
+"""
+from __future__ import annotations
+
+from typing import Iterable, Sequence, Tuple
+
+import numpy as np
+
+ELEM_BYTES = {"bf16": 2, "f32": 4}
+
+
+def distinct_adapters(ids: np.ndarray) -> np.ndarray:
+    ids = np.asarray(ids)
+    return np.unique(ids[ids >= 0])
+
+
+def projection_bytes(T_valid: int, h: int, o: int, ranks_touched: Iterable[int], e: int) -> int:
+    w = sum(int(r) * (h + o) * e for r in ranks_touched)
+    return T_valid * h * e + 2 * T_valid * o * e + w
+
+
+def projection_flops(ids: np.ndarray, ranks: np.ndarray, h: int, o: int) -> int:
+    """Multiply-adds counted as 2 flops: shrink T*r*h plus expand T*o*r per token."""
+    ids = np.asarray(ids)
+    r = np.asarray(ranks)[ids[ids >= 0]].astype(np.int64)
+    return int(2 * (r * h).sum() + 2 * (r * o).sum())
+
+
+def workload_bytes(wl) -> int:
+    """Algorithmic bytes of one step of a workload (all projections)."""
+    e = ELEM_BYTES[wl.dtype]
+    d = distinct_adapters(wl.ids)
+    T_valid = int((np.asarray(wl.ids) >= 0).sum())
+    tot = 0
+    for p in wl.projections:
+        tot += projection_bytes(T_valid, p.h, p.o, (p.ranks[i] for i in d), e)
+    return tot
+
+
+def workload_flops(wl) -> int:
+    return sum(projection_flops(wl.ids, p.ranks, p.h, p.o) for p in wl.projections)
+
+
+def adapter_bytes(shapes: Sequence[Tuple[int, int]], rank: int, layers: int, e: int) -> int:
+    """Storage of one adapter: for every adapted (h -> o) projection of every layer,
+    A is r x h and B is o x r."""
+    return layers * sum(rank * (h + o) * e for (h, o) in shapes)
