@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Throughput of the heterogeneous-batch LoRA delta on B200.
+
+One step = one pass of the hot path over one batch of synthetic, seeded inputs.  The default
+workload is the decode form: a q_proj-shaped layer (4096 -> 4096), 32 rank-16 bf16 adapters,
+64 tokens with uniform per-token adapter ids, scale 2, run through ``lora_bgmv`` (per-token
+ids grouped on the device, one fused launch).  Other workloads: ``--workload``.
+
+Timing: the input set (adapter weights, x, y, ids) is replicated into C copies whose total
+exceeds 4x the L2 size, and consecutive steps rotate through the copies, so every step reads
+its weights from HBM.  Steps are captured into a CUDA graph of C calls and replayed; the timed
+region is exactly K steps between a barrier + synchronize on both sides, timed with CUDA
+events on the launching stream, max over ranks.  With ``torchrun`` each rank runs its own
+independent batches (the path shards by tokens with no exchange): weak scaling.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+from workloads import accounting  # noqa: E402
+
+METRIC = "tokens/s of batched multi-LoRA delta; fraction of HBM roofline"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+L2_BYTES = 126 * 1024 * 1024
+
+DESCRIPTIONS = {
+    "tiny_sgmv": "h=o=256, 4 adapters r8 fp32, 16 tokens uniform ids, s=2 (lora_sgmv)",
+    "decode_bgmv": "q_proj 4096->4096, 32 adapters r16 bf16, 64 tokens uniform ids, s=2 (lora_bgmv)",
+    "multirank_decode": "4096->4096, 128 adapters r in {8,16,32,64} bf16, 256 tokens Zipf(1.0), s=16/r "
+                        "(lora_build_segments + lora_sgmv)",
+    "prefill_sgmv": "up_proj 4096->14336, 8 contiguous segments x 512 tokens, r64 bf16, s=0.5 (lora_sgmv)",
+    "many_adapter_qkvo": "q,o 4096->4096 and k,v 4096->1024, 1000 adapters r16 bf16, 512 tokens Zipf(0.8), "
+                         "s=2 (lora_build_segments + 4 x lora_sgmv)",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0: about one second of work)")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_bgmv", choices=list(workloads.WORKLOAD_NAMES))
+    ap.add_argument("--copies", type=int, default=0, help="input copies rotated across steps (0: auto)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle CPU-baseline budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a graph")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if the
+    summary says it still matches the current kernel."""
+    path = os.path.join(ROOT, "profiles", "%s_ncu.md" % workload)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip()
+    try:
+        if vals.get("current", "yes").lower() != "yes":
+            return None
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--id=%s" % gpu_id, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Copy:
+    """One replica of the workload's inputs on the device plus its adapter tables."""
+
+    def __init__(self, wl, L, torch, shared_ids=None):
+        from workloads.device import upload_projection
+        self.projs = []
+        self.tables = []
+        for p in wl.projections:
+            d = upload_projection(p, wl.dtype)
+            t = L.AdapterTable(d.A_ptrs, d.B_ptrs, d.ranks, d.scales, p.h, p.o,
+                               L.LORA_BF16 if wl.dtype == "bf16" else L.LORA_F32, keep=d)
+            self.projs.append(d)
+            self.tables.append(t)
+        self.ids = torch.from_numpy(wl.ids).cuda()
+        n, T = wl.n, wl.T
+        self.seg_t = dict(perm=torch.empty(T, dtype=torch.int32, device="cuda"),
+                          seg_ptr=torch.empty(n + 1, dtype=torch.int32, device="cuda"),
+                          seg_adapter=torch.empty(n, dtype=torch.int32, device="cuda"),
+                          num=torch.empty(1, dtype=torch.int32, device="cuda"))
+        ws_bytes = max(t.workspace_bytes(T) for t in self.tables)
+        self.ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        if wl.name == "prefill_sgmv":
+            seg_len = wl.spec.seg_len
+            self.pf = dict(seg_ptr=torch.arange(0, T + 1, seg_len, dtype=torch.int32, device="cuda"),
+                           seg_adapter=torch.arange(n, dtype=torch.int32, device="cuda"),
+                           num=torch.tensor([n], dtype=torch.int32, device="cuda"))
+            self.seg = L.make_segments(None, self.pf["seg_ptr"], self.pf["seg_adapter"], self.pf["num"], T, n, seg_len)
+        else:
+            s = self.seg_t
+            self.seg = L.make_segments(s["perm"], s["seg_ptr"], s["seg_adapter"], s["num"], T, n)
+
+    def nbytes(self):
+        tot = self.ids.numel() * 4 + self.ws.numel()
+        for d in self.projs:
+            tot += d.A_flat.numel() * d.A_flat.element_size() + d.B_flat.numel() * d.B_flat.element_size()
+            tot += d.x.numel() * d.x.element_size() + d.y0.numel() * d.y0.element_size()
+        return tot
+
+
+def make_step(wl, L):
+    """Returns (step(copy, stream_handle), launches per step, name of the dominant kernel)."""
+    name = wl.name
+    T = wl.T
+
+    if name == "decode_bgmv":
+        def step(c, s):
+            d, t = c.projs[0], c.tables[0]
+            L.lora_bgmv(t.handle, c.ids, T, d.x, d.h, d.y0, d.o, 0, c.ws, c.ws.numel(), s)
+        return step, 1, "lora_decode_kernel (fused, per-token ids)"
+    if name in ("tiny_sgmv", "multirank_decode", "many_adapter_qkvo"):
+        def step(c, s):
+            st = c.seg_t
+            L.lora_build_segments(c.tables[0].handle, c.ids, T, st["perm"], st["seg_ptr"], st["seg_adapter"],
+                                  st["num"], s)
+            for d, t in zip(c.projs, c.tables):
+                L.lora_sgmv(t.handle, c.seg, d.x, d.h, d.y0, d.o, 0, c.ws, c.ws.numel(), s)
+        return step, 1 + len(wl.projections), "lora_decode_kernel (fused, segments)"
+    if name == "prefill_sgmv":
+        def step(c, s):
+            d, t = c.projs[0], c.tables[0]
+            L.lora_sgmv(t.handle, c.seg, d.x, d.h, d.y0, d.o, 0, c.ws, c.ws.numel(), s)
+        return step, 1, "prefill path"
+    raise ValueError(name)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import heterogeneous_adapters_sgmv_b200 as L
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    seed = workloads.SEED_BASE + workloads.WORKLOAD_NAMES.index(args.workload) + 1000 * rank
+    wl = workloads.generate(args.workload, seed=seed)
+    T = wl.T
+    step, launches_per_step, kname = make_step(wl, L)
+    bytes_step = accounting.workload_bytes(wl)
+    flops_step = accounting.workload_flops(wl)
+    distinct = int(accounting.distinct_adapters(wl.ids).size)
+
+    first = Copy(wl, L, torch)
+    ws_bytes = first.nbytes()
+    C = args.copies or max(1, min(256, -(-4 * L2_BYTES // ws_bytes)))
+    copies = [first] + [Copy(wl, L, torch) for _ in range(C - 1)]
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    sh = int(stream.cuda_stream)
+    K = args.steps
+    if K <= 0:
+        # about one second of work, from a short eager probe
+        with torch.cuda.stream(stream):
+            for i in range(3 * C):
+                step(copies[i % C], sh)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            for i in range(2 * C):
+                step(copies[i % C], sh)
+        torch.cuda.synchronize()
+        per = (time.perf_counter() - t0) / (2 * C)
+        K = int(max(1000, min(2_000_000, 1.0 / max(per, 1e-7) * 3)))   # graph replay is faster than eager
+        K = max(C, K // C * C)
+    W = max(args.warmup, 3)
+
+    # warm-up (eager) then capture one graph of C steps (and one of K % C steps)
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            step(copies[i % C], sh)
+    torch.cuda.synchronize()
+    graphs = []
+    if not args.no_graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(C):
+                step(copies[i], int(torch.cuda.current_stream().cuda_stream))
+        graphs.append(g)
+        rem = K % C
+        g2 = None
+        if rem:
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2, stream=stream):
+                for i in range(rem):
+                    step(copies[i], int(torch.cuda.current_stream().cuda_stream))
+        for _ in range(2):
+            with torch.cuda.stream(stream):
+                g.replay()
+        torch.cuda.synchronize()
+
+    gpu_id = torch.cuda.get_device_properties(local_rank).uuid
+    gpu_id = "GPU-%s" % gpu_id if not str(gpu_id).startswith("GPU-") else str(gpu_id)
+    if dist:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.3)   # let the sampler start before the timed region
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        if args.no_graph:
+            for i in range(K):
+                step(copies[i % C], sh)
+        else:
+            for _ in range(K // C):
+                graphs[0].replay()
+            if K % C:
+                g2.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist:
+        dist.barrier(device_ids=[local_rank])
+    ms = float(ev0.elapsed_time(ev1))
+    if dist:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / K
+    value = world * T * K / (ms / 1e3)
+
+    # roofline of the dominant kernel: per launch (for one-launch steps the launch is the step)
+    peak, peak_kind = measured_peaks()
+    kernel_ms = ms_step if launches_per_step == 1 else None
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profile_traffic(args.workload),
+                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
+                else "fallback 6.65 TB/s",
+                "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                "algorithmic_bytes_per_launch": bytes_step if launches_per_step == 1 else None,
+                "algorithmic_bytes_per_step": bytes_step,
+                "kernel": kname,
+                "kernel_ms_per_launch": round(kernel_ms, 6) if kernel_ms else None,
+                "basis": "step time (one launch per step)" if launches_per_step == 1 else
+                "whole step (all launches)"}
+
+    # end to end through the C ABI with host buffers: H2D inputs, the call, D2H of y
+    e2e = None
+    if args.e2e_steps > 0:
+        c = copies[0]
+        d = c.projs[0]
+        hx = [torch.empty_like(p.x, device="cpu").pin_memory() for p in c.projs]
+        hy = [torch.empty_like(p.y0, device="cpu").pin_memory() for p in c.projs]
+        hout = [torch.empty_like(p.y0, device="cpu").pin_memory() for p in c.projs]
+        hids = torch.from_numpy(wl.ids).pin_memory()
+        for i, p in enumerate(c.projs):
+            hx[i].copy_(p.x)
+            hy[i].copy_(p.y0)
+        h2d = sum(t.numel() * t.element_size() for t in hx + hy) + hids.numel() * 4
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        Ke = args.e2e_steps
+
+        def e2e_step():
+            c.ids.copy_(hids, non_blocking=True)
+            for i, p in enumerate(c.projs):
+                p.x.copy_(hx[i], non_blocking=True)
+                p.y0.copy_(hy[i], non_blocking=True)
+            step(c, sh)
+            for i, p in enumerate(c.projs):
+                hout[i].copy_(p.y0, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(W):
+                e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier(device_ids=[local_rank])
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(Ke):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ems = float(e0.elapsed_time(e1))
+        if dist:
+            tt = torch.tensor([ems], device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": round(world * T * Ke / (ems / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": Ke, "ms_per_step": round(ems / Ke, 6),
+               "path": "pinned host -> cudaMemcpyAsync -> C-ABI call -> cudaMemcpyAsync -> pinned host"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    codes = {"bf16": "bf16", "f32": "f32"}
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": codes[wl.dtype], "data": "synthetic (seeded; random adapter weights and activations)",
+        "config": {"workload": "%s: %s" % (args.workload, DESCRIPTIONS[args.workload]),
+                   "tokens_per_step": T, "distinct_adapters_per_step": distinct,
+                   "algorithmic_bytes_per_step": bytes_step, "flops_per_step": flops_step,
+                   "l2": "rotating %d input copies (%.0f MB > 4x L2)" % (C, C * ws_bytes / 1e6),
+                   "graph": not args.no_graph, "pdl": bool(L.lora_get_option("pdl")),
+                   "parallelism": "replicas x%d (independent token batches, no collective)" % world},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks,
+        "gpu_launches": int(K * launches_per_step),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    for c in copies:
+        for t in c.tables:
+            t.close()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _oracle_tokens_per_s(wl, T_sample: int, seconds: float, threads: int = 0):
+    import oracle
+    sub = sample_workload(wl, T_sample)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        for pi in range(len(sub.projections)):
+            oracle.workload_reference(sub, pi, threads=threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return reps * T_sample / el, reps, el
+
+
+def sample_workload(wl, T_sample: int):
+    """The first T_sample tokens of the batch (same adapters, same weights)."""
+    import copy
+    if T_sample >= wl.T:
+        return wl
+    sub = copy.copy(wl)
+    sub.ids = wl.ids[:T_sample].copy()
+    sub.T = T_sample
+    sub.projections = []
+    for p in wl.projections:
+        q = copy.copy(p)
+        q.x = p.x[:T_sample]
+        q.y0 = p.y0[:T_sample]
+        sub.projections.append(q)
+    return sub
+
+
+def cpu_baseline(wl, seconds: float):
+    import oracle
+    threads = oracle.max_threads()
+    # calibrate on a small sample, then size the sample so one pass is a fraction of the budget
+    per_tok_s = None
+    Ts = min(wl.T, 8)
+    v, reps, el = _oracle_tokens_per_s(wl, Ts, 0.2, threads)
+    per_tok_s = 1.0 / v
+    T_sample = int(max(1, min(wl.T, seconds / 4 / per_tok_s)))
+    v, reps, el = _oracle_tokens_per_s(wl, T_sample, seconds, threads)
+    return {"value": round(v, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "first %d of %d tokens of one batch, all projections, repeated %d times (%.1f s), "
+                      "fp64 C loop with OpenMP over tokens" % (T_sample, wl.T, reps, el)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    wl = workloads.generate(args.workload)
+    threads = oracle.max_threads()
+    K, W = (args.steps if args.steps > 0 else 20), max(args.warmup, 3)
+    # size one step (a bounded sample of the batch) so that W + K steps take about a minute
+    v, _r, _e = _oracle_tokens_per_s(wl, min(wl.T, 4), 0.2, threads)
+    per_tok = 1.0 / v
+    T_sample = int(max(1, min(wl.T, 60.0 / (K + W) / per_tok)))
+    sub = sample_workload(wl, T_sample)
+    for _ in range(W):
+        for pi in range(len(sub.projections)):
+            oracle.workload_reference(sub, pi, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(K):
+        for pi in range(len(sub.projections)):
+            oracle.workload_reference(sub, pi, threads=threads)
+    el = time.perf_counter() - t0
+    value = K * T_sample / el
+    out = {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+           "ms_per_step": round(el / K * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+           "config": {"workload": "%s: %s" % (args.workload, DESCRIPTIONS[args.workload]),
+                      "tokens_per_step": T_sample},
+           "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
+                            "sample": "first %d of %d tokens per step" % (T_sample, wl.T)},
+           "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,408 @@
+// C ABI of liblora_sgmv.so: adapter tables, host-side validation, workspace carving and the
+// choice of device path.  Nothing here computes the delta; every step runs in the kernels of
+// decode.cu, segments.cu and prefill.cu.
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "lora_common.cuh"
+#include "lora_internal.h"
+
+namespace lora {
+
+static int64_t env_or(const char *name, int64_t dflt)
+{
+    const char *v = std::getenv(name);
+    if (!v || !*v) return dflt;
+    return std::strtoll(v, nullptr, 10);
+}
+
+Options &options()
+{
+    static Options o;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        o.pdl = env_or("LORA_PDL", o.pdl);
+        o.decode_stages = env_or("LORA_DECODE_STAGES", o.decode_stages);
+        o.decode_ctas_per_sm = env_or("LORA_DECODE_CTAS_PER_SM", o.decode_ctas_per_sm);
+        o.prefill_min_seg_len = env_or("LORA_PREFILL_MIN_SEG_LEN", o.prefill_min_seg_len);
+        o.split = env_or("LORA_SPLIT", o.split);
+    });
+    return o;
+}
+
+// prefill.cu
+bool prefill_supported(const lora_table *t);
+int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y,
+                   int64_t ldy, int32_t y_off, float *v, int32_t ldv, cudaStream_t s);
+
+}  // namespace lora
+
+using namespace lora;
+
+namespace {
+
+constexpr int kBgmvMaxT = 1024;
+constexpr int kBgmvMaxN = 4096;
+
+inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int esz(int dtype) { return dtype == LORA_BF16 ? 2 : 4; }
+inline int epc(int dtype) { return 16 / esz(dtype); }
+inline size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
+inline int ldv_of(const lora_table *t) { return (t->max_rank + 3) & ~3; }
+
+struct WsLayout {
+    size_t v, perm, seg_ptr, seg_adapter, num_segs, total;
+};
+
+WsLayout ws_layout(const lora_table *t, int32_t T)
+{
+    WsLayout w;
+    size_t off = 0;
+    w.v = off;
+    off += up256((size_t)T * ldv_of(t) * sizeof(float));
+    w.perm = off;
+    off += up256((size_t)T * sizeof(int32_t));
+    w.seg_ptr = off;
+    off += up256((size_t)(t->n + 1) * sizeof(int32_t));
+    w.seg_adapter = off;
+    off += up256((size_t)t->n * sizeof(int32_t));
+    w.num_segs = off;
+    off += 256;
+    w.total = off;
+    return w;
+}
+
+int check_table(const lora_table *t)
+{
+    if (!t || !t->d_desc) return LORA_ERR_INVALID_ARG;
+    return LORA_OK;
+}
+
+int check_io(const lora_table *t, const void *x, int64_t ldx, const void *y, int64_t ldy, int32_t y_off,
+             bool need_x, bool need_y)
+{
+    const int e = epc(t->dtype);
+    if (need_x) {
+        if (!x) return LORA_ERR_INVALID_ARG;
+        if (ldx < t->h) return LORA_ERR_INVALID_ARG;
+        if (!al16(x) || ldx % e) return LORA_ERR_UNSUPPORTED;
+    }
+    if (need_y) {
+        if (!y) return LORA_ERR_INVALID_ARG;
+        if (y_off < 0 || ldy < (int64_t)y_off + t->o) return LORA_ERR_INVALID_ARG;
+        if (!al16(y) || ldy % e || y_off % e) return LORA_ERR_UNSUPPORTED;
+    }
+    return LORA_OK;
+}
+
+int check_segments(const lora_segments *seg)
+{
+    if (!seg || !seg->seg_ptr || !seg->seg_adapter || !seg->num_segs) return LORA_ERR_INVALID_ARG;
+    if (seg->T < 0 || seg->max_segs < 0) return LORA_ERR_INVALID_ARG;
+    return LORA_OK;
+}
+
+DecodeParams base_params(const lora_table *t)
+{
+    DecodeParams p;
+    std::memset(&p, 0, sizeof p);
+    p.desc = t->d_desc;
+    p.n = t->n;
+    p.h = t->h;
+    p.o = t->o;
+    p.R = t->max_rank;
+    p.status = t->d_status;
+    return p;
+}
+
+void set_segments(DecodeParams &p, const lora_segments *seg)
+{
+    p.perm = seg->perm;
+    p.seg_ptr = seg->seg_ptr;
+    p.seg_adapter = seg->seg_adapter;
+    p.num_segs = seg->num_segs;
+    p.max_segs = seg->max_segs;
+    p.T = seg->T;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t dtype,
+                      const void *const *A, const void *const *B, const int32_t *ranks,
+                      const float *scales, void *stream)
+{
+    if (!out || !A || !B || !ranks || !scales) return LORA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (n < 1 || h < 1 || o < 1) return LORA_ERR_INVALID_ARG;
+    if (dtype != LORA_BF16 && dtype != LORA_F32) return LORA_ERR_UNSUPPORTED;
+    if (h % epc(dtype) || o % epc(dtype)) return LORA_ERR_UNSUPPORTED;
+    int max_rank = 0;
+    for (int i = 0; i < n; ++i) {
+        if (!A[i] || !B[i]) return LORA_ERR_INVALID_ARG;
+        if (ranks[i] < 1) return LORA_ERR_INVALID_ARG;
+        if (ranks[i] > LORA_MAX_RANK) return LORA_ERR_UNSUPPORTED;
+        if (!al16(A[i]) || !al16(B[i])) return LORA_ERR_UNSUPPORTED;
+        if (ranks[i] > max_rank) max_rank = ranks[i];
+    }
+    lora_table *t = new (std::nothrow) lora_table();
+    if (!t) return LORA_ERR_INVALID_ARG;
+    t->n = n;
+    t->h = h;
+    t->o = o;
+    t->dtype = dtype;
+    t->max_rank = max_rank;
+    t->d_desc = nullptr;
+    t->d_status = nullptr;
+    t->d_tmaps = nullptr;
+    if (cudaGetDevice(&t->device) != cudaSuccess) {
+        delete t;
+        return LORA_ERR_CUDA;
+    }
+    t->A.assign(A, A + n);
+    t->B.assign(B, B + n);
+    t->ranks.assign(ranks, ranks + n);
+    t->scales.assign(scales, scales + n);
+    AdapterDesc *h_desc = new (std::nothrow) AdapterDesc[n];
+    if (!h_desc) {
+        delete t;
+        return LORA_ERR_INVALID_ARG;
+    }
+    for (int i = 0; i < n; ++i) {
+        h_desc[i].A = A[i];
+        h_desc[i].B = B[i];
+        h_desc[i].rank = ranks[i];
+        h_desc[i].scale = scales[i];
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int rc = LORA_OK;
+    if (cudaMalloc(&t->d_desc, sizeof(AdapterDesc) * n) != cudaSuccess ||
+        cudaMalloc(&t->d_status, 256) != cudaSuccess ||
+        cudaMemcpyAsync(t->d_desc, h_desc, sizeof(AdapterDesc) * n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemsetAsync(t->d_status, 0, 256, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+        rc = LORA_ERR_CUDA;
+    delete[] h_desc;
+    if (rc != LORA_OK) {
+        lora_table_destroy(t);
+        return rc;
+    }
+    *out = t;
+    return LORA_OK;
+}
+
+int lora_table_destroy(lora_table *t)
+{
+    if (!t) return LORA_OK;
+    int prev = 0;
+    cudaGetDevice(&prev);
+    cudaSetDevice(t->device);
+    cudaDeviceSynchronize();
+    if (t->d_desc) cudaFree(t->d_desc);
+    if (t->d_status) cudaFree(t->d_status);
+    if (t->d_tmaps) cudaFree(t->d_tmaps);
+    cudaSetDevice(prev);
+    delete t;
+    return LORA_OK;
+}
+
+int lora_table_info(const lora_table *t, int32_t *n, int32_t *h, int32_t *o, int32_t *max_rank, int32_t *dtype)
+{
+    if (!t) return LORA_ERR_INVALID_ARG;
+    if (n) *n = t->n;
+    if (h) *h = t->h;
+    if (o) *o = t->o;
+    if (max_rank) *max_rank = t->max_rank;
+    if (dtype) *dtype = t->dtype;
+    return LORA_OK;
+}
+
+size_t lora_workspace_bytes(const lora_table *t, int32_t T)
+{
+    if (!t || T < 0) return 256;
+    return ws_layout(t, T).total;
+}
+
+int lora_build_segments(const lora_table *t, const int32_t *d_ids, int32_t T, int32_t *d_perm,
+                        int32_t *d_seg_ptr, int32_t *d_seg_adapter, int32_t *d_num_segs, void *stream)
+{
+    int rc = check_table(t);
+    if (rc) return rc;
+    if (T < 0 || !d_seg_ptr || !d_seg_adapter || !d_num_segs) return LORA_ERR_INVALID_ARG;
+    if (T > 0 && (!d_ids || !d_perm)) return LORA_ERR_INVALID_ARG;
+    if (T > LORA_MAX_SEGMENT_TOKENS) return LORA_ERR_UNSUPPORTED;
+    return launch_build_segments(d_ids, T, t->n, d_perm, d_seg_ptr, d_seg_adapter, d_num_segs, t->d_status,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+int lora_shrink(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, float *v,
+                int32_t ldv, void *stream)
+{
+    int rc = check_table(t);
+    if (rc) return rc;
+    if ((rc = check_segments(seg))) return rc;
+    if ((rc = check_io(t, x, ldx, nullptr, 0, 0, true, false))) return rc;
+    if (!v || ldv < t->max_rank) return LORA_ERR_INVALID_ARG;
+    if (ldv % 4 || !al16(v)) return LORA_ERR_UNSUPPORTED;
+    if (seg->T == 0 || seg->max_segs == 0) return LORA_OK;
+    DecodeParams p = base_params(t);
+    set_segments(p, seg);
+    p.x = x;
+    p.ldx = ldx;
+    p.v = v;
+    p.ldv = ldv;
+    return launch_decode(kModeShrink, kSrcSegments, p, t->dtype, static_cast<cudaStream_t>(stream));
+}
+
+int lora_expand(const lora_table *t, const lora_segments *seg, const float *v, int32_t ldv, void *y,
+                int64_t ldy, int32_t y_off, void *stream)
+{
+    int rc = check_table(t);
+    if (rc) return rc;
+    if ((rc = check_segments(seg))) return rc;
+    if ((rc = check_io(t, nullptr, 0, y, ldy, y_off, false, true))) return rc;
+    if (!v || ldv < t->max_rank) return LORA_ERR_INVALID_ARG;
+    if (ldv % 4 || !al16(v)) return LORA_ERR_UNSUPPORTED;
+    if (seg->T == 0 || seg->max_segs == 0) return LORA_OK;
+    DecodeParams p = base_params(t);
+    set_segments(p, seg);
+    p.y = y;
+    p.ldy = ldy;
+    p.y_off = y_off;
+    p.v = const_cast<float *>(v);
+    p.ldv = ldv;
+    return launch_decode(kModeExpand, kSrcSegments, p, t->dtype, static_cast<cudaStream_t>(stream));
+}
+
+int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y,
+              int64_t ldy, int32_t y_off, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_table(t);
+    if (rc) return rc;
+    if ((rc = check_segments(seg))) return rc;
+    if ((rc = check_io(t, x, ldx, y, ldy, y_off, true, true))) return rc;
+    if (seg->T == 0 || seg->max_segs == 0) return LORA_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Options &opt = options();
+    const bool prefill = opt.prefill_min_seg_len > 0 && seg->max_seg_len >= opt.prefill_min_seg_len &&
+                         seg->perm == nullptr && prefill_supported(t);
+    if (prefill || opt.split) {
+        const WsLayout w = ws_layout(t, seg->T);
+        if (!ws || ws_bytes < w.total) return LORA_ERR_WORKSPACE;
+        if (!al16(ws)) return LORA_ERR_UNSUPPORTED;
+        float *v = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + w.v);
+        if (prefill) return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, ldv_of(t), s);
+        if ((rc = lora_shrink(t, seg, x, ldx, v, ldv_of(t), stream))) return rc;
+        return lora_expand(t, seg, v, ldv_of(t), y, ldy, y_off, stream);
+    }
+    DecodeParams p = base_params(t);
+    set_segments(p, seg);
+    p.x = x;
+    p.ldx = ldx;
+    p.y = y;
+    p.ldy = ldy;
+    p.y_off = y_off;
+    return launch_decode(kModeFused, kSrcSegments, p, t->dtype, s);
+}
+
+int lora_bgmv(const lora_table *t, const int32_t *d_ids, int32_t T, const void *x, int64_t ldx, void *y,
+              int64_t ldy, int32_t y_off, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_table(t);
+    if (rc) return rc;
+    if (T < 0) return LORA_ERR_INVALID_ARG;
+    if ((rc = check_io(t, x, ldx, y, ldy, y_off, true, true))) return rc;
+    if (T == 0) return LORA_OK;
+    if (!d_ids) return LORA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T <= kBgmvMaxT && t->n <= kBgmvMaxN && !options().split) {
+        DecodeParams p = base_params(t);
+        p.ids = d_ids;
+        p.T = T;
+        p.x = x;
+        p.ldx = ldx;
+        p.y = y;
+        p.ldy = ldy;
+        p.y_off = y_off;
+        return launch_decode(kModeFused, kSrcIds, p, t->dtype, s);
+    }
+    // Larger batches: sort into the workspace, then run the segmented form.
+    if (T > LORA_MAX_SEGMENT_TOKENS) return LORA_ERR_UNSUPPORTED;
+    const WsLayout w = ws_layout(t, T);
+    if (!ws || ws_bytes < w.total) return LORA_ERR_WORKSPACE;
+    if (!al16(ws)) return LORA_ERR_UNSUPPORTED;
+    uint8_t *b = static_cast<uint8_t *>(ws);
+    lora_segments seg;
+    std::memset(&seg, 0, sizeof seg);
+    seg.perm = reinterpret_cast<int32_t *>(b + w.perm);
+    seg.seg_ptr = reinterpret_cast<int32_t *>(b + w.seg_ptr);
+    seg.seg_adapter = reinterpret_cast<int32_t *>(b + w.seg_adapter);
+    seg.num_segs = reinterpret_cast<int32_t *>(b + w.num_segs);
+    seg.T = T;
+    seg.max_segs = t->n;
+    if ((rc = lora_build_segments(t, d_ids, T, const_cast<int32_t *>(seg.perm), const_cast<int32_t *>(seg.seg_ptr),
+                                  const_cast<int32_t *>(seg.seg_adapter), const_cast<int32_t *>(seg.num_segs),
+                                  stream)))
+        return rc;
+    return lora_sgmv(t, &seg, x, ldx, y, ldy, y_off, ws, ws_bytes, stream);
+}
+
+int lora_get_status(const lora_table *t, uint32_t *h_status, int32_t reset, void *stream)
+{
+    if (!t || !h_status) return LORA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t w = 0;
+    if (cudaMemcpyAsync(&w, t->d_status, sizeof w, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    if (reset && (cudaMemsetAsync(t->d_status, 0, sizeof w, s) != cudaSuccess ||
+                  cudaStreamSynchronize(s) != cudaSuccess))
+        return LORA_ERR_CUDA;
+    *h_status = w;
+    if (w == 0) return LORA_OK;
+    return (w & LORA_STATUS_TIMEOUT) ? LORA_ERR_TIMEOUT : LORA_ERR_DEVICE_STATUS;
+}
+
+const char *lora_status_string(int code)
+{
+    switch (code) {
+    case LORA_OK: return "ok";
+    case LORA_ERR_INVALID_ARG: return "invalid argument";
+    case LORA_ERR_UNSUPPORTED: return "unsupported configuration (rank, alignment, dtype or size limit)";
+    case LORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LORA_ERR_CUDA: return "CUDA runtime error";
+    case LORA_ERR_TIMEOUT: return "a device-side bounded wait ran out";
+    case LORA_ERR_DEVICE_STATUS: return "the device latched an error (bad id or segment entry)";
+    default: return "unknown status";
+    }
+}
+
+int lora_set_option(const char *key, int64_t value)
+{
+    if (!key) return LORA_ERR_INVALID_ARG;
+    Options &o = options();
+    if (!std::strcmp(key, "pdl")) o.pdl = value;
+    else if (!std::strcmp(key, "decode_stages")) o.decode_stages = value;
+    else if (!std::strcmp(key, "decode_ctas_per_sm")) o.decode_ctas_per_sm = value;
+    else if (!std::strcmp(key, "prefill_min_seg_len")) o.prefill_min_seg_len = value;
+    else if (!std::strcmp(key, "split")) o.split = value;
+    else return LORA_ERR_INVALID_ARG;
+    return LORA_OK;
+}
+
+int lora_get_option(const char *key, int64_t *value)
+{
+    if (!key || !value) return LORA_ERR_INVALID_ARG;
+    const Options &o = options();
+    if (!std::strcmp(key, "pdl")) *value = o.pdl;
+    else if (!std::strcmp(key, "decode_stages")) *value = o.decode_stages;
+    else if (!std::strcmp(key, "decode_ctas_per_sm")) *value = o.decode_ctas_per_sm;
+    else if (!std::strcmp(key, "prefill_min_seg_len")) *value = o.prefill_min_seg_len;
+    else if (!std::strcmp(key, "split")) *value = o.split;
+    else return LORA_ERR_INVALID_ARG;
+    return LORA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Host-side internals shared by the translation units of liblora_sgmv.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "lora_sgmv.h"
+
+struct CUtensorMap_st;
+
+namespace lora {
+struct AdapterDesc;
+
+// Decode kernel modes: shrink+expand fused, shrink only (v to global), expand only (v from global).
+enum DecodeMode : int { kModeFused = 0, kModeShrink = 1, kModeExpand = 2 };
+// Where the work units come from: a segment table, or per-token ids grouped on the device.
+enum UnitSource : int { kSrcSegments = 0, kSrcIds = 1 };
+
+struct DecodeParams {
+    const AdapterDesc *desc;
+    int32_t n, h, o, R;    // adapters, in/out features, max rank of the table
+    const void *x;
+    int64_t ldx;
+    void *y;
+    int64_t ldy;
+    int32_t y_off;
+    int32_t ldv;
+    float *v;
+    const int32_t *perm, *seg_ptr, *seg_adapter, *num_segs;
+    int32_t max_segs;
+    const int32_t *ids;
+    int32_t T;
+    uint32_t *status;
+    int32_t stages;        // pipeline depth
+    int32_t stage_bytes;   // bytes of one stage (header + data)
+    int32_t ids_smem;      // kSrcIds: bytes of the id / leader scratch in shared memory
+};
+
+struct Options {
+    int64_t pdl = 1;
+    int64_t decode_stages = 0;       // 0: automatic
+    int64_t decode_ctas_per_sm = 0;  // 0: automatic
+    int64_t prefill_min_seg_len = 256;
+    int64_t split = 0;
+};
+Options &options();
+
+// Launchers (return a LORA_* code).
+int launch_decode(int mode, int src, const DecodeParams &p, int dtype, cudaStream_t s);
+int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *perm, int32_t *seg_ptr,
+                          int32_t *seg_adapter, int32_t *num_segs, uint32_t *status, cudaStream_t s);
+size_t decode_smem_bytes(int src, int R, int n, int T, int stages, int *stage_bytes, int *ids_smem, int dtype);
+
+}  // namespace lora
+
+struct lora_table {
+    int32_t n, h, o, dtype, max_rank;
+    int device;
+    lora::AdapterDesc *d_desc;
+    uint32_t *d_status;
+    std::vector<const void *> A, B;
+    std::vector<int32_t> ranks;
+    std::vector<float> scales;
+    // tcgen05 prefill path: per-adapter tensor maps (device array), built on first use.
+    void *d_tmaps;
+};

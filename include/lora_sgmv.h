@@ -1,0 +1,177 @@
+/*
+ * lora_sgmv.h -- C ABI of the heterogeneous-batch LoRA delta for B200 (sm_100a).
+ *
+ * The operation.  A batch of T tokens, each naming its own adapter i = id[t] and that
+ * adapter's rank r_i, receives the low-rank update of one projection of one layer:
+ *
+ *     v[t, 0:r_i]        = x[t, 0:h] . A_i^T                (shrink, scale 1, fp32 result)
+ *     y[t, off + n]     += s_i * sum_k v[t, k] * B_i[n, k]   (expand, n < o)
+ *
+ * Sources (multi-LoRA serving pages):
+ *   - "TGI Multi-LoRA: Deploy Once, Serve 30 Models", section "Technical Foundation: LoRA"
+ *     (frozen base weight plus two small trained matrices A and B) and section "How
+ *     Multi-LoRA Serving Works" (one adapter id per request; requests for different adapters
+ *     share one forward pass as a heterogeneous batch).
+ *   - "Compress then Serve" review thread, authors' rebuttal on Punica: SGMV groups the
+ *     requests that use the same LoRA model; the add_lora_slice_with_sigma pseudocode
+ *     applies A with scale 1 into an fp32 buffer of shape (tokens, R), then B with the
+ *     scale into the column slice [y_offset, y_offset + y_slice_size) of y, the adapter of
+ *     each token coming from a per-token index vector (its "indices").
+ *   - "how does this differ from S-LoRA?" (LoRAX issue): adapters of different ranks in one
+ *     batch, served by one kernel.
+ *
+ * Layouts (all row-major, element type E = bf16 or fp32 as the table says):
+ *   x  [T, ldx]   first h columns used           y  [T, ldy]   columns [y_offset, y_offset+o)
+ *   A_i [r_i, h]  (PEFT lora_A orientation)      B_i [o, r_i]  (PEFT lora_B orientation)
+ *   v  [T, ldv]   fp32, indexed by token (not by sorted position)
+ *
+ * Alignment: every pointer to x, y, A_i, B_i, v is 16-byte aligned; h, o, ldx, ldy and
+ * y_offset are multiples of 16 / sizeof(E); ldv is a multiple of 4.  Violations return
+ * LORA_ERR_UNSUPPORTED before anything is launched.
+ *
+ * Streams.  Every call enqueues on the given CUDA stream (a cudaStream_t passed as void*;
+ * NULL is the legacy default stream).  The hot calls (lora_build_segments, lora_shrink,
+ * lora_expand, lora_sgmv, lora_bgmv) never allocate, never synchronise the host, and never
+ * read device memory from the host.
+ *
+ * Errors.  Each call returns LORA_OK (0) or a negative LORA_ERR_* code.  Problems the host
+ * can see (null pointers, sizes, alignment, workspace size) are rejected before launch.
+ * Problems only the device can see -- an id outside [-1, n), a segment entry out of range,
+ * a bounded wait that ran out -- never trap: the offending token or segment is skipped and
+ * a bit is latched into the table's device status word, which lora_get_status reads.
+ * There is no CPU fallback: an unsupported configuration is an error.
+ *
+ * Ownership.  The caller owns x, y, v, ids, segment arrays, workspace and every A_i / B_i
+ * buffer, and keeps the weights alive while a table refers to them.  A table owns only its
+ * device descriptor array (adapter pointers, ranks, scales) and its status word.
+ */
+#ifndef LORA_SGMV_H
+#define LORA_SGMV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element types of a table (x, y, A_i and B_i share it). */
+#define LORA_F32 0
+#define LORA_BF16 1
+
+/* Return codes. */
+#define LORA_OK 0
+#define LORA_ERR_INVALID_ARG (-1)   /* null pointer, negative size, bad id in host data   */
+#define LORA_ERR_UNSUPPORTED (-2)   /* rank > LORA_MAX_RANK, alignment, dtype, size limits */
+#define LORA_ERR_WORKSPACE (-3)     /* workspace pointer null or smaller than required      */
+#define LORA_ERR_CUDA (-4)          /* a CUDA runtime call failed                           */
+#define LORA_ERR_TIMEOUT (-5)       /* a device-side bounded wait ran out (status word)     */
+#define LORA_ERR_DEVICE_STATUS (-6) /* lora_get_status found a latched device error         */
+
+/* Bits of the device status word. */
+#define LORA_STATUS_BAD_ID 1u       /* an id outside [-1, n) was skipped                    */
+#define LORA_STATUS_TIMEOUT 2u      /* a bounded wait gave up; that block stopped early     */
+#define LORA_STATUS_BAD_SEGMENT 4u  /* a segment entry (adapter, bounds, perm) was skipped */
+
+/* Limits. */
+#define LORA_MAX_RANK 128            /* largest r_i a table accepts                        */
+#define LORA_MAX_SEGMENT_TOKENS 8192 /* largest T lora_build_segments sorts in one call    */
+
+typedef struct lora_table lora_table; /* opaque */
+
+/* Segments: tokens grouped by adapter ("grouping requests that use the same LoRA model").
+ * Segment s covers sorted positions [seg_ptr[s], seg_ptr[s+1]); the token at sorted position
+ * p is perm[p], or p itself when perm is NULL (tokens already contiguous per adapter, as in
+ * prefill).  All arrays are device memory and may be produced by lora_build_segments. */
+typedef struct lora_segments {
+    const int32_t *perm;        /* [>= seg_ptr[num_segs]] token index per sorted position, or NULL */
+    const int32_t *seg_ptr;     /* [max_segs + 1] */
+    const int32_t *seg_adapter; /* [max_segs]    adapter of each segment */
+    const int32_t *num_segs;    /* [1]           number of segments S (<= max_segs) */
+    int32_t T;                  /* rows of x and y */
+    int32_t max_segs;           /* capacity of the segment arrays (host value) */
+    int32_t max_seg_len;        /* host hint: no segment is longer (0 = unknown) */
+    int32_t reserved;
+} lora_segments;
+
+/* Register the adapters of one (layer, projection).  A and B are HOST arrays of n DEVICE
+ * pointers; A[i] is [ranks[i], h_in], B[i] is [h_out, ranks[i]], both of element type dtype.
+ * ranks[i] in [1, LORA_MAX_RANK]; scales[i] is s_i.  The descriptor array is copied to the
+ * device on `stream`.  Stands in for the stacked per-layer weights and layer index of the
+ * pseudocode: one table per (layer, projection), adapters neither contiguous nor padded. */
+int lora_table_create(lora_table **out, int32_t n_adapters, int32_t h_in, int32_t h_out,
+                      int32_t dtype, const void *const *A, const void *const *B,
+                      const int32_t *ranks, const float *scales, void *stream);
+
+/* Free the table's device memory (synchronises the device first).  NULL is accepted. */
+int lora_table_destroy(lora_table *table);
+
+/* Table metadata (any output pointer may be NULL). */
+int lora_table_info(const lora_table *table, int32_t *n_adapters, int32_t *h_in,
+                    int32_t *h_out, int32_t *max_rank, int32_t *dtype);
+
+/* Bytes of device workspace that lora_sgmv and lora_bgmv need for T tokens (a multiple of
+ * 256; 0 is never returned). */
+size_t lora_workspace_bytes(const lora_table *table, int32_t T);
+
+/* Segment bookkeeping (SGMV grouping): a stable sort of the tokens by adapter id.
+ * Outputs, all device arrays: perm[T] (token of each sorted position; only the first
+ * seg_ptr[num_segs] entries are written), seg_ptr[n + 1], seg_adapter[n], num_segs[1].
+ * Segments come in ascending adapter id, one per adapter with at least one token, tokens in
+ * batch order inside a segment.  id -1 means "no adapter" and is left out; other ids outside
+ * [0, n) are left out and latch LORA_STATUS_BAD_ID.  T <= LORA_MAX_SEGMENT_TOKENS.
+ * Bit-exact: the result is unique. */
+int lora_build_segments(const lora_table *table, const int32_t *d_ids, int32_t T,
+                        int32_t *d_perm, int32_t *d_seg_ptr, int32_t *d_seg_adapter,
+                        int32_t *d_num_segs, void *stream);
+
+/* Shrink step alone: v[t, 0:r_i] = x[t] . A_i^T for every token of every segment (fp32
+ * accumulation, scale 1).  Columns >= r_i of v and rows of tokens outside all segments are
+ * not written.  ldv >= the table's max rank. */
+int lora_shrink(const lora_table *table, const lora_segments *seg, const void *x,
+                int64_t ldx, float *v, int32_t ldv, void *stream);
+
+/* Expand step alone: y[t, y_offset + n] = round(y[t, y_offset + n] + s_i * v[t, 0:r_i] . B_i[n])
+ * for every token of every segment, n < o, rounding once to nearest-even in E. */
+int lora_expand(const lora_table *table, const lora_segments *seg, const float *v,
+                int32_t ldv, void *y, int64_t ldy, int32_t y_offset, void *stream);
+
+/* SGMV: shrink and expand for sorted segments, in place on the y slice.  Picks the path:
+ * the fused cluster kernel (decode), or the tcgen05 tensor-core path when the hint
+ * max_seg_len is long, perm is NULL and the table is bf16 (prefill).  ws may be NULL when
+ * ws_bytes is 0 and the chosen path needs none; otherwise ws_bytes >=
+ * lora_workspace_bytes(table, seg->T). */
+int lora_sgmv(const lora_table *table, const lora_segments *seg, const void *x, int64_t ldx,
+              void *y, int64_t ldy, int32_t y_offset, void *ws, size_t ws_bytes, void *stream);
+
+/* BGMV: the same update driven by per-token ids (d_ids[T], device) without a caller-built
+ * segment table, as the per-token "indices" of the pseudocode.  Tokens sharing an adapter
+ * are grouped on the device so each adapter's weights are read once per group.  For
+ * T <= 1024 and n <= 4096 this is one launch that needs no workspace; larger batches sort
+ * into the workspace first. */
+int lora_bgmv(const lora_table *table, const int32_t *d_ids, int32_t T, const void *x,
+              int64_t ldx, void *y, int64_t ldy, int32_t y_offset, void *ws, size_t ws_bytes,
+              void *stream);
+
+/* Read (and with reset != 0, clear) the table's device status word into *h_status.
+ * Synchronises `stream`.  Returns LORA_OK when the word is 0, LORA_ERR_TIMEOUT when the
+ * timeout bit is set, otherwise LORA_ERR_DEVICE_STATUS. */
+int lora_get_status(const lora_table *table, uint32_t *h_status, int32_t reset, void *stream);
+
+/* Static text for a return code. */
+const char *lora_status_string(int code);
+
+/* Runtime knobs (process-wide, for tuning and tests).  key: "pdl" (0/1, programmatic
+ * dependent launch between consecutive calls), "decode_stages", "decode_ctas_per_sm",
+ * "prefill_min_seg_len" (segment-length hint at or above which lora_sgmv takes the tcgen05
+ * path; 0 disables that path), "split" (1: lora_sgmv runs lora_shrink then lora_expand
+ * through the workspace instead of the fused kernel).  Returns LORA_ERR_INVALID_ARG for an
+ * unknown key. */
+int lora_set_option(const char *key, int64_t value);
+int lora_get_option(const char *key, int64_t *value);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_SGMV_H */

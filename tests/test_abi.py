@@ -1,0 +1,67 @@
+"""The C-ABI library loads on a machine without a GPU and exports every entry point that
+include/lora_sgmv.h declares; host-only calls behave as documented.  No compute call is made."""
+import ctypes
+import os
+import re
+
+import heterogeneous_adapters_sgmv_b200 as L
+from heterogeneous_adapters_sgmv_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    txt = open(os.path.join(ROOT, "include", "lora_sgmv.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(lora_\w+)\s*\(", txt)))
+
+
+def test_library_builds_and_exports_every_declared_symbol():
+    path = B.build()
+    lib = ctypes.CDLL(path)
+    names = declared_functions()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(L.EXPORTS) == names
+
+
+def test_host_only_calls():
+    L._load()
+    assert L.status_string(L.LORA_ERR_WORKSPACE).startswith("workspace")
+    assert L.status_string(12345) == "unknown status"
+    lib = L._load()
+    assert lib.lora_table_info(None, None, None, None, None, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_workspace_bytes(None, 5) == 256
+    assert lib.lora_table_destroy(None) == L.LORA_OK
+    old = L.lora_get_option("split")
+    L.lora_set_option("split", 1)
+    assert L.lora_get_option("split") == 1
+    L.lora_set_option("split", old)
+    try:
+        L.lora_set_option("no_such_knob", 1)
+        raise AssertionError("unknown option accepted")
+    except L.LoraError as e:
+        assert e.code == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_table_create(None, 1, 8, 8, 1, None, None, None, None, None) == L.LORA_ERR_INVALID_ARG
+
+
+def test_header_constants_match_binding():
+    txt = open(os.path.join(ROOT, "include", "lora_sgmv.h")).read()
+    for name in ("LORA_F32", "LORA_BF16", "LORA_OK", "LORA_ERR_INVALID_ARG", "LORA_ERR_UNSUPPORTED",
+                 "LORA_ERR_WORKSPACE", "LORA_ERR_CUDA", "LORA_ERR_TIMEOUT", "LORA_ERR_DEVICE_STATUS",
+                 "LORA_STATUS_BAD_ID", "LORA_STATUS_TIMEOUT", "LORA_STATUS_BAD_SEGMENT", "LORA_MAX_RANK",
+                 "LORA_MAX_SEGMENT_TOKENS"):
+        m = re.search(r"#define %s \(?(-?\d+)u?\)?" % name, txt)
+        assert m, name
+        assert int(m.group(1)) == getattr(L, name), name
+
+
+def test_product_path_does_not_use_the_oracle():
+    """The package neither imports nor names the oracle: no CPU fallback exists."""
+    pkg = os.path.join(ROOT, "heterogeneous_adapters_sgmv_b200")
+    for dirpath, _d, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read().lower()
+                assert "oracle" not in src, f
