@@ -14,7 +14,8 @@ import os
 from typing import Optional, Sequence
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblora_sgmv.so")
+# LORA_SGMV_LIB selects another build of the same library (e.g. a phase-traced one).
+LIB_PATH = os.environ.get("LORA_SGMV_LIB") or os.path.join(_HERE, "liblora_sgmv.so")
 
 LORA_F32 = 0
 LORA_BF16 = 1

@@ -35,21 +35,28 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in sources() + headers())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False, out: str = None,
+          defines=()) -> str:
+    """Compile every csrc/*.cu into one shared library (default: the in-tree liblora_sgmv.so).
+    ``defines`` adds -D flags, e.g. ("LORA_TRACE",) for the phase-traced build written to ``out``."""
+    target = out or LIB
+    if not force and not defines and out is None and up_to_date():
         return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC] + FLAGS + ["-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"),
-                            "--threads", "0", "-o", tmp] + sources()
+    tmp = target + ".tmp%d" % os.getpid()
+    cmd = [NVCC] + FLAGS + ["-D%s" % d for d in defines] + [
+        "-I", os.path.join(ROOT, "include"), "-I", os.path.join(HERE, "csrc"), "--threads", "0", "-o", tmp] + sources()
     if ptxas_v:
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_v="--ptxas-v" in sys.argv)
-    print(LIB)
+    trace_out = None
+    if "--trace" in sys.argv:
+        trace_out = sys.argv[sys.argv.index("--trace") + 1]
+    print(build(force="--force" in sys.argv, verbose=True, ptxas_v="--ptxas-v" in sys.argv, out=trace_out,
+                defines=("LORA_TRACE",) if trace_out else ()))

@@ -7,29 +7,34 @@
 //  * A cluster of 8 CTAs owns one work unit at a time: up to 16 tokens of one adapter (one
 //    SGMV segment chunk, or one group of equal ids in the per-token BGMV form).  CTA j of the
 //    cluster streams the j-th eighth of h for the shrink and the j-th eighth of o for the
-//    expand, so each adapter's A_i and B_i are read exactly once per unit and every token of
-//    the unit reuses that read.
-//  * One producer warp per CTA moves all operands with untiled bulk async copies (TMA engine,
-//    no multicast) into a ring of shared-memory stages guarded by mbarriers; it runs ahead
-//    across units, so B_i and y of a unit are in flight while its shrink is computed.
-//  * Shrink: warp-level split-K.  A lane owns 16 bytes at two places of each 1 KiB row; 8
-//    partial dot products per lane are folded across the warp with a transposed butterfly
-//    (9 shuffles) instead of 8 separate reductions.
-//  * The 8 partial intermediates of a cluster are summed in a fixed CTA order through
-//    distributed shared memory, synchronised by remote mbarrier arrivals (no grid barrier, no
-//    atomics, bit-identical run to run).
-//  * Expand: each thread owns two output columns (bf16) and all tokens of the unit, reads its
-//    B rows once from shared memory and updates y from the staged copy; results are rounded
-//    once (round-to-nearest-even) and stored with coalesced 32-bit stores.
+//    expand, so each adapter's A_i and B_i are read once per unit and every token of the unit
+//    reuses that read.
+//  * One producer warp per CTA runs ahead across units: it stages this CTA's slice of A_i with
+//    2-D tensor-map TMA loads (one or two instructions per unit) and its slice of B_i with one
+//    bulk copy, into a ring of shared-memory stages guarded by mbarriers, and hints the unit's
+//    x and y rows into L2.  No multicast anywhere.
+//  * Consumer warps stage x and y rows with coalesced 128-bit loads.  Shrink: warp-level
+//    split-K, a lane owns 16 bytes at two places of each 1 KiB row; 8 partial dot products per
+//    lane are folded across the warp with a transposed butterfly.
+//  * Each CTA pushes its partial intermediate into every peer's shared memory with st.async
+//    (completion counted in bytes on the peer's mbarrier); every CTA then sums the 8 partials in
+//    fixed CTA order.  No atomics, no grid barrier: bit-identical run to run.
+//  * Expand: a thread owns two output columns (bf16) and walks the unit's tokens; one rounding
+//    (nearest-even) per output, coalesced 32-bit stores.
 //  * Persistent grid: as many clusters as fit, each walking the unit list with a stride.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <climits>
-#include <cstdio>
 #include <mutex>
 
 #include "lora_common.cuh"
 #include "lora_internal.h"
 
 namespace lora {
+#ifdef LORA_TRACE
+__device__ unsigned long long lora_trace_buf[kTraceCtas * kTraceSlots];
+#endif
 namespace {
 
 constexpr int kCluster = 8;
@@ -37,7 +42,9 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;   // + one producer warp
 constexpr int kTokChunk = 16;               // tokens per work unit
-constexpr int kRowBytes = 1024;             // one staged row of a tile
+constexpr int kRowBytes = 1024;             // h-subtile row (shrink) / o-subtile span (expand);
+                                            // 512 for ranks above 64 (smaller stages)
+constexpr int kBoxBytes = 512;              // one TMA box row of A
 constexpr int kMaxStages = 4;
 constexpr int kHeaderBytes = 128;
 
@@ -47,18 +54,19 @@ enum : int32_t { kFlagFirst = 1, kFlagLast = 2 };
 struct __align__(16) StageHeader {
     int32_t kind, flags, adapter, rank;
     float scale;
-    int32_t L, off, len;        // tokens; first column (shrink: of h, expand: row of o) and extent
+    int32_t L, off, len;   // tokens; first column of h (shrink) or row of o (expand); extent
     int32_t tok[kTokChunk];
 };
 static_assert(sizeof(StageHeader) <= kHeaderBytes, "header");
 
 struct __align__(8) SmemCtl {
-    uint64_t full[kMaxStages];
-    uint64_t empty[kMaxStages];
-    uint64_t vready[2];
-    uint64_t vfree[2];
+    uint64_t full[kMaxStages];    // TMA data landed (tx bytes) + producer arrival
+    uint64_t meta[kMaxStages];    // header written (producer arrival)
+    uint64_t empty[kMaxStages];   // consumer warps released the stage
+    uint64_t recv;                // peers' partials landed (tx bytes) + own arrival
+    uint64_t freed;               // every peer finished reading its partials of the last unit
     int32_t n_groups;
-    int32_t pending[kTokChunk];  // producer's token list while grouping ids
+    int32_t pending[kTokChunk];   // producer's token list while grouping ids
 };
 constexpr int kCtlBytes = 256;
 static_assert(sizeof(SmemCtl) <= kCtlBytes, "ctl");
@@ -74,33 +82,37 @@ template <> struct Tr<float> {
 __host__ __device__ constexpr int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
 struct Layout {
-    int ids_off, v_off, stage_off, RP, total;
+    int ids_off, xs_off, ys_off, vpart_off, recv_off, vsum_off, stage_off, RP, total;
 };
+
+__host__ __device__ inline int row_bytes_for(int R) { return R > 64 ? kRowBytes / 2 : kRowBytes; }
 
 __host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int stages, int stage_bytes)
 {
     Layout l;
+    const int rowb = row_bytes_for(R);
     l.RP = round_up(R, 8);
     l.ids_off = kCtlBytes;
     const int ids_bytes = (src == kSrcIds) ? round_up(4 * (2 * T + n), 128) : 0;
-    l.v_off = l.ids_off + ids_bytes;
-    const int v_bytes = round_up(3 * kTokChunk * l.RP * 4, 128);   // vpart[2] + vfull
-    l.stage_off = l.v_off + v_bytes;
+    l.xs_off = l.ids_off + ids_bytes;
+    l.ys_off = l.xs_off + kTokChunk * rowb;
+    l.vpart_off = l.ys_off + kTokChunk * rowb;
+    l.recv_off = l.vpart_off + round_up(kTokChunk * l.RP * 4, 128);
+    l.vsum_off = l.recv_off + kCluster * kTokChunk * l.RP * 4;
+    l.stage_off = l.vsum_off + round_up(kTokChunk * l.RP * 4, 128);
     l.total = l.stage_off + stages * stage_bytes;
     return l;
 }
 
-// 16 staged bytes -> EPC floats
-__device__ __forceinline__ void load16(const uint8_t *p, float *o, __nv_bfloat16 *)
+__device__ __forceinline__ void cvt16(const uint4 w, float *o, __nv_bfloat16 *)
 {
-    const uint4 w = *reinterpret_cast<const uint4 *>(p);
     o[0] = bf16_lo(w.x); o[1] = bf16_hi(w.x); o[2] = bf16_lo(w.y); o[3] = bf16_hi(w.y);
     o[4] = bf16_lo(w.z); o[5] = bf16_hi(w.z); o[6] = bf16_lo(w.w); o[7] = bf16_hi(w.w);
 }
-__device__ __forceinline__ void load16(const uint8_t *p, float *o, float *)
+__device__ __forceinline__ void cvt16(const uint4 w, float *o, float *)
 {
-    const float4 w = *reinterpret_cast<const float4 *>(p);
-    o[0] = w.x; o[1] = w.y; o[2] = w.z; o[3] = w.w;
+    o[0] = __uint_as_float(w.x); o[1] = __uint_as_float(w.y);
+    o[2] = __uint_as_float(w.z); o[3] = __uint_as_float(w.w);
 }
 
 // Sum 8 per-lane values over the 32 lanes of a warp.  On return lane L holds the total of
@@ -137,20 +149,82 @@ __device__ __forceinline__ float warp_reduce8(float (&a)[8], int lane)
     return r;
 }
 
+// Partial shrink of one staged tile by one warp.  The warp owns rank rows k = warp + 8*i; it
+// takes RB of them at a time against TG = 8 / RB tokens, so every butterfly folds 8 values.
+// A is staged as [box][row][512 B] (box 1 starts after r rows of box 0), x as [token][1 KiB];
+// a lane reads 16-byte chunks `lane` (box 0) and `lane + 32` (box 1).  Operands are read from
+// shared memory at the point of use (nothing held across tokens), which keeps registers low.
+template <typename E, int RB>
+__device__ __forceinline__ void shrink_rows(const uint8_t *A, const uint8_t *xs, int rowb, float *vpart, int RP,
+                                            int r, int L, int nch, int warp, int lane, bool first)
+{
+    constexpr int EPC = Tr<E>::EPC;
+    constexpr int TG = 8 / RB;
+    const bool okA = lane < nch, okB = lane + 32 < nch;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    const int nrows = (r > warp) ? (r - warp + 7) / 8 : 0;
+    for (int rb0 = 0; rb0 < nrows; rb0 += RB) {
+        for (int t0 = 0; t0 < L; t0 += TG) {
+            float acc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+            for (int tt = 0; tt < TG; ++tt) {
+                if (t0 + tt < L) {
+                    const uint8_t *xr = xs + (t0 + tt) * rowb;
+                    const uint4 x0 = okA ? *reinterpret_cast<const uint4 *>(xr + lane * 16) : z;
+                    const uint4 x1 = okB ? *reinterpret_cast<const uint4 *>(xr + 512 + lane * 16) : z;
+                    float xv[2][EPC];
+                    cvt16(x0, xv[0], (E *)nullptr);
+                    cvt16(x1, xv[1], (E *)nullptr);
+#pragma unroll
+                    for (int i = 0; i < RB; ++i) {
+                        if (rb0 + i < nrows) {
+                            const uint8_t *row = A + (warp + 8 * (rb0 + i)) * kBoxBytes;
+                            float av[EPC];
+                            float sum = 0.f;
+                            cvt16(okA ? *reinterpret_cast<const uint4 *>(row + lane * 16) : z, av, (E *)nullptr);
+#pragma unroll
+                            for (int e = 0; e < EPC; ++e) sum = fmaf(xv[0][e], av[e], sum);
+                            cvt16(okB ? *reinterpret_cast<const uint4 *>(row + r * kBoxBytes + lane * 16) : z, av,
+                                  (E *)nullptr);
+#pragma unroll
+                            for (int e = 0; e < EPC; ++e) sum = fmaf(xv[1][e], av[e], sum);
+                            acc[tt * RB + i] = sum;
+                        }
+                    }
+                }
+            }
+            const float tot = warp_reduce8(acc, lane);
+            const int vi = (lane >> 2) & 7;
+            const int l = t0 + vi / RB, i = vi % RB;
+            const int k = warp + 8 * (rb0 + i);
+            if ((lane & 3) == 0 && l < L && rb0 + i < nrows) {
+                float *dst = vpart + l * RP + k;
+                *dst = first ? tot : *dst + tot;
+            }
+        }
+    }
+}
+
 template <typename E, int MODE, int SRC>
-__global__ void __launch_bounds__(kThreads, 1)
-lora_decode_kernel(const __grid_constant__ DecodeParams p)
+__global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_constant__ DecodeParams p)
 {
     using T_ = Tr<E>;
     constexpr int ESZ = T_::ESZ, EPC = T_::EPC, CPT = T_::CPT;
-    constexpr int W = kRowBytes / ESZ;          // elements of one staged row
-    constexpr int CHUNKS = kRowBytes / 16;      // 16-byte chunks per staged row
+    constexpr int BOXW = kBoxBytes / ESZ;       // elements of one TMA box row
+    const int rowb = row_bytes_for(p.R);        // bytes of one staged row
+    const int W = rowb / ESZ;                   // elements of one h-subtile / rows of one o-subtile
+    const int CHUNKS = rowb / 16;               // 16-byte chunks per h-subtile row
 
     extern __shared__ __align__(128) uint8_t smem[];
     SmemCtl &ctl = *reinterpret_cast<SmemCtl *>(smem);
     const Layout lay = make_layout(SRC, p.R, p.n, p.T, p.stages, p.stage_bytes);
-    float *vpart = reinterpret_cast<float *>(smem + lay.v_off);            // [2][kTokChunk][RP]
-    float *vfull = vpart + 2 * kTokChunk * lay.RP;                          // [kTokChunk][RP]
+    uint8_t *xs = smem + lay.xs_off;
+    uint8_t *ys = smem + lay.ys_off;
+    float *vpart = reinterpret_cast<float *>(smem + lay.vpart_off);   // [kTokChunk][RP] this CTA's partial
+    float *recv = reinterpret_cast<float *>(smem + lay.recv_off);     // [kCluster][kTokChunk][RP] from peers
+    float *vsum = reinterpret_cast<float *>(smem + lay.vsum_off);     // [kTokChunk][RP] the unit's intermediate
     uint8_t *stage_base = smem + lay.stage_off;
     const int RP = lay.RP;
     const int S = p.stages;
@@ -159,26 +233,28 @@ lora_decode_kernel(const __grid_constant__ DecodeParams p)
     const uint32_t crank = cluster_ctarank();
     const int cid = (int)cluster_id_x(), G = (int)nclusters_x();
 
+    if (tid == 0) LORA_TRACE_MARK(0);
     pdl_wait();
     pdl_launch_dependents();
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&ctl.full[s]), 1);
+            mbar_init(smem_u32(&ctl.meta[s]), 1);
             mbar_init(smem_u32(&ctl.empty[s]), kConsumerWarps);
         }
-        for (int q = 0; q < 2; ++q) {
-            mbar_init(smem_u32(&ctl.vready[q]), kCluster);
-            mbar_init(smem_u32(&ctl.vfree[q]), kCluster);
-        }
+        mbar_init(smem_u32(&ctl.recv), 1);
+        mbar_init(smem_u32(&ctl.freed), kCluster);
         fence_mbar_init_cluster();
     }
 
-    // Per-token ids: group equal ids on the device.  A group is led by the first token that
-    // carries its id; groups are listed in the order of their leaders.
+    // Per-token ids: tokens with equal ids form one group.  When there are no more adapters
+    // than clusters, cluster c simply owns adapter c; otherwise a group is led by the first
+    // token carrying its id and groups are listed in the order of their leaders.
     int32_t *ids_s = reinterpret_cast<int32_t *>(smem + lay.ids_off);
     int32_t *first = ids_s + p.T;
     int32_t *leaders = first + p.n;
+    const bool direct_ids = (SRC == kSrcIds) && p.n <= G;
     if (SRC == kSrcIds) {
         bool bad = false;
         for (int t = tid; t < p.T; t += kThreads) {
@@ -186,27 +262,31 @@ lora_decode_kernel(const __grid_constant__ DecodeParams p)
             ids_s[t] = a;
             bad |= (a < -1 || a >= p.n);
         }
-        for (int i = tid; i < p.n; i += kThreads) first[i] = INT_MAX;
-        if (__syncthreads_or(bad) && tid == 0 && crank == 0) atomicOr(p.status, LORA_STATUS_BAD_ID);
-        for (int t = tid; t < p.T; t += kThreads) {
-            const int32_t a = ids_s[t];
-            if (a >= 0 && a < p.n) atomicMin(&first[a], t);
-        }
-        __syncthreads();
-        if (warp == 0) {
-            int cnt = 0;
-            for (int base = 0; base < p.T; base += 32) {
-                const int t = base + lane;
-                const int32_t a = t < p.T ? ids_s[t] : -1;
-                const bool lead = a >= 0 && a < p.n && first[a] == t;
-                const uint32_t m = __ballot_sync(0xffffffffu, lead);
-                if (lead) leaders[cnt + __popc(m & ((1u << lane) - 1u))] = t;
-                cnt += __popc(m);
+        if (!direct_ids)
+            for (int i = tid; i < p.n; i += kThreads) first[i] = INT_MAX;
+        if (__syncthreads_or(bad) && tid == 0 && crank == 0 && cid == 0) atomicOr(p.status, LORA_STATUS_BAD_ID);
+        if (!direct_ids) {
+            for (int t = tid; t < p.T; t += kThreads) {
+                const int32_t a = ids_s[t];
+                if (a >= 0 && a < p.n) atomicMin(&first[a], t);
             }
-            if (lane == 0) ctl.n_groups = cnt;
+            __syncthreads();
+            if (warp == 0) {
+                int cnt = 0;
+                for (int base = 0; base < p.T; base += 32) {
+                    const int t = base + lane;
+                    const int32_t a = t < p.T ? ids_s[t] : -1;
+                    const bool lead = a >= 0 && a < p.n && first[a] == t;
+                    const uint32_t m = __ballot_sync(0xffffffffu, lead);
+                    if (lead) leaders[cnt + __popc(m & ((1u << lane) - 1u))] = t;
+                    cnt += __popc(m);
+                }
+                if (lane == 0) ctl.n_groups = cnt;
+            }
         }
     }
     cluster_sync_all();   // barrier inits visible cluster-wide; group list ready
+    if (tid == 0) LORA_TRACE_MARK(1);
 
     // h and o ranges of this CTA, in 16-byte chunks of h and EPC-row groups of o
     const int hchunks = p.h / EPC, ogroups = p.o / EPC;
@@ -222,44 +302,38 @@ lora_decode_kernel(const __grid_constant__ DecodeParams p)
         // ================================ producer warp ================================
         int issued = 0;
         bool alive = true;
-        auto next_stage = [&](StageHeader *&hdr, uint8_t *&data, uint32_t &full_bar) -> bool {
-            const int s = issued % S;
-            const int m = issued / S;
-            if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) return false;
-            hdr = reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
-            data = stage_base + (size_t)s * p.stage_bytes + kHeaderBytes;
-            full_bar = smem_u32(&ctl.full[s]);
-            return true;
-        };
-        // Issue every tile of one unit: adapter a, tokens tok[0, L) (valid in lane l < L).
+        // Issue every tile of one unit: adapter a, tokens held by lanes 0..L-1 (my_tok).
         auto emit_unit = [&](int a, int my_tok, int L) {
             const AdapterDesc d = p.desc[a];
             const int r = d.rank;
-            const uint8_t *Ab = static_cast<const uint8_t *>(d.A);
+            const char *tmapA = reinterpret_cast<const char *>(p.tmA) + (size_t)a * 128;
             const uint8_t *Bb = static_cast<const uint8_t *>(d.B);
+            if (lane == 0) LORA_TRACE_MARK(2);
             const int ntiles = n_shrink + n_expand;
             for (int j = 0; j < ntiles && alive; ++j) {
-                StageHeader *hdr;
-                uint8_t *data;
-                uint32_t fb;
-                if (!next_stage(hdr, data, fb)) {
+                const int s = issued % S, m = issued / S;
+                if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
                     alive = false;
                     break;
                 }
+                StageHeader *hdr = reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
+                const uint32_t data = smem_u32(stage_base + (size_t)s * p.stage_bytes + kHeaderBytes);
+                const uint32_t fb = smem_u32(&ctl.full[s]);
                 const bool shrink = j < n_shrink;
-                int off, len;
+                int off, len, nbox = 0;
                 uint32_t bytes;
                 if (shrink) {
                     const int c0 = hc0 + j * CHUNKS;
                     const int c1 = min(hc1, c0 + CHUNKS);
                     off = c0 * EPC;
                     len = max(0, c1 - c0) * EPC;
-                    bytes = (uint32_t)((r + L) * len * ESZ);
+                    nbox = (len + BOXW - 1) / BOXW;
+                    bytes = (uint32_t)(nbox * r * kBoxBytes);
                 } else {
                     const int jj = j - n_shrink;
                     off = og0 * EPC + jj * W;
                     len = min(W, orows - jj * W);
-                    bytes = (uint32_t)(len * r * ESZ + L * len * ESZ);
+                    bytes = (uint32_t)(len * r * ESZ);
                 }
                 if (lane < L) hdr->tok[lane] = my_tok;
                 if (lane == 0) {
@@ -275,36 +349,27 @@ lora_decode_kernel(const __grid_constant__ DecodeParams p)
                     hdr->len = len;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive_expect_tx(fb, bytes);
-                __syncwarp();
-                if (len > 0) {
-                    const uint32_t dst = smem_u32(data);
+                if (lane == 0) {
+                    mbar_arrive(smem_u32(&ctl.meta[s]));
+                    mbar_arrive_expect_tx(fb, bytes);
                     if (shrink) {
-                        // r rows of A_i, then L rows of x, each len elements from column `off`
-                        for (int c = lane; c < r; c += 32)
-                            bulk_g2s(dst + c * kRowBytes, Ab + ((int64_t)c * p.h + off) * ESZ, len * ESZ, fb);
-                        // x rows (token of row l lives in lane l)
-                        for (int l = 0; l < L; ++l) {
-                            const int t = __shfl_sync(0xffffffffu, my_tok, l);
-                            if (lane == (l & 31))
-                                bulk_g2s(dst + (r + l) * kRowBytes,
-                                         static_cast<const uint8_t *>(p.x) + ((int64_t)t * p.ldx + off) * ESZ,
-                                         len * ESZ, fb);
-                        }
-                    } else {
-                        const int yoff = round_up(len * r * ESZ, 128);
-                        if (lane == 0) bulk_g2s(dst, Bb + (int64_t)off * r * ESZ, len * r * ESZ, fb);
-                        for (int l = 0; l < L; ++l) {
-                            const int t = __shfl_sync(0xffffffffu, my_tok, l);
-                            if (lane == ((l + 1) & 31))
-                                bulk_g2s(dst + yoff + l * kRowBytes,
-                                         static_cast<uint8_t *>(p.y) +
-                                             ((int64_t)t * p.ldy + p.y_off + off) * ESZ,
-                                         len * ESZ, fb);
-                        }
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d(data + b * r * kBoxBytes, tmapA, off + b * BOXW, 0, fb);
+                    } else if (len > 0) {
+                        bulk_g2s(data, Bb + (int64_t)off * r * ESZ, len * r * ESZ, fb);
                     }
                 }
+                // L2 hints for the rows the consumers load for this tile
+                const int lines = (len * ESZ + 127) / 128;
+                for (int l = 0; l < L; ++l) {
+                    const int t = __shfl_sync(0xffffffffu, my_tok, l);
+                    const uint8_t *row =
+                        shrink ? static_cast<const uint8_t *>(p.x) + ((int64_t)t * p.ldx + off) * ESZ
+                               : static_cast<const uint8_t *>(p.y) + ((int64_t)t * p.ldy + p.y_off + off) * ESZ;
+                    for (int c = lane; c < lines; c += 32) prefetch_l2(row + c * 128);
+                }
                 ++issued;
+                if (lane == 0) LORA_TRACE_MARK(shrink ? 3 : 4);
             }
         };
 
@@ -325,23 +390,21 @@ lora_decode_kernel(const __grid_constant__ DecodeParams p)
                     const uint32_t m = __ballot_sync(0xffffffffu, ok);
                     if (m != __ballot_sync(0xffffffffu, lane < L0) && lane == 0 && crank == 0)
                         atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
-                    // compact valid tokens to lanes 0..popc(m)-1
-                    const int dst_lane = __popc(m & ((1u << lane) - 1u));
+                    // compact the valid tokens to lanes 0 .. popc(m) - 1, order kept
                     int my_tok = 0;
                     for (int l = 0; l < L0; ++l) {
                         const int tl = __shfl_sync(0xffffffffu, t, l);
-                        const int dl = __shfl_sync(0xffffffffu, dst_lane, l);
-                        if (((m >> l) & 1u) && lane == dl) my_tok = tl;
+                        if (((m >> l) & 1u) && lane == __popc(m & ((1u << l) - 1u))) my_tok = tl;
                     }
                     const int L = __popc(m);
                     if (L > 0) emit_unit(a, my_tok, L);
                 }
             }
         } else {
-            const int ng = ctl.n_groups;
+            const int ng = direct_ids ? p.n : ctl.n_groups;
             for (int g = cid; g < ng && alive; g += G) {
-                const int t0 = leaders[g];
-                const int a = ids_s[t0];
+                const int t0 = direct_ids ? 0 : leaders[g];
+                const int a = direct_ids ? g : ids_s[t0];
                 int cnt = 0;
                 for (int base = t0; base < p.T && alive; base += 32) {
                     const int t = base + lane;
@@ -371,188 +434,178 @@ lora_decode_kernel(const __grid_constant__ DecodeParams p)
         }
         // end marker
         if (alive) {
-            StageHeader *hdr;
-            uint8_t *data;
-            uint32_t fb;
-            if (next_stage(hdr, data, fb)) {
+            const int s = issued % S, m = issued / S;
+            if (m < 1 || mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
                 if (lane == 0) {
-                    hdr->kind = kTileEnd;
-                    mbar_arrive(fb);
+                    reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes)->kind = kTileEnd;
+                    mbar_arrive(smem_u32(&ctl.meta[s]));
+                    mbar_arrive(smem_u32(&ctl.full[s]));
                 }
                 ++issued;
             }
         }
-        // drain: no bulk copy may still be writing into this CTA's shared memory at exit
+        // drain: no copy may still be writing into this CTA's shared memory at exit
         for (int i = max(0, issued - S); i < issued; ++i)
             mbar_wait(smem_u32(&ctl.full[i % S]), (i / S) & 1, p.status);
         return;
     }
 
     // =================================== consumers ===================================
-    int u = 0;   // units whose intermediate has been reduced (fused / shrink modes)
+    int u = 0;   // units whose intermediate has been exchanged (fused / shrink modes)
     for (int it = 0;; ++it) {
         const int s = it % S;
-        if (!mbar_wait(smem_u32(&ctl.full[s]), (it / S) & 1, p.status)) break;
+        const uint32_t ph = (it / S) & 1;
+        if (!mbar_wait(smem_u32(&ctl.meta[s]), ph, p.status)) break;
         const StageHeader &hdr = *reinterpret_cast<const StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
-        const uint8_t *data = stage_base + (size_t)s * p.stage_bytes + kHeaderBytes;
         const int kind = hdr.kind;
         if (kind == kTileEnd) break;
         const int r = hdr.rank, L = hdr.L, flags = hdr.flags, len = hdr.len, off = hdr.off;
-        bool ok = true;
+        const uint8_t *data = stage_base + (size_t)s * p.stage_bytes + kHeaderBytes;
+        const int nch = len / EPC;   // 16-byte chunks per staged row
+
+        // Load this tile's x rows (shrink) or y rows (expand) while the TMA lands: row l,
+        // 16-byte chunk c, four chunks per thread at most (16 rows x 1 KiB).
+        uint4 ld[4];
+        const int total = L * nch;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + kConsumers * i;
+            ld[i] = make_uint4(0, 0, 0, 0);
+            if (e < total) {
+                const int l = e / nch, c = e - l * nch;
+                const int64_t t = hdr.tok[l];
+                const uint8_t *src =
+                    (kind == kTileShrink)
+                        ? static_cast<const uint8_t *>(p.x) + (t * p.ldx + off) * ESZ + c * 16
+                        : static_cast<const uint8_t *>(p.y) + (t * p.ldy + p.y_off + off) * ESZ + c * 16;
+                ld[i] = *reinterpret_cast<const uint4 *>(src);
+            }
+        }
+        named_bar_sync(1, kConsumers);   // every consumer is done with the previous tile's buffers
+        uint8_t *stg = (kind == kTileShrink) ? xs : ys;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + kConsumers * i;
+            if (e < total) {
+                const int l = e / nch, c = e - l * nch;
+                *reinterpret_cast<uint4 *>(stg + l * rowb + c * 16) = ld[i];
+            }
+        }
+        if (!mbar_wait(smem_u32(&ctl.full[s]), ph, p.status)) break;
+        if (tid == 0) LORA_TRACE_MARK(8 + (it < 3 ? it : 3));
+        named_bar_sync(1, kConsumers);
 
         if (kind == kTileShrink) {
-            const int q = u & 1;
-            float *vp = vpart + q * kTokChunk * RP;
-            if ((flags & kFlagFirst) && u >= 2)
-                ok = mbar_wait_cluster(smem_u32(&ctl.vfree[q]), ((u >> 1) - 1) & 1, p.status);
-            if (!ok) break;
-            // ---- partial shrink over this CTA's slice of h: P[l][k] = sum_j X[l][j] A[k][j]
-            const int nchunks = len / EPC;
-            const int cA = lane, cB = lane + 32;
-            const int nkg = (r + 7) >> 3;
-            for (int slot = warp; slot < L * nkg; slot += kConsumerWarps) {
-                const int l = slot / nkg, kg = slot - l * nkg;
-                float xv[2 * EPC];
-                const uint8_t *xr = data + (r + l) * kRowBytes;
-                if (cA < nchunks) load16(xr + cA * 16, xv, (E *)nullptr);
-                else for (int e = 0; e < EPC; ++e) xv[e] = 0.f;
-                if (cB < nchunks) load16(xr + cB * 16, xv + EPC, (E *)nullptr);
-                else for (int e = 0; e < EPC; ++e) xv[EPC + e] = 0.f;
-                float acc[8];
-#pragma unroll
-                for (int qq = 0; qq < 8; ++qq) {
-                    acc[qq] = 0.f;
-                    const int k = kg * 8 + qq;
-                    if (k < r) {
-                        const uint8_t *ar = data + k * kRowBytes;
-                        float av[EPC];
-                        if (cA < nchunks) {
-                            load16(ar + cA * 16, av, (E *)nullptr);
-#pragma unroll
-                            for (int e = 0; e < EPC; ++e) acc[qq] = fmaf(xv[e], av[e], acc[qq]);
-                        }
-                        if (cB < nchunks) {
-                            load16(ar + cB * 16, av, (E *)nullptr);
-#pragma unroll
-                            for (int e = 0; e < EPC; ++e) acc[qq] = fmaf(xv[EPC + e], av[e], acc[qq]);
-                        }
-                    }
-                }
-                const float tot = warp_reduce8(acc, lane);
-                const int k = kg * 8 + ((lane >> 2) & 7);
-                if ((lane & 3) == 0 && k < r) {
-                    float *dst = vp + l * RP + k;
-                    *dst = (flags & kFlagFirst) ? tot : *dst + tot;
-                }
+            const bool first = flags & kFlagFirst;
+            // ---- partial shrink over this CTA's slice of h
+            if (warp < min(r, 8)) {
+                const int rw = (r - warp + 7) / 8;   // rows of this warp
+                if (rw >= 8) shrink_rows<E, 8>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
+                else if (rw >= 4) shrink_rows<E, 4>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
+                else if (rw >= 2) shrink_rows<E, 2>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
+                else shrink_rows<E, 1>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
             }
             if (flags & kFlagLast) {
-                // ---- sum the cluster's partials in CTA order 0..7 through distributed smem
+                if (tid == 0) LORA_TRACE_MARK(12);
                 named_bar_sync(1, kConsumers);
-                if (tid == 0)
-                    for (int j = 0; j < kCluster; ++j) mbar_arrive_remote(smem_u32(&ctl.vready[q]), j);
-                ok = mbar_wait_cluster(smem_u32(&ctl.vready[q]), (u >> 1) & 1, p.status);
-                if (!ok) break;
-                const uint32_t vp_addr = smem_u32(vp);
+                // ---- push the partial into every CTA of the cluster (this one included)
+                if (u >= 1 && !mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status)) break;
+                const int nq = L * RP / 4;
+                const uint32_t my_slot = smem_u32(recv + crank * kTokChunk * RP);
+                const uint32_t rbar = smem_u32(&ctl.recv);
+                for (int e = tid; e < nq * kCluster; e += kConsumers) {
+                    const int peer = e / nq, q = e - peer * nq;
+                    const float4 v = *reinterpret_cast<const float4 *>(vpart + q * 4);
+                    st_async_v4(my_slot + q * 16, rbar, peer, v);
+                }
+                if (tid == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(kCluster * nq * 16));
+                if (!mbar_wait_cluster(rbar, u & 1, p.status)) break;
+                if (tid == 0) LORA_TRACE_MARK(13);
+                // ---- sum the 8 partials in CTA order
                 for (int e = tid; e < L * RP; e += kConsumers) {
-                    const int l = e / RP, k = e - l * RP;
+                    const int k = e % RP;
                     float acc = 0.f;
-                    if (k < r)
-                        for (int j = 0; j < kCluster; ++j) acc += ld_dsmem_f32(vp_addr + 4u * (l * RP + k), j);
-                    vfull[e] = acc;
+                    if (k < r) {
+#pragma unroll
+                        for (int j = 0; j < kCluster; ++j) acc += recv[j * kTokChunk * RP + e];
+                    }
+                    vsum[e] = acc;
                 }
                 named_bar_sync(1, kConsumers);
-                if (tid == 0)
-                    for (int j = 0; j < kCluster; ++j) mbar_arrive_remote(smem_u32(&ctl.vfree[q]), j);
+                if (tid < kCluster) mbar_arrive_remote(smem_u32(&ctl.freed), tid);
+                if (tid == 0) LORA_TRACE_MARK(14);
                 if (MODE == kModeShrink && crank == 0) {
                     for (int e = tid; e < L * r; e += kConsumers) {
                         const int l = e / r, k = e - l * r;
-                        p.v[(int64_t)hdr.tok[l] * p.ldv + k] = vfull[l * RP + k];
+                        p.v[(int64_t)hdr.tok[l] * p.ldv + k] = vsum[l * RP + k];
                     }
                 }
                 ++u;
             }
         } else {  // kTileExpand
             if (MODE == kModeExpand && (flags & kFlagFirst)) {
-                named_bar_sync(1, kConsumers);
                 for (int e = tid; e < L * RP; e += kConsumers) {
                     const int l = e / RP, k = e - l * RP;
-                    vfull[e] = (k < r) ? p.v[(int64_t)hdr.tok[l] * p.ldv + k] : 0.f;
+                    vsum[e] = (k < r) ? p.v[(int64_t)hdr.tok[l] * p.ldv + k] : 0.f;
                 }
                 named_bar_sync(1, kConsumers);
             }
+            const float sc = hdr.scale;
             const int c = tid * CPT;   // first column of this thread within the tile
             if (c < len) {
-                const int yoff = round_up(len * r * ESZ, 128);
-                float acc[kTokChunk][CPT];
+                const uint8_t *brow = data + (size_t)c * r * ESZ;   // CPT consecutive rows of B
+                for (int l = 0; l < L; ++l) {
+                    const float *vr = vsum + l * RP;
+                    float acc[CPT];
 #pragma unroll
-                for (int l = 0; l < kTokChunk; ++l)
+                    for (int j = 0; j < CPT; ++j) acc[j] = 0.f;
+                    if ((r % EPC) == 0) {
+                        for (int k = 0; k < r; k += EPC) {
+                            float vv[EPC];
 #pragma unroll
-                    for (int j = 0; j < CPT; ++j) acc[l][j] = 0.f;
-                if ((r % EPC) == 0) {
-                    for (int k = 0; k < r; k += EPC) {
-                        float b[CPT][EPC];
+                            for (int e = 0; e < EPC; e += 4) {
+                                const float4 t4 = *reinterpret_cast<const float4 *>(vr + k + e);
+                                vv[e] = t4.x; vv[e + 1] = t4.y; vv[e + 2] = t4.z; vv[e + 3] = t4.w;
+                            }
 #pragma unroll
-                        for (int j = 0; j < CPT; ++j) load16(data + ((c + j) * r + k) * ESZ, b[j], (E *)nullptr);
+                            for (int j = 0; j < CPT; ++j) {
+                                float b[EPC];
+                                cvt16(*reinterpret_cast<const uint4 *>(brow + ((size_t)j * r + k) * ESZ), b,
+                                      (E *)nullptr);
 #pragma unroll
-                        for (int l = 0; l < kTokChunk; ++l) {
-                            if (l < L) {
-                                const float *vr = vfull + l * RP + k;
-                                float vv[EPC];
-#pragma unroll
-                                for (int e = 0; e < EPC; e += 4) {
-                                    const float4 t4 = *reinterpret_cast<const float4 *>(vr + e);
-                                    vv[e] = t4.x; vv[e + 1] = t4.y; vv[e + 2] = t4.z; vv[e + 3] = t4.w;
-                                }
-#pragma unroll
-                                for (int j = 0; j < CPT; ++j)
-#pragma unroll
-                                    for (int e = 0; e < EPC; ++e) acc[l][j] = fmaf(vv[e], b[j][e], acc[l][j]);
+                                for (int e = 0; e < EPC; ++e) acc[j] = fmaf(vv[e], b[e], acc[j]);
                             }
                         }
-                    }
-                } else {
-                    for (int k = 0; k < r; ++k) {
-                        float b[CPT];
+                    } else {
+                        for (int k = 0; k < r; ++k) {
 #pragma unroll
-                        for (int j = 0; j < CPT; ++j) {
-                            const E *bp = reinterpret_cast<const E *>(data) + (c + j) * r + k;
-                            b[j] = (float)(*bp);
+                            for (int j = 0; j < CPT; ++j)
+                                acc[j] = fmaf(vr[k], (float)reinterpret_cast<const E *>(brow)[j * r + k], acc[j]);
                         }
-#pragma unroll
-                        for (int l = 0; l < kTokChunk; ++l)
-                            if (l < L)
-#pragma unroll
-                                for (int j = 0; j < CPT; ++j) acc[l][j] = fmaf(vfull[l * RP + k], b[j], acc[l][j]);
                     }
-                }
-                const float sc = hdr.scale;
-#pragma unroll
-                for (int l = 0; l < kTokChunk; ++l) {
-                    if (l < L) {
-                        const uint8_t *yr = data + yoff + l * kRowBytes + c * ESZ;
-                        const int64_t gofs = (int64_t)hdr.tok[l] * p.ldy + p.y_off + off + c;
-                        if constexpr (CPT == 2) {
-                            const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
-                            const float y0 = fmaf(sc, acc[l][0], bf16_lo(w));
-                            const float y1 = fmaf(sc, acc[l][1], bf16_hi(w));
-                            *reinterpret_cast<uint32_t *>(static_cast<E *>(p.y) + gofs) = pack_bf16x2(y0, y1);
-                        } else {
-                            const float w = *reinterpret_cast<const float *>(yr);
-                            static_cast<float *>(p.y)[gofs] = fmaf(sc, acc[l][0], w);
-                        }
+                    const uint8_t *yr = ys + l * rowb + c * ESZ;
+                    const int64_t gofs = (int64_t)hdr.tok[l] * p.ldy + p.y_off + off + c;
+                    if constexpr (CPT == 2) {
+                        const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
+                        const float y0 = fmaf(sc, acc[0], bf16_lo(w));
+                        const float y1 = fmaf(sc, acc[1], bf16_hi(w));
+                        *reinterpret_cast<uint32_t *>(static_cast<E *>(p.y) + gofs) = pack_bf16x2(y0, y1);
+                    } else {
+                        const float w = *reinterpret_cast<const float *>(yr);
+                        static_cast<float *>(p.y)[gofs] = fmaf(sc, acc[0], w);
                     }
                 }
             }
         }
+        if (tid == 0) LORA_TRACE_MARK(kind == kTileShrink ? 15 : 16);
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
     }
-    // No CTA of the cluster may leave while a peer can still read its partials or arrive on
-    // its barriers: wait for the last release of each intermediate slot.
-    if (MODE != kModeExpand) {
-        if (u >= 1) mbar_wait_cluster(smem_u32(&ctl.vfree[(u - 1) & 1]), ((u - 1) >> 1) & 1, p.status);
-        if (u >= 2) mbar_wait_cluster(smem_u32(&ctl.vfree[(u - 2) & 1]), ((u - 2) >> 1) & 1, p.status);
-    }
+    if (tid == 0) LORA_TRACE_MARK(17);
+    // No CTA may leave while a peer can still arrive on its barriers: wait until every peer
+    // has released the partials of the last unit.
+    if (MODE != kModeExpand && u >= 1) mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status);
+    if (tid == 0) LORA_TRACE_MARK(18);
 }
 
 template <typename E, int MODE, int SRC>
@@ -563,25 +616,25 @@ int launch_one(const DecodeParams &p0, cudaStream_t s)
     const Options &opt = options();
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LORA_ERR_CUDA;
+    if (dev >= 64) return LORA_ERR_UNSUPPORTED;
     static std::once_flag once[64];
     static int max_optin[64];
     static int n_sms[64];
-    if (dev >= 64) return LORA_ERR_UNSUPPORTED;
     std::call_once(once[dev], [&] {
         cudaDeviceGetAttribute(&max_optin[dev], cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         cudaDeviceGetAttribute(&n_sms[dev], cudaDevAttrMultiProcessorCount, dev);
     });
     // Pipeline depth: aim for two CTAs per SM unless told otherwise.
-    const int stage_bytes = kHeaderBytes + (p.R + kTokChunk) * kRowBytes;
+    const int stage_bytes = kHeaderBytes + p.R * row_bytes_for(p.R);
     const int fixed = make_layout(SRC, p.R, p.n, p.T, 0, stage_bytes).total;
-    int ctas_per_sm = opt.decode_ctas_per_sm > 0 ? (int)opt.decode_ctas_per_sm : 2;
+    const int ctas_per_sm = opt.decode_ctas_per_sm > 0 ? (int)opt.decode_ctas_per_sm : 2;
     int stages = (int)opt.decode_stages;
     if (stages <= 0) {
         const int budget = (228 * 1024) / ctas_per_sm - 1024 - fixed;
-        stages = min(kMaxStages, budget / stage_bytes);
-        if (stages < 2) stages = 2;
+        stages = max(2, min(kMaxStages, budget / stage_bytes));
     }
-    stages = max(2, min(kMaxStages, stages));
+    stages = max(1, min(kMaxStages, stages));
+    while (stages > 1 && make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes).total > max_optin[dev]) --stages;
     const Layout lay = make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes);
     if (lay.total > max_optin[dev]) return LORA_ERR_UNSUPPORTED;
     p.stages = stages;
@@ -646,11 +699,51 @@ int launch_typed(int mode, int src, const DecodeParams &p, cudaStream_t s)
 
 int launch_decode(int mode, int src, const DecodeParams &p, int dtype, cudaStream_t s)
 {
+    if (!p.tmA) return LORA_ERR_INVALID_ARG;
     if (dtype == LORA_BF16) return launch_typed<__nv_bfloat16>(mode, src, p, s);
     if (dtype == LORA_F32) return launch_typed<float>(mode, src, p, s);
     return LORA_ERR_UNSUPPORTED;
 }
 
-size_t decode_ids_limit_bytes(int n, int T) { return (size_t)round_up(4 * (2 * T + n), 128); }
+// Tensor map of one adapter's A_i [rank, h] for the shrink: boxes of 512 bytes by `rank` rows,
+// no swizzle, zero fill past the end of h.
+int encode_tmap_A(void *out128, const void *A, int dtype, int h, int rank)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!encode) return LORA_ERR_CUDA;
+    const int esz = dtype == LORA_BF16 ? 2 : 4;
+    const cuuint64_t dims[2] = {(cuuint64_t)h, (cuuint64_t)rank};
+    const cuuint64_t strides[1] = {(cuuint64_t)h * esz};
+    const cuuint32_t box[2] = {(cuuint32_t)(kBoxBytes / esz), (cuuint32_t)rank};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult rc = encode(reinterpret_cast<CUtensorMap *>(out128),
+                               dtype == LORA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                               2, const_cast<void *>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return rc == CUDA_SUCCESS ? LORA_OK : LORA_ERR_UNSUPPORTED;
+}
 
 }  // namespace lora
+
+#ifdef LORA_TRACE
+// Instrumented builds only: copy the per-CTA phase marks to the host (n <= 4096 * 32 values).
+extern "C" int lora_trace_read(unsigned long long *host, int n)
+{
+    if (n > lora::kTraceCtas * lora::kTraceSlots) n = lora::kTraceCtas * lora::kTraceSlots;
+    return cudaMemcpyFromSymbol(host, lora::lora_trace_buf, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : -4;
+}
+extern "C" int lora_trace_clear(void)
+{
+    static unsigned long long zero[lora::kTraceCtas * lora::kTraceSlots];
+    return cudaMemcpyToSymbol(lora::lora_trace_buf, zero, sizeof zero) == cudaSuccess ? 0 : -4;
+}
+#endif

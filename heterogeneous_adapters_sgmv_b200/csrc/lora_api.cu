@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "lora_common.cuh"
 #include "lora_internal.h"
@@ -109,6 +110,7 @@ DecodeParams base_params(const lora_table *t)
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
     p.desc = t->d_desc;
+    p.tmA = t->d_tmaps;
     p.n = t->n;
     p.h = t->h;
     p.o = t->o;
@@ -179,10 +181,15 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int rc = LORA_OK;
-    if (cudaMalloc(&t->d_desc, sizeof(AdapterDesc) * n) != cudaSuccess ||
-        cudaMalloc(&t->d_status, 256) != cudaSuccess ||
-        cudaMemcpyAsync(t->d_desc, h_desc, sizeof(AdapterDesc) * n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemsetAsync(t->d_status, 0, 256, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    std::vector<uint8_t> h_tmaps((size_t)n * 128, 0);
+    for (int i = 0; i < n && rc == LORA_OK; ++i)
+        rc = encode_tmap_A(h_tmaps.data() + (size_t)i * 128, A[i], dtype, h, ranks[i]);
+    if (rc == LORA_OK &&
+        (cudaMalloc(&t->d_desc, sizeof(AdapterDesc) * n) != cudaSuccess ||
+         cudaMalloc(&t->d_tmaps, (size_t)n * 128) != cudaSuccess || cudaMalloc(&t->d_status, 256) != cudaSuccess ||
+         cudaMemcpyAsync(t->d_desc, h_desc, sizeof(AdapterDesc) * n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+         cudaMemcpyAsync(t->d_tmaps, h_tmaps.data(), (size_t)n * 128, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+         cudaMemsetAsync(t->d_status, 0, 256, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess))
         rc = LORA_ERR_CUDA;
     delete[] h_desc;
     if (rc != LORA_OK) {

@@ -146,6 +146,34 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
+
+// 2-D tiled TMA load (no multicast) of box {c0, c1} of `tmap` into this CTA's shared memory.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t c0, int32_t c1, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+// Hint: bring a 128-byte line into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Asynchronous store of 16 bytes into cluster CTA `rank`'s shared memory at the same offset as
+// `local_addr`; completion is counted in bytes on that CTA's mbarrier at offset `local_bar`.
+__device__ __forceinline__ void st_async_v4(uint32_t local_addr, uint32_t local_bar, uint32_t rank, float4 v)
+{
+    uint32_t ra, rb;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(local_bar), "r"(rank));
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(ra),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(rb)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------------------------------
 // cluster
 
@@ -176,12 +204,14 @@ __device__ __forceinline__ void cluster_sync_all()
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Loads from a peer CTA's shared memory.  No memory clobber: callers order them after the
+// acquiring wait that made the peer's data visible, and independent loads stay in flight together.
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank)
 {
     uint32_t remote;
     float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote));
     return v;
 }
 
@@ -192,8 +222,7 @@ __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_addr, uint32_t r
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
     asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(remote)
-                 : "memory");
+                 : "r"(remote));
     return v;
 }
 
@@ -211,5 +240,23 @@ __device__ __forceinline__ void pdl_launch_dependents()
 {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+
+// ---------------------------------------------------------------------------------------
+// optional phase tracing (compiled in only with -DLORA_TRACE): per-CTA clock64 marks
+
+#ifdef LORA_TRACE
+constexpr int kTraceCtas = 4096;
+constexpr int kTraceSlots = 32;
+// defined (once) by the translation unit that uses the marks
+#define LORA_TRACE_MARK(slot)                                                              \
+    do {                                                                                   \
+        if (blockIdx.x < (unsigned)::lora::kTraceCtas)                                     \
+            ::lora::lora_trace_buf[blockIdx.x * ::lora::kTraceSlots + (slot)] = clock64(); \
+    } while (0)
+#else
+#define LORA_TRACE_MARK(slot) \
+    do {                      \
+    } while (0)
+#endif
 
 }  // namespace lora

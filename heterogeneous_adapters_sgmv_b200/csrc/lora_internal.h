@@ -20,6 +20,7 @@ enum UnitSource : int { kSrcSegments = 0, kSrcIds = 1 };
 
 struct DecodeParams {
     const AdapterDesc *desc;
+    const void *tmA;       // device array of 128-byte tensor maps, one per adapter (A_i slices)
     int32_t n, h, o, R;    // adapters, in/out features, max rank of the table
     const void *x;
     int64_t ldx;
@@ -51,7 +52,8 @@ Options &options();
 int launch_decode(int mode, int src, const DecodeParams &p, int dtype, cudaStream_t s);
 int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *perm, int32_t *seg_ptr,
                           int32_t *seg_adapter, int32_t *num_segs, uint32_t *status, cudaStream_t s);
-size_t decode_smem_bytes(int src, int R, int n, int T, int stages, int *stage_bytes, int *ids_smem, int dtype);
+// Encode the TMA tensor map of A_i [rank, h] used by the decode shrink (host side).
+int encode_tmap_A(void *out128, const void *A, int dtype, int h, int rank);
 
 }  // namespace lora
 
@@ -63,6 +65,6 @@ struct lora_table {
     std::vector<const void *> A, B;
     std::vector<int32_t> ranks;
     std::vector<float> scales;
-    // tcgen05 prefill path: per-adapter tensor maps (device array), built on first use.
+    // per-adapter TMA tensor maps of A_i (device array of 128-byte CUtensorMap)
     void *d_tmaps;
 };
