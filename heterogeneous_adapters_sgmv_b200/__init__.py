@@ -31,11 +31,13 @@ LORA_STATUS_TIMEOUT = 2
 LORA_STATUS_BAD_SEGMENT = 4
 LORA_MAX_RANK = 128
 LORA_MAX_SEGMENT_TOKENS = 8192
+LORA_NOALLOC_SCRATCH_FLOATS = 262144
 
 EXPORTS = (
     "lora_table_create", "lora_table_destroy", "lora_table_info", "lora_workspace_bytes",
     "lora_build_segments", "lora_shrink", "lora_expand", "lora_sgmv", "lora_bgmv",
     "lora_get_status", "lora_status_string", "lora_set_option", "lora_get_option",
+    "lora_sgmv_noalloc",
 )
 
 
@@ -81,6 +83,7 @@ def _load():
         "lora_expand": ([P, ctypes.POINTER(lora_segments), P, I32, P, I64, I32, P], ctypes.c_int),
         "lora_sgmv": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
         "lora_bgmv": ([P, P, I32, P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
+        "lora_sgmv_noalloc": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, I32, P], ctypes.c_int),
         "lora_get_status": ([P, ctypes.POINTER(ctypes.c_uint32), I32, P], ctypes.c_int),
         "lora_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "lora_set_option": ([ctypes.c_char_p, I64], ctypes.c_int),
@@ -173,6 +176,14 @@ def lora_sgmv(table: int, seg: lora_segments, x, ldx: int, y, ldy: int, y_offset
               ws_bytes: int = 0, stream=None) -> None:
     _check(_load().lora_sgmv(table, ctypes.byref(seg), _ptr(x), ldx, _ptr(y), ldy, y_offset, _ptr(ws), ws_bytes,
                              _stream(stream)), "lora_sgmv")
+
+
+def lora_sgmv_noalloc(table: int, seg: lora_segments, x, ldx: int, y, ldy: int, y_offset: int, stream=None) -> None:
+    """SGMV for callers that cannot allocate device memory: the fp32 intermediate lives in a
+    fixed 1 MiB array owned by the library (T * ldv <= LORA_NOALLOC_SCRATCH_FLOATS).  Calls
+    that may overlap on the GPU share that array and must be serialised by the caller."""
+    _check(_load().lora_sgmv_noalloc(table, ctypes.byref(seg), _ptr(x), ldx, _ptr(y), ldy, y_offset,
+                                     _stream(stream)), "lora_sgmv_noalloc")
 
 
 def lora_bgmv(table: int, ids, T: int, x, ldx: int, y, ldy: int, y_offset: int, ws=None, ws_bytes: int = 0,

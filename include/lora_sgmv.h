@@ -158,6 +158,23 @@ int lora_bgmv(const lora_table *table, const int32_t *d_ids, int32_t T, const vo
  * timeout bit is set, otherwise LORA_ERR_DEVICE_STATUS. */
 int lora_get_status(const lora_table *table, uint32_t *h_status, int32_t reset, void *stream);
 
+/* SGMV without any workspace from the caller.  There is no counterpart on the multi-LoRA
+ * pages; it exists for callers that cannot allocate device memory themselves (a framework
+ * that owns all GPU memory through its own allocator, a runtime with a fixed memory budget,
+ * or a path where a cudaMalloc/cudaFree and the synchronisation it may bring is not allowed).
+ * Same arguments and result as lora_sgmv minus the workspace: it runs lora_shrink into a
+ * library-owned device array of LORA_NOALLOC_SCRATCH_FLOATS floats (1 MiB, held on every GPU
+ * that loads the library until the process exits), then lora_expand from it.  Limit:
+ * seg->T * ldv <= LORA_NOALLOC_SCRATCH_FLOATS with ldv = max rank rounded up to 4, else
+ * LORA_ERR_WORKSPACE is returned and nothing is launched.  It calls no allocating routine.
+ * The first call on a device looks up the array's address on that device (make that first
+ * call outside any stream capture).  All calls share the one array: calls that can overlap on
+ * the GPU (different streams, or different host threads) race on it and must be serialised by
+ * the caller.  The array keeps the last call's contents; nothing relies on it starting at 0. */
+#define LORA_NOALLOC_SCRATCH_FLOATS 262144
+int lora_sgmv_noalloc(const lora_table *table, const lora_segments *seg, const void *x, int64_t ldx,
+                      void *y, int64_t ldy, int32_t y_offset, void *stream);
+
 /* Static text for a return code. */
 const char *lora_status_string(int code);
 
