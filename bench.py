@@ -200,7 +200,7 @@ def make_step(wl, L):
         def step(c, s):
             d, t = c.projs[0], c.tables[0]
             L.lora_sgmv(t.handle, c.seg, d.x, d.h, d.y0, d.o, 0, c.ws, c.ws.numel(), s)
-        return step, 1, "prefill path"
+        return step, 2, "prefill_shrink_kernel + prefill_expand_kernel (tcgen05)"
     raise ValueError(name)
 
 
@@ -377,7 +377,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": "%s: %s" % (args.workload, DESCRIPTIONS[args.workload]),
                    "tokens_per_step": T, "distinct_adapters_per_step": distinct,
                    "algorithmic_bytes_per_step": bytes_step, "flops_per_step": flops_step,
-                   "l2": "rotating %d input copies (%.0f MB > 4x L2)" % (C, C * ws_bytes / 1e6),
+                   "l2": "rotating %d input copies, %.0f MB in total against a 126 MB L2%s" % (
+                       C, C * ws_bytes / 1e6, "" if C * ws_bytes >= 4 * L2_BYTES else " (copy count capped)"),
                    "graph": not args.no_graph, "pdl": bool(L.lora_get_option("pdl")),
                    "parallelism": "replicas x%d (independent token batches, no collective)" % world},
         "roofline": roofline,

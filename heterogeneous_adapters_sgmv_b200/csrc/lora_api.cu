@@ -160,6 +160,8 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
     t->d_desc = nullptr;
     t->d_status = nullptr;
     t->d_tmaps = nullptr;
+    t->d_tmaps_pfA = nullptr;
+    t->d_tmaps_pfB = nullptr;
     if (cudaGetDevice(&t->device) != cudaSuccess) {
         delete t;
         return LORA_ERR_CUDA;
@@ -192,6 +194,7 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
          cudaMemsetAsync(t->d_status, 0, 256, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess))
         rc = LORA_ERR_CUDA;
     delete[] h_desc;
+    if (rc == LORA_OK) rc = prefill_build_maps(t);
     if (rc != LORA_OK) {
         lora_table_destroy(t);
         return rc;
@@ -210,6 +213,8 @@ int lora_table_destroy(lora_table *t)
     if (t->d_desc) cudaFree(t->d_desc);
     if (t->d_status) cudaFree(t->d_status);
     if (t->d_tmaps) cudaFree(t->d_tmaps);
+    if (t->d_tmaps_pfA) cudaFree(t->d_tmaps_pfA);
+    if (t->d_tmaps_pfB) cudaFree(t->d_tmaps_pfB);
     cudaSetDevice(prev);
     delete t;
     return LORA_OK;

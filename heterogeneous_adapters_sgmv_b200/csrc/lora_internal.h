@@ -9,6 +9,7 @@
 #include "lora_sgmv.h"
 
 struct CUtensorMap_st;
+struct lora_table;
 
 namespace lora {
 struct AdapterDesc;
@@ -52,6 +53,8 @@ Options &options();
 int launch_decode(int mode, int src, const DecodeParams &p, int dtype, cudaStream_t s);
 int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *perm, int32_t *seg_ptr,
                           int32_t *seg_adapter, int32_t *num_segs, uint32_t *status, cudaStream_t s);
+// Tensor maps of every adapter for the tcgen05 prefill path (no-op when the table does not qualify).
+int prefill_build_maps(lora_table *t);
 // Encode the TMA tensor map of A_i [rank, h] used by the decode shrink (host side).
 int encode_tmap_A(void *out128, const void *A, int dtype, int h, int rank);
 
@@ -67,4 +70,6 @@ struct lora_table {
     std::vector<float> scales;
     // per-adapter TMA tensor maps of A_i (device array of 128-byte CUtensorMap)
     void *d_tmaps;
+    // prefill path (bf16, ranks multiple of 8 and <= 64): 128-byte-swizzled maps of A_i, B_i
+    void *d_tmaps_pfA, *d_tmaps_pfB;
 };

@@ -1,16 +1,619 @@
-// Prefill path for long contiguous segments (tcgen05 tensor cores); not yet available in
-// this build: lora_sgmv keeps long segments on the decode kernels.
+// Prefill path of the LoRA delta for long, contiguous segments on the 5th-generation tensor
+// cores (tcgen05): per segment the shrink v = x . A_i^T (scale 1, fp32) and the expand
+// y += s_i * v . B_i^T are dense contractions ("Compress then Serve" review thread,
+// add_lora_slice pseudocode; "TGI Multi-LoRA" page, "Technical Foundation: LoRA").
+//
+// Shrink kernel: one cluster of 8 CTAs per (segment, 128-token tile); CTA j takes the j-th
+// eighth of h.  A producer thread streams x and A_i tiles (64 columns of h, 128-byte swizzle)
+// with 2-D tensor-map TMA loads into a 4-deep ring; one thread issues tcgen05.mma
+// (M = 128 tokens, N = rank rounded up to 16, K = 16) accumulating in tensor memory; the
+// partials are summed in fixed CTA order through distributed shared memory and written to
+// v in fp32.
+//
+// Expand kernel: one CTA per (segment, 128-token tile, 128-column tile of o).  The fp32
+// intermediate is split into bf16 hi + lo (v = hi + lo to about 16 bits), written into shared
+// memory in the 128-byte-swizzled K-major layout the tensor core reads, and multiplied with
+// the B_i tile (TMA) in 8 MMAs of K = 16.  The y tile arrives by TMA; the epilogue reads the
+// accumulator from tensor memory row by row, adds s_i * acc to y, rounds once to bf16 and
+// stores with coalesced 16-byte stores masked to the segment, so neighbouring segments are
+// never touched.
+//
+// No TMA multicast.  Every wait is bounded; on timeout a status bit is latched, in-flight
+// copies are drained and tensor memory is released before the CTA exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+#include <vector>
+
 #include "lora_common.cuh"
 #include "lora_internal.h"
 
 namespace lora {
+namespace {
 
-bool prefill_supported(const lora_table *) { return false; }
+constexpr int kTileM = 128;          // tokens per tile
+constexpr int kTileN = 128;          // columns of o per expand tile
+constexpr int kBK = 64;              // columns of h per shrink k-block (128 bytes of bf16)
+constexpr int kKSplit = 8;           // CTAs per shrink cluster
+constexpr int kStages = 4;           // shrink pipeline depth
+constexpr int kThreadsPF = 128;      // 4 warps: one TMEM lane quarter each
+constexpr int kMaxRankPF = 64;
 
-int launch_prefill(const lora_table *, const lora_segments *, const void *, int64_t, void *, int64_t, int32_t,
-                   float *, int32_t, cudaStream_t)
+// ------------------------------------------------------------------- tcgen05 helpers
+
+__device__ __forceinline__ void tmem_alloc(uint32_t smem_dst, uint32_t ncols)
 {
-    return LORA_ERR_UNSUPPORTED;
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem desc] . B[smem desc]^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive (once) on `bar` when all previously issued MMAs of this thread have completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Shared-memory descriptor of a K-major operand stored with the 128-byte swizzle: rows of
+// 128 bytes, 8-row atoms of 1024 bytes stacked along M/N (stride 1024), sm_100 descriptor
+// version 1.  Advancing K by 16 bf16 within the 128-byte row adds 32 bytes to the start.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;              // leading byte offset (unused with this swizzle)
+    d |= (uint64_t)(1024u >> 4) << 32;    // stride byte offset: next 8-row atom
+    d |= (uint64_t)1u << 46;              // descriptor version
+    d |= (uint64_t)2u << 61;              // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk c of row m in a 128-byte-swizzled [rows][128 B] tile.
+__device__ __forceinline__ uint32_t sw128_off(int m, int c) { return (uint32_t)(m * 128 + ((c ^ (m & 7)) << 4)); }
+
+struct PrefillParams {
+    CUtensorMap tmap_io;          // shrink: x [T, h]; expand: y slice [T, o]   (box 64 x 128)
+    const AdapterDesc *desc;
+    const uint8_t *tm_A;          // per adapter: tensor map of A_i, box 64 x roundup(r, 16)
+    const uint8_t *tm_B;          // per adapter: tensor map of B_i, box 64 x 128
+    const int32_t *seg_ptr, *seg_adapter, *num_segs;
+    int32_t max_segs, T, h, o, n;
+    float *v;
+    int32_t ldv;
+    void *y;
+    int64_t ldy;
+    int32_t y_off;
+    uint32_t *status;
+};
+
+// Map a global 128-token tile index to (segment, first row, rows).  One warp scans the
+// segment table; returns false when the index is past the last tile.
+__device__ bool find_tile(const PrefillParams &p, int g, int *seg, int *row0, int *rows, int *adapter)
+{
+    const int lane = threadIdx.x & 31;
+    const int nseg = min(*p.num_segs, p.max_segs);
+    int base_tiles = 0;
+    for (int s0 = 0; s0 < nseg; s0 += 32) {
+        const int s = s0 + lane;
+        int len = 0;
+        if (s < nseg) len = max(0, min(p.seg_ptr[s + 1], p.T) - max(p.seg_ptr[s], 0));   // bad bounds: empty
+        const int tiles = (len + kTileM - 1) / kTileM;
+        int incl = tiles;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        const int excl = base_tiles + incl - tiles;
+        const bool hit = (g >= excl) && (g < excl + tiles);
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            const int s_hit = __shfl_sync(0xffffffffu, s, src);
+            const int e_hit = __shfl_sync(0xffffffffu, excl, src);
+            const int start = max(p.seg_ptr[s_hit], 0);
+            const int end = min(p.seg_ptr[s_hit + 1], p.T);
+            *seg = s_hit;
+            *row0 = start + (g - e_hit) * kTileM;
+            *rows = min(kTileM, end - *row0);
+            *adapter = p.seg_adapter[s_hit];
+            return true;
+        }
+        base_tiles += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return false;
+}
+
+struct __align__(8) ShrinkCtl {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t done;
+    uint32_t tmem_base;
+    int32_t info[5];   // valid, row0, rows, adapter, rank
+};
+
+__global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __grid_constant__ PrefillParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment for the swizzled tiles
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int kXBytes = kTileM * 128;              // 16 KiB
+    constexpr int kABytes = kMaxRankPF * 128;          //  8 KiB (room for rank <= 64)
+    constexpr int kStageBytes = kXBytes + kABytes;
+    ShrinkCtl &ctl = *reinterpret_cast<ShrinkCtl *>(smem + kStages * kStageBytes);
+    float *part = reinterpret_cast<float *>(smem);     // [128][PRS] fp32, reuses the ring after the MMAs
+    constexpr int PRS = kMaxRankPF + 4;                // padded row stride of the partial
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t crank = cluster_ctarank();
+    const int g = (int)cluster_id_x();
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        int s, row0 = 0, rows = 0, a = 0;
+        const bool ok = find_tile(p, g, &s, &row0, &rows, &a);
+        if (lane == 0) {
+            const bool good = ok && a >= 0 && a < p.n && rows > 0;
+            if (ok && !good && crank == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+            ctl.info[0] = good ? 1 : 0;
+            ctl.info[1] = row0;
+            ctl.info[2] = rows;
+            ctl.info[3] = a;
+            ctl.info[4] = good ? p.desc[a].rank : 0;
+            for (int i = 0; i < kStages; ++i) {
+                mbar_init(smem_u32(&ctl.full[i]), 1);
+                mbar_init(smem_u32(&ctl.empty[i]), 1);
+            }
+            mbar_init(smem_u32(&ctl.done), 1);
+            fence_mbar_init_cluster();
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&ctl.tmem_base), 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const bool valid = ctl.info[0] != 0;
+    const int row0 = ctl.info[1], rows = ctl.info[2], a = ctl.info[3], r = ctl.info[4];
+    const int npad = (r + 15) & ~15;
+    const uint32_t tmem = ctl.tmem_base;
+    const int nkb_all = (p.h + kBK - 1) / kBK;
+    const int kb0 = (int)((int64_t)crank * nkb_all / kKSplit);
+    const int kb1 = (int)((int64_t)(crank + 1) * nkb_all / kKSplit);
+    const int nkb = valid ? kb1 - kb0 : 0;
+    bool ok = true;
+
+    if (valid && nkb > 0) {
+        if (warp == 0 && lane == 0) {
+            // producer: x tile (128 tokens x 64 columns) and A_i tile (npad rows x 64 columns)
+            const void *tA = p.tm_A + (size_t)a * 128;
+            const uint32_t bytes = (uint32_t)(kXBytes + npad * 128);
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % kStages, m = kb / kStages;
+                if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) break;
+                uint8_t *st = smem + s * kStageBytes;
+                const uint32_t fb = smem_u32(&ctl.full[s]);
+                mbar_arrive_expect_tx(fb, bytes);
+                const int k0 = (kb0 + kb) * kBK;
+                tma_load_2d(smem_u32(st), &p.tmap_io, k0, row0, fb);
+                tma_load_2d(smem_u32(st + kXBytes), tA, k0, 0, fb);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // MMA issuer
+            const uint32_t idesc = idesc_bf16(kTileM, npad);
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % kStages, m = kb / kStages;
+                if (!mbar_wait(smem_u32(&ctl.full[s]), m & 1, p.status)) break;
+                tc_fence_after();
+                uint8_t *st = smem + s * kStageBytes;
+                const uint64_t ad = sw128_desc(smem_u32(st));
+                const uint64_t bd = sw128_desc(smem_u32(st + kXBytes));
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                    umma_bf16(tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+                umma_commit(smem_u32(&ctl.empty[s]));
+            }
+            umma_commit(smem_u32(&ctl.done));
+        }
+        __syncwarp();
+        ok = mbar_wait(smem_u32(&ctl.done), 0, p.status);
+        tc_fence_after();
+    }
+    // ---- epilogue: partial [128][npad] from tensor memory (zeros when this CTA had no k-blocks)
+    __syncthreads();   // the ring is free: all MMAs and loads that fed them are complete
+    const int m = warp * 32 + lane;   // row of the tile = TMEM lane
+    if (valid) {
+        for (int c0 = 0; c0 < npad; c0 += 32) {
+            float acc[32];
+            if (nkb > 0 && ok) {
+                tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, acc);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i < npad) part[m * PRS + c0 + i] = acc[i];
+        }
+    }
+    cluster_sync_all();   // every CTA's partial is visible to its peers
+    if (valid) {
+        // CTA j reduces rows [16 j, 16 j + 16) over the 8 partials, in CTA order
+        const uint32_t part_addr = smem_u32(part);
+        for (int e = tid; e < 16 * r; e += kThreadsPF) {
+            const int rr = crank * 16 + e / r, k = e % r;
+            float sum = 0.f;
+            float pv[kKSplit];
+#pragma unroll
+            for (int j = 0; j < kKSplit; ++j) pv[j] = ld_dsmem_f32(part_addr + 4u * (rr * PRS + k), j);
+#pragma unroll
+            for (int j = 0; j < kKSplit; ++j) sum += pv[j];
+            if (rr < rows) p.v[(int64_t)(row0 + rr) * p.ldv + k] = sum;
+        }
+    }
+    cluster_sync_all();   // no peer reads this CTA's partial any more
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 64);
+}
+
+struct __align__(8) ExpandCtl {
+    uint64_t bar_b, bar_y, bar_mma;
+    uint32_t tmem_base;
+    int32_t info[6];   // valid, row0, rows, adapter, rank, scale bits
+};
+
+__global__ void __launch_bounds__(kThreadsPF, 1) prefill_expand_kernel(const __grid_constant__ PrefillParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *vhi = smem;                   // [128][128 B] swizzled, bf16 hi part of v
+    uint8_t *vlo = smem + 16384;           // bf16 lo part
+    uint8_t *bt = smem + 32768;            // B_i tile: 128 rows of o x 64 ranks, swizzled
+    uint8_t *yt = smem + 49152;            // y tile: two 64-column boxes [128][128 B], swizzled
+    ExpandCtl &ctl = *reinterpret_cast<ExpandCtl *>(smem + 81920);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nt = blockIdx.x;
+    const int g = blockIdx.y;
+    const int col0 = nt * kTileN;
+    const int ncols = min(kTileN, p.o - col0);
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        int s, row0 = 0, rows = 0, a = 0;
+        const bool ok = find_tile(p, g, &s, &row0, &rows, &a);
+        if (lane == 0) {
+            const bool good = ok && a >= 0 && a < p.n && rows > 0 && ncols > 0;
+            if (ok && !good && nt == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+            ctl.info[0] = good ? 1 : 0;
+            ctl.info[1] = row0;
+            ctl.info[2] = rows;
+            ctl.info[3] = a;
+            ctl.info[4] = good ? p.desc[a].rank : 0;
+            ctl.info[5] = good ? __float_as_int(p.desc[a].scale) : 0;
+            mbar_init(smem_u32(&ctl.bar_b), 1);
+            mbar_init(smem_u32(&ctl.bar_y), 1);
+            mbar_init(smem_u32(&ctl.bar_mma), 1);
+            fence_mbar_init_cluster();
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&ctl.tmem_base), 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const bool valid = ctl.info[0] != 0;
+    const int row0 = ctl.info[1], rows = ctl.info[2], a = ctl.info[3], r = ctl.info[4];
+    const float sc = __int_as_float(ctl.info[5]);
+    const uint32_t tmem = ctl.tmem_base;
+    bool ok = true;
+
+    if (valid) {
+        if (tid == 0) {
+            const uint32_t bb = smem_u32(&ctl.bar_b), yb = smem_u32(&ctl.bar_y);
+            mbar_arrive_expect_tx(bb, 16384);
+            tma_load_2d(smem_u32(bt), p.tm_B + (size_t)a * 128, 0, col0, bb);
+            mbar_arrive_expect_tx(yb, 32768);
+            tma_load_2d(smem_u32(yt), &p.tmap_io, col0, row0, yb);
+            tma_load_2d(smem_u32(yt + 16384), &p.tmap_io, col0 + 64, row0, yb);
+        }
+        // ---- v tile: row m of the tile, split into bf16 hi + lo, 128-byte swizzle, zero past r
+        {
+            const int m = tid;
+            const bool rv = m < rows;
+            const float *vr = p.v + (int64_t)(row0 + m) * p.ldv;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int k = c * 8 + e;
+                    f[e] = (rv && k < r) ? vr[k] : 0.f;
+                }
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(f[e], f[e + 1]);
+                    const float2 hf = __bfloat1622float2(h2);
+                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(f[e] - hf.x, f[e + 1] - hf.y);
+                    hi[e / 2] = *reinterpret_cast<const uint32_t *>(&h2);
+                    lo[e / 2] = *reinterpret_cast<const uint32_t *>(&l2);
+                }
+                *reinterpret_cast<uint4 *>(vhi + sw128_off(m, c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(vlo + sw128_off(m, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        fence_proxy_async_smem();   // generic-proxy writes of v become visible to the tensor core
+        __syncthreads();
+        if (tid == 32) {
+            // MMA issuer: acc[128 x 128] = vhi . B^T + vlo . B^T
+            if (mbar_wait(smem_u32(&ctl.bar_b), 0, p.status)) {
+                tc_fence_after();
+                const uint32_t idesc = idesc_bf16(kTileM, kTileN);
+                const uint64_t dh = sw128_desc(smem_u32(vhi)), dl = sw128_desc(smem_u32(vlo));
+                const uint64_t db = sw128_desc(smem_u32(bt));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) umma_bf16(tmem, dh + 2 * k, db + 2 * k, idesc, k != 0 ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) umma_bf16(tmem, dl + 2 * k, db + 2 * k, idesc, 1u);
+            }
+            umma_commit(smem_u32(&ctl.bar_mma));
+        }
+        __syncwarp();
+        ok = mbar_wait(smem_u32(&ctl.bar_mma), 0, p.status);
+        ok = mbar_wait(smem_u32(&ctl.bar_y), 0, p.status) && ok;
+        tc_fence_after();
+        // ---- epilogue: thread m owns row m; y + s * acc, rounded once, written back in place
+        if (ok) {
+            const int m = tid;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kTileN; c0 += 32) {
+                float acc[32];
+                tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, acc);
+                uint8_t *box = yt + (c0 >= 64 ? 16384 : 0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int chunk = ((c0 & 63) >> 3) + q;
+                    uint4 *pw = reinterpret_cast<uint4 *>(box + sw128_off(m, chunk));
+                    uint4 w = *pw;
+                    uint32_t *wv = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float y0 = fmaf(sc, acc[q * 8 + 2 * e], bf16_lo(wv[e]));
+                        const float y1 = fmaf(sc, acc[q * 8 + 2 * e + 1], bf16_hi(wv[e]));
+                        wv[e] = pack_bf16x2(y0, y1);
+                    }
+                    *pw = w;
+                }
+            }
+        }
+        __syncthreads();
+        // ---- coalesced stores of the tile's valid rows and columns (two rows per warp step)
+        if (ok) {
+            uint8_t *yg = static_cast<uint8_t *>(p.y);
+            for (int rr = warp * 32 + (lane >> 4); rr < warp * 32 + 32; rr += 2) {
+                const int chunk = lane & 15;
+                if (rr < rows && chunk * 8 < ncols) {
+                    const uint8_t *box = yt + (chunk >= 8 ? 16384 : 0);
+                    const uint4 w = *reinterpret_cast<const uint4 *>(box + sw128_off(rr, chunk & 7));
+                    *reinterpret_cast<uint4 *>(yg + ((int64_t)(row0 + rr) * p.ldy + p.y_off + col0 + chunk * 8) * 2) = w;
+                }
+            }
+        }
+    }
+    if (!ok && tid == 0) {
+        // drain whatever may still be landing before shared memory is released
+        mbar_wait(smem_u32(&ctl.bar_b), 0, p.status);
+        mbar_wait(smem_u32(&ctl.bar_y), 0, p.status);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 128);
+}
+
+// ------------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return encode;
+}
+
+// bf16 2-D map [rows, cols] with row stride `ld` elements, box 64 columns x box_rows, 128B swizzle.
+int encode_sw128(CUtensorMap *out, const void *base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_rows)
+{
+    auto encode = get_encode();
+    if (!encode) return LORA_ERR_CUDA;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult rc = encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return rc == CUDA_SUCCESS ? LORA_OK : LORA_ERR_UNSUPPORTED;
+}
+
+constexpr int kShrinkSmem = kStages * (kTileM * 128 + kMaxRankPF * 128) + 256 + 1024;
+constexpr int kExpandSmem = 81920 + 256 + 1024;
+static_assert(kStages * (kTileM * 128 + kMaxRankPF * 128) >= kTileM * (kMaxRankPF + 4) * 4, "partial fits ring");
+
+}  // namespace
+
+bool prefill_supported(const lora_table *t) { return t && t->d_tmaps_pfA && t->d_tmaps_pfB; }
+
+// Tensor maps of every adapter for the prefill path (bf16 tables, ranks multiple of 8, <= 64).
+int prefill_build_maps(lora_table *t)
+{
+    if (t->dtype != LORA_BF16) return LORA_OK;
+    for (int i = 0; i < t->n; ++i)
+        if (t->ranks[i] > kMaxRankPF || t->ranks[i] % 8) return LORA_OK;
+    std::vector<uint8_t> ha((size_t)t->n * 128), hb((size_t)t->n * 128);
+    for (int i = 0; i < t->n; ++i) {
+        const int r = t->ranks[i];
+        if (encode_sw128(reinterpret_cast<CUtensorMap *>(ha.data() + (size_t)i * 128), t->A[i], t->h, r, t->h,
+                         (r + 15) & ~15) != LORA_OK ||
+            encode_sw128(reinterpret_cast<CUtensorMap *>(hb.data() + (size_t)i * 128), t->B[i], r, t->o, r, kTileN) !=
+                LORA_OK)
+            return LORA_OK;   // leave the path off for this table
+    }
+    if (cudaMalloc(&t->d_tmaps_pfA, ha.size()) != cudaSuccess) return LORA_ERR_CUDA;
+    if (cudaMalloc(&t->d_tmaps_pfB, hb.size()) != cudaSuccess) return LORA_ERR_CUDA;
+    if (cudaMemcpy(t->d_tmaps_pfA, ha.data(), ha.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(t->d_tmaps_pfB, hb.data(), hb.size(), cudaMemcpyHostToDevice) != cudaSuccess)
+        return LORA_ERR_CUDA;
+    return LORA_OK;
+}
+
+int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y, int64_t ldy,
+                   int32_t y_off, float *v, int32_t ldv, cudaStream_t s)
+{
+    if (!prefill_supported(t)) return LORA_ERR_UNSUPPORTED;
+    PrefillParams p;
+    std::memset(&p, 0, sizeof p);
+    p.desc = t->d_desc;
+    p.tm_A = static_cast<const uint8_t *>(t->d_tmaps_pfA);
+    p.tm_B = static_cast<const uint8_t *>(t->d_tmaps_pfB);
+    p.seg_ptr = seg->seg_ptr;
+    p.seg_adapter = seg->seg_adapter;
+    p.num_segs = seg->num_segs;
+    p.max_segs = seg->max_segs;
+    p.T = seg->T;
+    p.h = t->h;
+    p.o = t->o;
+    p.n = t->n;
+    p.v = v;
+    p.ldv = ldv;
+    p.y = y;
+    p.ldy = ldy;
+    p.y_off = y_off;
+    p.status = t->d_status;
+    const int mt_bound = seg->max_segs + (seg->T + kTileM - 1) / kTileM;
+
+    static bool attr_done[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LORA_ERR_CUDA;
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(prefill_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kShrinkSmem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(prefill_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kExpandSmem) !=
+                cudaSuccess)
+            return LORA_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+    const Options &opt = options();
+
+    // shrink: clusters of kKSplit CTAs, one cluster per 128-token tile
+    int rc = encode_sw128(&p.tmap_io, x, (uint64_t)t->h, (uint64_t)seg->T, (uint64_t)ldx, kTileM);
+    if (rc != LORA_OK) return rc;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kKSplit * mt_bound);
+        cfg.blockDim = dim3(kThreadsPF);
+        cfg.dynamicSmemBytes = kShrinkSmem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kKSplit;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        int na = 1;
+        if (opt.pdl) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        if (cudaLaunchKernelEx(&cfg, prefill_shrink_kernel, p) != cudaSuccess) return LORA_ERR_CUDA;
+    }
+    // expand: one CTA per (128-token tile, 128-column tile)
+    rc = encode_sw128(&p.tmap_io, static_cast<uint8_t *>(y) + (int64_t)y_off * 2, (uint64_t)t->o, (uint64_t)seg->T,
+                      (uint64_t)ldy, kTileM);
+    if (rc != LORA_OK) return rc;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((t->o + kTileN - 1) / kTileN, mt_bound);
+        cfg.blockDim = dim3(kThreadsPF);
+        cfg.dynamicSmemBytes = kExpandSmem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        int na = 0;
+        if (opt.pdl) {
+            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[na].val.programmaticStreamSerializationAllowed = 1;
+            ++na;
+        }
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        if (cudaLaunchKernelEx(&cfg, prefill_expand_kernel, p) != cudaSuccess) return LORA_ERR_CUDA;
+    }
+    return LORA_OK;
 }
 
 }  // namespace lora

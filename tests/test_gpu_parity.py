@@ -395,3 +395,77 @@ def test_pdl_on_and_off_agree():
         L.lora_set_option("pdl", 1)
     y1 = dp.bgmv(dp.y())
     assert torch.equal(y0, y1)
+
+
+# ------------------------------------------------------------------ tcgen05 prefill path
+
+def _prefill_case(seg_lens, h, o, ranks, seed=5, delta_only=False):
+    T, n = sum(seg_lens), len(seg_lens)
+    wl = workloads.generate("prefill_sgmv", T=T, n=n, seg_len=max(seg_lens), shapes=(("up", h, o, 0),),
+                            ranks=ranks, seed=seed, delta_only=delta_only)
+    wl.ids = np.concatenate([np.full(l, i, np.int32) for i, l in enumerate(seg_lens)])
+    dp = DeviceProj(wl)
+    ptr = torch.from_numpy(np.concatenate([[0], np.cumsum(seg_lens)]).astype(np.int32)).cuda()
+    ad = torch.arange(n, dtype=torch.int32, device="cuda")
+    num = torch.tensor([n], dtype=torch.int32, device="cuda")
+    seg = L.make_segments(None, ptr, ad, num, T, n, max(seg_lens))
+    return wl, dp, seg, (ptr, ad, num)
+
+
+def _kernels_launched(fn):
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        fn()
+        torch.cuda.synchronize()
+    return {e.name for e in prof.events() if e.device_type.name == "CUDA"}
+
+
+@pytest.mark.parametrize("seg_lens,h,o,ranks", [
+    ([300], 512, 256, (16,)),
+    ([130, 100, 700, 1, 256], 1024, 384, (64, 8, 32, 16, 64)),
+    ([257, 513, 129], 4096, 1024 + 64, (64, 32, 48)),
+])
+def test_prefill_tcgen05_ragged_segments_and_ranks(seg_lens, h, o, ranks):
+    """Segments that are not multiples of the 128-token tile, o not a multiple of the
+    128-column tile, ranks 8..64: the tensor-core path matches the oracle and the CUDA-core
+    path within tolerance, and it is the path that ran."""
+    wl, dp, seg, _keep = _prefill_case(seg_lens, h, o, ranks)
+    ref = oracle.workload_reference(wl)
+    y = dp.y()
+    names = _kernels_launched(lambda: dp.sgmv(y, seg))
+    assert any("prefill_expand_kernel" in k for k in names) and any("prefill_shrink_kernel" in k for k in names)
+    assert_close(dp.to_np(y), ref, wl.dtype, "tcgen05 prefill")
+    L.lora_set_option("prefill_min_seg_len", 0)
+    try:
+        y2 = dp.sgmv(dp.y(), seg)
+    finally:
+        L.lora_set_option("prefill_min_seg_len", 256)
+    assert_close(dp.to_np(y2), ref, wl.dtype, "decode path on prefill segments")
+    assert dp.status() == (0, 0)
+
+
+def test_prefill_tcgen05_output_slice_untouched_outside():
+    wl, dp, seg, _keep = _prefill_case([257, 513], 4096, 1024, (64,))
+    o = 1024
+    wide = torch.randn(wl.T, o + 192, device="cuda").to(torch.bfloat16)
+    wide[:, 128:128 + o] = dp.d.y0
+    before = wide.clone()
+    ws = dp.workspace()
+    L.lora_sgmv(dp.table.handle, seg, dp.d.x, dp.d.x.shape[1], wide, wide.shape[1], 128, ws, ws.numel())
+    ref = oracle.workload_reference(wl)
+    assert_close(dp.to_np(wide[:, 128:128 + o].contiguous()), ref, wl.dtype, "slice")
+    assert torch.equal(wide[:, :128], before[:, :128]) and torch.equal(wide[:, 128 + o:], before[:, 128 + o:])
+
+
+def test_prefill_tcgen05_zero_B_leaves_y_bit_identical():
+    wl, dp, seg, _keep = _prefill_case([300, 200], 1024, 512, (64,))
+    dp.d.B_flat.zero_()
+    y = dp.sgmv(dp.y(), seg)
+    assert torch.equal(y, dp.d.y0)
+
+
+def test_prefill_tcgen05_deterministic():
+    wl, dp, seg, _keep = _prefill_case([512, 384], 4096, 2048, (64,))
+    y1 = dp.sgmv(dp.y(), seg)
+    y2 = dp.sgmv(dp.y(), seg)
+    assert torch.equal(y1, y2)
