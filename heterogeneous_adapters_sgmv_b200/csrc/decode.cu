@@ -13,14 +13,18 @@
 //    2-D tensor-map TMA loads (one or two instructions per unit) and its slice of B_i with one
 //    bulk copy, into a ring of shared-memory stages guarded by mbarriers, and hints the unit's
 //    x and y rows into L2.  No multicast anywhere.
-//  * Consumer warps stage x and y rows with coalesced 128-bit loads.  Shrink: warp-level
-//    split-K, a lane owns 16 bytes at two places of each 1 KiB row; 8 partial dot products per
-//    lane are folded across the warp with a transposed butterfly.
+//  * Consumer warps stage x (and the unit's y) rows with coalesced 128-bit loads.  Shrink:
+//    warp-level split-K; a warp owns rank rows k = warp + 8 i, a lane 16 bytes at two places of
+//    each 1 KiB row; each dot product is folded across the warp with a 5-step butterfly.
 //  * Each CTA pushes its partial intermediate into every peer's shared memory with st.async
 //    (completion counted in bytes on the peer's mbarrier); every CTA then sums the 8 partials in
 //    fixed CTA order.  No atomics, no grid barrier: bit-identical run to run.
 //  * Expand: a thread owns two output columns (bf16) and walks the unit's tokens; one rounding
 //    (nearest-even) per output, coalesced 32-bit stores.
+//  * Short kernels like this one are dominated by instruction fetch, so the per-unit code is
+//    kept to a few compact loops (no wide unrolling, no run-time integer division), and work
+//    that reads no input (barrier set-up, the adapter descriptor when a cluster owns a fixed
+//    adapter) happens before the wait on the previous grid.
 //  * Persistent grid: as many clusters as fit, each walking the unit list with a stride.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -115,97 +119,18 @@ __device__ __forceinline__ void cvt16(const uint4 w, float *o, float *)
     o[2] = __uint_as_float(w.z); o[3] = __uint_as_float(w.w);
 }
 
-// Sum 8 per-lane values over the 32 lanes of a warp.  On return lane L holds the total of
-// value index (L >> 2) & 7.  Fixed order, so the result is deterministic.
-__device__ __forceinline__ float warp_reduce8(float (&a)[8], int lane)
+// Sum over the 32 lanes of a warp (fixed butterfly order: deterministic).
+__device__ __forceinline__ float warp_sum(float v)
 {
-    {
-        const bool up = lane & 16;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float send = up ? a[q] : a[q + 4];
-            const float keep = up ? a[q + 4] : a[q];
-            a[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-        }
-    }
-    {
-        const bool up = lane & 8;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const float send = up ? a[q] : a[q + 2];
-            const float keep = up ? a[q + 2] : a[q];
-            a[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-    }
-    {
-        const bool up = lane & 4;
-        const float send = up ? a[0] : a[1];
-        const float keep = up ? a[1] : a[0];
-        a[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    float r = a[0];
-    r += __shfl_xor_sync(0xffffffffu, r, 2);
-    r += __shfl_xor_sync(0xffffffffu, r, 1);
-    return r;
+    v += __shfl_xor_sync(0xffffffffu, v, 16);
+    v += __shfl_xor_sync(0xffffffffu, v, 8);
+    v += __shfl_xor_sync(0xffffffffu, v, 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v;
 }
 
-// Partial shrink of one staged tile by one warp.  The warp owns rank rows k = warp + 8*i; it
-// takes RB of them at a time against TG = 8 / RB tokens, so every butterfly folds 8 values.
-// A is staged as [box][row][512 B] (box 1 starts after r rows of box 0), x as [token][1 KiB];
-// a lane reads 16-byte chunks `lane` (box 0) and `lane + 32` (box 1).  Operands are read from
-// shared memory at the point of use (nothing held across tokens), which keeps registers low.
-template <typename E, int RB>
-__device__ __forceinline__ void shrink_rows(const uint8_t *A, const uint8_t *xs, int rowb, float *vpart, int RP,
-                                            int r, int L, int nch, int warp, int lane, bool first)
-{
-    constexpr int EPC = Tr<E>::EPC;
-    constexpr int TG = 8 / RB;
-    const bool okA = lane < nch, okB = lane + 32 < nch;
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    const int nrows = (r > warp) ? (r - warp + 7) / 8 : 0;
-    for (int rb0 = 0; rb0 < nrows; rb0 += RB) {
-        for (int t0 = 0; t0 < L; t0 += TG) {
-            float acc[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-#pragma unroll
-            for (int tt = 0; tt < TG; ++tt) {
-                if (t0 + tt < L) {
-                    const uint8_t *xr = xs + (t0 + tt) * rowb;
-                    const uint4 x0 = okA ? *reinterpret_cast<const uint4 *>(xr + lane * 16) : z;
-                    const uint4 x1 = okB ? *reinterpret_cast<const uint4 *>(xr + 512 + lane * 16) : z;
-                    float xv[2][EPC];
-                    cvt16(x0, xv[0], (E *)nullptr);
-                    cvt16(x1, xv[1], (E *)nullptr);
-#pragma unroll
-                    for (int i = 0; i < RB; ++i) {
-                        if (rb0 + i < nrows) {
-                            const uint8_t *row = A + (warp + 8 * (rb0 + i)) * kBoxBytes;
-                            float av[EPC];
-                            float sum = 0.f;
-                            cvt16(okA ? *reinterpret_cast<const uint4 *>(row + lane * 16) : z, av, (E *)nullptr);
-#pragma unroll
-                            for (int e = 0; e < EPC; ++e) sum = fmaf(xv[0][e], av[e], sum);
-                            cvt16(okB ? *reinterpret_cast<const uint4 *>(row + r * kBoxBytes + lane * 16) : z, av,
-                                  (E *)nullptr);
-#pragma unroll
-                            for (int e = 0; e < EPC; ++e) sum = fmaf(xv[1][e], av[e], sum);
-                            acc[tt * RB + i] = sum;
-                        }
-                    }
-                }
-            }
-            const float tot = warp_reduce8(acc, lane);
-            const int vi = (lane >> 2) & 7;
-            const int l = t0 + vi / RB, i = vi % RB;
-            const int k = warp + 8 * (rb0 + i);
-            if ((lane & 3) == 0 && l < L && rb0 + i < nrows) {
-                float *dst = vpart + l * RP + k;
-                *dst = first ? tot : *dst + tot;
-            }
-        }
-    }
-}
+__device__ __forceinline__ int ceil_log2(int v) { return v <= 1 ? 0 : 32 - __clz(v - 1); }
 
 template <typename E, int MODE, int SRC>
 __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_constant__ DecodeParams p)
@@ -215,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     constexpr int BOXW = kBoxBytes / ESZ;       // elements of one TMA box row
     const int rowb = row_bytes_for(p.R);        // bytes of one staged row
     const int W = rowb / ESZ;                   // elements of one h-subtile / rows of one o-subtile
-    const int CHUNKS = rowb / 16;               // 16-byte chunks per h-subtile row
+    const int CHUNKS = rowb / 16;               // 16-byte chunks per staged row (64 or 32)
+    const int lgC = CHUNKS == 64 ? 6 : 5;
 
     extern __shared__ __align__(128) uint8_t smem[];
     SmemCtl &ctl = *reinterpret_cast<SmemCtl *>(smem);
@@ -227,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     float *vsum = reinterpret_cast<float *>(smem + lay.vsum_off);     // [kTokChunk][RP] the unit's intermediate
     uint8_t *stage_base = smem + lay.stage_off;
     const int RP = lay.RP;
+    const int lgRP = ceil_log2(RP);
     const int S = p.stages;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -234,9 +161,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     const int cid = (int)cluster_id_x(), G = (int)nclusters_x();
 
     if (tid == 0) LORA_TRACE_MARK(0);
-    pdl_wait();
-    pdl_launch_dependents();
-
+    // Set-up that reads no input may overlap the previous grid (programmatic launch).
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(smem_u32(&ctl.full[s]), 1);
@@ -247,45 +172,53 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         mbar_init(smem_u32(&ctl.freed), kCluster);
         fence_mbar_init_cluster();
     }
+    __syncthreads();            // barriers initialised for this CTA
+    cluster_arrive_relaxed();   // peers wait for this before their first remote access to us
 
-    // Per-token ids: tokens with equal ids form one group.  When there are no more adapters
-    // than clusters, cluster c simply owns adapter c; otherwise a group is led by the first
-    // token carrying its id and groups are listed in the order of their leaders.
+    // Per-token ids: tokens with equal ids form one group.  With no more adapters than
+    // clusters, cluster c owns adapter c and its producer scans the ids itself; otherwise a
+    // group is led by the first token carrying its id and groups are listed in leader order.
     int32_t *ids_s = reinterpret_cast<int32_t *>(smem + lay.ids_off);
     int32_t *first = ids_s + p.T;
     int32_t *leaders = first + p.n;
     const bool direct_ids = (SRC == kSrcIds) && p.n <= G;
-    if (SRC == kSrcIds) {
+    // The adapter table is immutable after creation: in direct mode this cluster's descriptor
+    // and tensor map are fetched before waiting for the previous grid.
+    AdapterDesc pre_desc = {};
+    if (direct_ids && warp == kConsumerWarps && cid < p.n) {
+        pre_desc = p.desc[cid];
+        if (lane == 0) prefetch_tensormap(reinterpret_cast<const char *>(p.tmA) + (size_t)cid * 128);
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+    if (SRC == kSrcIds && !direct_ids) {
         bool bad = false;
         for (int t = tid; t < p.T; t += kThreads) {
             const int32_t a = p.ids[t];
             ids_s[t] = a;
             bad |= (a < -1 || a >= p.n);
         }
-        if (!direct_ids)
-            for (int i = tid; i < p.n; i += kThreads) first[i] = INT_MAX;
+        for (int i = tid; i < p.n; i += kThreads) first[i] = INT_MAX;
         if (__syncthreads_or(bad) && tid == 0 && crank == 0 && cid == 0) atomicOr(p.status, LORA_STATUS_BAD_ID);
-        if (!direct_ids) {
-            for (int t = tid; t < p.T; t += kThreads) {
-                const int32_t a = ids_s[t];
-                if (a >= 0 && a < p.n) atomicMin(&first[a], t);
-            }
-            __syncthreads();
-            if (warp == 0) {
-                int cnt = 0;
-                for (int base = 0; base < p.T; base += 32) {
-                    const int t = base + lane;
-                    const int32_t a = t < p.T ? ids_s[t] : -1;
-                    const bool lead = a >= 0 && a < p.n && first[a] == t;
-                    const uint32_t m = __ballot_sync(0xffffffffu, lead);
-                    if (lead) leaders[cnt + __popc(m & ((1u << lane) - 1u))] = t;
-                    cnt += __popc(m);
-                }
-                if (lane == 0) ctl.n_groups = cnt;
-            }
+        for (int t = tid; t < p.T; t += kThreads) {
+            const int32_t a = ids_s[t];
+            if (a >= 0 && a < p.n) atomicMin(&first[a], t);
         }
+        __syncthreads();
+        if (warp == 0) {
+            int cnt = 0;
+            for (int base = 0; base < p.T; base += 32) {
+                const int t = base + lane;
+                const int32_t a = t < p.T ? ids_s[t] : -1;
+                const bool lead = a >= 0 && a < p.n && first[a] == t;
+                const uint32_t m = __ballot_sync(0xffffffffu, lead);
+                if (lead) leaders[cnt + __popc(m & ((1u << lane) - 1u))] = t;
+                cnt += __popc(m);
+            }
+            if (lane == 0) ctl.n_groups = cnt;
+        }
+        __syncthreads();
     }
-    cluster_sync_all();   // barrier inits visible cluster-wide; group list ready
     if (tid == 0) LORA_TRACE_MARK(1);
 
     // h and o ranges of this CTA, in 16-byte chunks of h and EPC-row groups of o
@@ -302,15 +235,104 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         // ================================ producer warp ================================
         int issued = 0;
         bool alive = true;
-        // Issue every tile of one unit: adapter a, tokens held by lanes 0..L-1 (my_tok).
-        auto emit_unit = [&](int a, int my_tok, int L) {
-            const AdapterDesc d = p.desc[a];
+        if (direct_ids) {
+            // stage the ids for this warp's scan; cluster 0 CTA 0 reports bad ids
+            bool bad = false;
+            for (int t = lane; t < p.T; t += 32) {
+                const int32_t v = p.ids[t];
+                ids_s[t] = v;
+                bad |= (v < -1 || v >= p.n);
+            }
+            if (__any_sync(0xffffffffu, bad) && lane == 0 && crank == 0 && cid == 0)
+                atomicOr(p.status, LORA_STATUS_BAD_ID);
+            __syncwarp();
+        }
+        // Walk this cluster's units; each yields (adapter, descriptor, tokens in lanes 0..L-1).
+        int seg = cid, q = 0, g = cid, base = -1, cnt = 0;
+        for (;;) {
+            int a = -1, my_tok = 0, L = 0;
+            AdapterDesc d = {};
+            if (SRC == kSrcSegments) {
+                const int nseg = min(*p.num_segs, p.max_segs);
+                while (seg < nseg && L == 0) {
+                    const int sa = p.seg_adapter[seg];
+                    const int p0 = p.seg_ptr[seg], p1 = p.seg_ptr[seg + 1];
+                    if (sa < 0 || sa >= p.n || p0 < 0 || p1 < p0 || p1 > p.T) {
+                        if (lane == 0 && crank == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+                        seg += G;
+                        q = 0;
+                        continue;
+                    }
+                    const int start = p0 + q;
+                    const int L0 = min(kTokChunk, p1 - start);
+                    int t = -1;
+                    if (lane < L0) t = p.perm ? p.perm[start + lane] : start + lane;
+                    const bool ok = lane < L0 && t >= 0 && t < p.T;
+                    const uint32_t m = __ballot_sync(0xffffffffu, ok);
+                    if (m != __ballot_sync(0xffffffffu, lane < L0) && lane == 0 && crank == 0)
+                        atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+                    // compact the valid tokens to lanes 0 .. popc(m) - 1, order kept
+                    const int dst = __popc(m & ((1u << lane) - 1u));
+                    if (ok) ctl.pending[dst] = t;
+                    __syncwarp();
+                    my_tok = ctl.pending[lane & (kTokChunk - 1)];
+                    __syncwarp();
+                    L = __popc(m);
+                    a = sa;
+                    q += kTokChunk;
+                    if (p0 + q >= p1) {
+                        seg += G;
+                        q = 0;
+                    }
+                }
+                if (L > 0) d = p.desc[a];
+            } else {
+                const int ng = direct_ids ? min(p.n, cid + 1) : ctl.n_groups;
+                while (g < ng && L == 0) {
+                    const int t0 = direct_ids ? 0 : leaders[g];
+                    const int ga = direct_ids ? g : ids_s[t0];
+                    if (base < 0) base = t0;
+                    // gather up to kTokChunk members of group g, resuming at `base`
+                    while (base < p.T && cnt < kTokChunk) {
+                        const int t = base + lane;
+                        const uint32_t m = __ballot_sync(0xffffffffu, t < p.T && ids_s[t] == ga);
+                        const int take = min(__popc(m), kTokChunk - cnt);
+                        const int rk = __popc(m & ((1u << lane) - 1u));
+                        if (((m >> lane) & 1u) && rk < take) ctl.pending[cnt + rk] = t;
+                        cnt += take;
+                        if (take < __popc(m)) {
+                            // resume just after the last member taken
+                            uint32_t mm = m;
+                            for (int i = 0; i < take; ++i) mm &= mm - 1u;
+                            base += __ffs(mm) - 1;
+                        } else {
+                            base += 32;
+                        }
+                    }
+                    __syncwarp();
+                    if (cnt > 0) {
+                        my_tok = ctl.pending[lane & (kTokChunk - 1)];
+                        L = cnt;
+                        a = ga;
+                        d = direct_ids ? pre_desc : p.desc[ga];
+                    }
+                    __syncwarp();
+                    cnt = 0;
+                    if (base >= p.T) {
+                        g += G;
+                        base = -1;
+                    }
+                }
+            }
+            if (L == 0 || !alive) break;
+
+            // ---- issue every tile of this unit
             const int r = d.rank;
             const char *tmapA = reinterpret_cast<const char *>(p.tmA) + (size_t)a * 128;
             const uint8_t *Bb = static_cast<const uint8_t *>(d.B);
             if (lane == 0) LORA_TRACE_MARK(2);
             const int ntiles = n_shrink + n_expand;
-            for (int j = 0; j < ntiles && alive; ++j) {
+            for (int j = 0; j < ntiles; ++j) {
                 const int s = issued % S, m = issued / S;
                 if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
                     alive = false;
@@ -359,77 +381,15 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         bulk_g2s(data, Bb + (int64_t)off * r * ESZ, len * r * ESZ, fb);
                     }
                 }
-                // L2 hints for the rows the consumers load for this tile
-                const int lines = (len * ESZ + 127) / 128;
-                for (int l = 0; l < L; ++l) {
-                    const int t = __shfl_sync(0xffffffffu, my_tok, l);
+                // L2 hints for the rows the consumers load for this tile (lane l: row l)
+                if (lane < L) {
                     const uint8_t *row =
-                        shrink ? static_cast<const uint8_t *>(p.x) + ((int64_t)t * p.ldx + off) * ESZ
-                               : static_cast<const uint8_t *>(p.y) + ((int64_t)t * p.ldy + p.y_off + off) * ESZ;
-                    for (int c = lane; c < lines; c += 32) prefetch_l2(row + c * 128);
+                        shrink ? static_cast<const uint8_t *>(p.x) + ((int64_t)my_tok * p.ldx + off) * ESZ
+                               : static_cast<const uint8_t *>(p.y) + ((int64_t)my_tok * p.ldy + p.y_off + off) * ESZ;
+                    for (int c = 0; c < len * ESZ; c += 128) prefetch_l2(row + c);
                 }
                 ++issued;
                 if (lane == 0) LORA_TRACE_MARK(shrink ? 3 : 4);
-            }
-        };
-
-        if (SRC == kSrcSegments) {
-            const int nseg = min(*p.num_segs, p.max_segs);
-            for (int s = cid; s < nseg && alive; s += G) {
-                const int a = p.seg_adapter[s];
-                const int p0 = p.seg_ptr[s], p1 = p.seg_ptr[s + 1];
-                if (a < 0 || a >= p.n || p0 < 0 || p1 < p0 || p1 > p.T) {
-                    if (lane == 0 && crank == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
-                    continue;
-                }
-                for (int q = p0; q < p1 && alive; q += kTokChunk) {
-                    const int L0 = min(kTokChunk, p1 - q);
-                    int t = -1;
-                    if (lane < L0) t = p.perm ? p.perm[q + lane] : q + lane;
-                    const bool ok = lane < L0 && t >= 0 && t < p.T;
-                    const uint32_t m = __ballot_sync(0xffffffffu, ok);
-                    if (m != __ballot_sync(0xffffffffu, lane < L0) && lane == 0 && crank == 0)
-                        atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
-                    // compact the valid tokens to lanes 0 .. popc(m) - 1, order kept
-                    int my_tok = 0;
-                    for (int l = 0; l < L0; ++l) {
-                        const int tl = __shfl_sync(0xffffffffu, t, l);
-                        if (((m >> l) & 1u) && lane == __popc(m & ((1u << l) - 1u))) my_tok = tl;
-                    }
-                    const int L = __popc(m);
-                    if (L > 0) emit_unit(a, my_tok, L);
-                }
-            }
-        } else {
-            const int ng = direct_ids ? p.n : ctl.n_groups;
-            for (int g = cid; g < ng && alive; g += G) {
-                const int t0 = direct_ids ? 0 : leaders[g];
-                const int a = direct_ids ? g : ids_s[t0];
-                int cnt = 0;
-                for (int base = t0; base < p.T && alive; base += 32) {
-                    const int t = base + lane;
-                    const bool match = t < p.T && ids_s[t] == a;
-                    uint32_t m = __ballot_sync(0xffffffffu, match);
-                    while (m && alive) {
-                        const int take = min(__popc(m), kTokChunk - cnt);
-                        const int rk = __popc(m & ((1u << lane) - 1u));
-                        if (((m >> lane) & 1u) && rk < take) ctl.pending[cnt + rk] = t;
-                        for (int i = 0; i < take; ++i) m &= m - 1u;
-                        cnt += take;
-                        __syncwarp();
-                        if (cnt == kTokChunk) {
-                            const int my_tok = ctl.pending[lane & (kTokChunk - 1)];
-                            __syncwarp();
-                            emit_unit(a, my_tok, cnt);
-                            cnt = 0;
-                        }
-                    }
-                }
-                if (cnt > 0 && alive) {
-                    const int my_tok = ctl.pending[lane & (kTokChunk - 1)];
-                    __syncwarp();
-                    emit_unit(a, my_tok, cnt);
-                }
             }
         }
         // end marker
@@ -452,10 +412,14 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
 
     // =================================== consumers ===================================
     int u = 0;   // units whose intermediate has been exchanged (fused / shrink modes)
+    bool cluster_waited = false;
+    bool y_staged = false;   // ys already holds the rows of the unit's first expand tile
+    const int ylen = min(W, orows);   // length of the first expand tile of this CTA
     for (int it = 0;; ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
         if (!mbar_wait(smem_u32(&ctl.meta[s]), ph, p.status)) break;
+        if (tid == 0 && it < 2) LORA_TRACE_MARK(5 + 5 * it);
         const StageHeader &hdr = *reinterpret_cast<const StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
         const int kind = hdr.kind;
         if (kind == kTileEnd) break;
@@ -463,90 +427,128 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         const uint8_t *data = stage_base + (size_t)s * p.stage_bytes + kHeaderBytes;
         const int nch = len / EPC;   // 16-byte chunks per staged row
 
-        // Load this tile's x rows (shrink) or y rows (expand) while the TMA lands: row l,
-        // 16-byte chunk c, four chunks per thread at most (16 rows x 1 KiB).
-        uint4 ld[4];
-        const int total = L * nch;
+        // Rows to stage while the TMA lands: x for a shrink tile, y for an expand tile (unless
+        // the unit's first shrink tile already brought y along).  Element e = (row l, chunk c)
+        // with c < CHUNKS; four elements per thread at most (16 rows x CHUNKS chunks).
+        const bool xy = kind == kTileShrink;
+        const bool also_y = (MODE == kModeFused) && xy && (flags & kFlagFirst) && ylen > 0;
+        const bool own = !(kind == kTileExpand && (flags & kFlagFirst) && y_staged);
+        uint4 ld[4], ldy[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int e = tid + kConsumers * i;
-            ld[i] = make_uint4(0, 0, 0, 0);
-            if (e < total) {
-                const int l = e / nch, c = e - l * nch;
+            const int l = e >> lgC, c = e & (CHUNKS - 1);
+            ld[i] = ldy[i] = make_uint4(0, 0, 0, 0);
+            if (l < L) {
                 const int64_t t = hdr.tok[l];
-                const uint8_t *src =
-                    (kind == kTileShrink)
-                        ? static_cast<const uint8_t *>(p.x) + (t * p.ldx + off) * ESZ + c * 16
-                        : static_cast<const uint8_t *>(p.y) + (t * p.ldy + p.y_off + off) * ESZ + c * 16;
-                ld[i] = *reinterpret_cast<const uint4 *>(src);
+                if (own && c < nch)
+                    ld[i] = *reinterpret_cast<const uint4 *>(
+                        xy ? static_cast<const uint8_t *>(p.x) + (t * p.ldx + off) * ESZ + c * 16
+                           : static_cast<const uint8_t *>(p.y) + (t * p.ldy + p.y_off + off) * ESZ + c * 16);
+                if (also_y && c < ylen / EPC)
+                    ldy[i] = *reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.y) +
+                                                             (t * p.ldy + p.y_off + og0 * EPC) * ESZ + c * 16);
             }
         }
         named_bar_sync(1, kConsumers);   // every consumer is done with the previous tile's buffers
-        uint8_t *stg = (kind == kTileShrink) ? xs : ys;
+        if (tid == 0 && it < 2) LORA_TRACE_MARK(6 + 5 * it);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int e = tid + kConsumers * i;
-            if (e < total) {
-                const int l = e / nch, c = e - l * nch;
-                *reinterpret_cast<uint4 *>(stg + l * rowb + c * 16) = ld[i];
+            const int l = e >> lgC, c = e & (CHUNKS - 1);
+            if (l < L) {
+                if (own && c < nch) *reinterpret_cast<uint4 *>((xy ? xs : ys) + l * rowb + c * 16) = ld[i];
+                if (also_y && c < ylen / EPC) *reinterpret_cast<uint4 *>(ys + l * rowb + c * 16) = ldy[i];
             }
         }
+        if (also_y) y_staged = true;
+        if (kind == kTileExpand) y_staged = false;
         if (!mbar_wait(smem_u32(&ctl.full[s]), ph, p.status)) break;
-        if (tid == 0) LORA_TRACE_MARK(8 + (it < 3 ? it : 3));
+        if (tid == 0 && it < 2) LORA_TRACE_MARK(7 + 5 * it);
         named_bar_sync(1, kConsumers);
+        if (tid == 0 && it < 2) LORA_TRACE_MARK(8 + 5 * it);
 
         if (kind == kTileShrink) {
             const bool first = flags & kFlagFirst;
-            // ---- partial shrink over this CTA's slice of h
-            if (warp < min(r, 8)) {
-                const int rw = (r - warp + 7) / 8;   // rows of this warp
-                if (rw >= 8) shrink_rows<E, 8>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
-                else if (rw >= 4) shrink_rows<E, 4>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
-                else if (rw >= 2) shrink_rows<E, 2>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
-                else shrink_rows<E, 1>(data, xs, rowb, vpart, RP, r, L, nch, warp, lane, first);
+            // ---- partial shrink over this CTA's slice of h: warp w owns rows w, w + 8, ...;
+            // A is staged as [box][row][512 B] (box 1 after r rows of box 0), x as [token][row].
+            const bool okA = lane < nch, okB = lane + 32 < nch;
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            if (warp < r) {
+                for (int l = 0; l < L; ++l) {
+                    const uint8_t *xr = xs + l * rowb;
+                    float xv[2 * EPC];
+                    cvt16(okA ? *reinterpret_cast<const uint4 *>(xr + lane * 16) : z, xv, (E *)nullptr);
+                    cvt16(okB ? *reinterpret_cast<const uint4 *>(xr + 512 + lane * 16) : z, xv + EPC, (E *)nullptr);
+                    for (int k = warp; k < r; k += kConsumerWarps) {
+                        const uint8_t *row = data + k * kBoxBytes;
+                        float av[2 * EPC];
+                        cvt16(okA ? *reinterpret_cast<const uint4 *>(row + lane * 16) : z, av, (E *)nullptr);
+                        cvt16(okB ? *reinterpret_cast<const uint4 *>(row + r * kBoxBytes + lane * 16) : z, av + EPC,
+                              (E *)nullptr);
+                        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                        for (int e = 0; e < EPC; ++e) {
+                            s0 = fmaf(xv[e], av[e], s0);
+                            s1 = fmaf(xv[EPC + e], av[EPC + e], s1);
+                        }
+                        const float tot = warp_sum(s0 + s1);
+                        if (lane == 0) {
+                            float *dst = vpart + l * RP + k;
+                            *dst = first ? tot : *dst + tot;
+                        }
+                    }
+                }
             }
             if (flags & kFlagLast) {
-                if (tid == 0) LORA_TRACE_MARK(12);
+                if (tid == 0) LORA_TRACE_MARK(15);
                 named_bar_sync(1, kConsumers);
+                if (tid == 0) LORA_TRACE_MARK(16);
                 // ---- push the partial into every CTA of the cluster (this one included)
+                if (!cluster_waited) {
+                    cluster_wait_acquire();   // every peer has initialised its barriers
+                    cluster_waited = true;
+                }
                 if (u >= 1 && !mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status)) break;
-                const int nq = L * RP / 4;
+                if (tid == 0) LORA_TRACE_MARK(17);
+                const int nq = L * RP / 4;            // float4 quads of the partial
+                const int lgq = ceil_log2(nq);
                 const uint32_t my_slot = smem_u32(recv + crank * kTokChunk * RP);
                 const uint32_t rbar = smem_u32(&ctl.recv);
-                for (int e = tid; e < nq * kCluster; e += kConsumers) {
-                    const int peer = e / nq, q = e - peer * nq;
-                    const float4 v = *reinterpret_cast<const float4 *>(vpart + q * 4);
-                    st_async_v4(my_slot + q * 16, rbar, peer, v);
+                for (int e = tid; e < (kCluster << lgq); e += kConsumers) {
+                    const int peer = e >> lgq, qd = e & ((1 << lgq) - 1);
+                    if (qd < nq) {
+                        const float4 v = *reinterpret_cast<const float4 *>(vpart + qd * 4);
+                        st_async_v4(my_slot + qd * 16, rbar, peer, v);
+                    }
                 }
                 if (tid == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(kCluster * nq * 16));
+                if (tid == 0) LORA_TRACE_MARK(18);
                 if (!mbar_wait_cluster(rbar, u & 1, p.status)) break;
-                if (tid == 0) LORA_TRACE_MARK(13);
-                // ---- sum the 8 partials in CTA order
-                for (int e = tid; e < L * RP; e += kConsumers) {
-                    const int k = e % RP;
-                    float acc = 0.f;
+                if (tid == 0) LORA_TRACE_MARK(19);
+                // ---- sum the 8 partials in CTA order (entries k >= r are never read)
+                for (int e = tid; e < (L << lgRP); e += kConsumers) {
+                    const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
                     if (k < r) {
+                        float acc = 0.f;
 #pragma unroll
-                        for (int j = 0; j < kCluster; ++j) acc += recv[j * kTokChunk * RP + e];
+                        for (int j = 0; j < kCluster; ++j) acc += recv[(j * kTokChunk + l) * RP + k];
+                        vsum[l * RP + k] = acc;
+                        if (MODE == kModeShrink && crank == 0) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = acc;
                     }
-                    vsum[e] = acc;
                 }
+                if (tid == 0) LORA_TRACE_MARK(20);
                 named_bar_sync(1, kConsumers);
+                if (tid == 0) LORA_TRACE_MARK(21);
                 if (tid < kCluster) mbar_arrive_remote(smem_u32(&ctl.freed), tid);
-                if (tid == 0) LORA_TRACE_MARK(14);
-                if (MODE == kModeShrink && crank == 0) {
-                    for (int e = tid; e < L * r; e += kConsumers) {
-                        const int l = e / r, k = e - l * r;
-                        p.v[(int64_t)hdr.tok[l] * p.ldv + k] = vsum[l * RP + k];
-                    }
-                }
+                if (tid == 0) LORA_TRACE_MARK(22);
                 ++u;
             }
         } else {  // kTileExpand
             if (MODE == kModeExpand && (flags & kFlagFirst)) {
-                for (int e = tid; e < L * RP; e += kConsumers) {
-                    const int l = e / RP, k = e - l * RP;
-                    vsum[e] = (k < r) ? p.v[(int64_t)hdr.tok[l] * p.ldv + k] : 0.f;
+                for (int e = tid; e < (L << lgRP); e += kConsumers) {
+                    const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
+                    if (k < r) vsum[l * RP + k] = p.v[(int64_t)hdr.tok[l] * p.ldv + k];
                 }
                 named_bar_sync(1, kConsumers);
             }
@@ -597,15 +599,15 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 }
             }
         }
-        if (tid == 0) LORA_TRACE_MARK(kind == kTileShrink ? 15 : 16);
+        if (tid == 0 && it < 2) LORA_TRACE_MARK(9 + 5 * it);
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
     }
-    if (tid == 0) LORA_TRACE_MARK(17);
+    if (tid == 0) LORA_TRACE_MARK(24);
     // No CTA may leave while a peer can still arrive on its barriers: wait until every peer
     // has released the partials of the last unit.
     if (MODE != kModeExpand && u >= 1) mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status);
-    if (tid == 0) LORA_TRACE_MARK(18);
+    if (tid == 0) LORA_TRACE_MARK(25);
 }
 
 template <typename E, int MODE, int SRC>

@@ -81,15 +81,20 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank)
                  : "memory");
 }
 
+// One bounded-time probe of a phase.  The suspend-time hint lets the hardware park the thread
+// until the phase completes (or ~0.5 ms pass) instead of spinning, so waiting warps do not take
+// issue slots from the warps that are working.
+constexpr uint32_t kSuspendHintNs = 500000u;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n .reg .pred p;\n"
-        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -99,39 +104,37 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     uint32_t ok;
     asm volatile(
         "{\n .reg .pred p;\n"
-        " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n"
         " selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
 
-// Bounded waits: false after ~2 s, with LORA_STATUS_TIMEOUT latched into *status.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status)
+// Bounded waits: false after ~2 s, with LORA_STATUS_TIMEOUT latched into *status.  The fast
+// path (phase already complete) is inlined; the polling loop is a separate function so the hot
+// code stays small (instruction-cache misses dominate short kernels).
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint32_t *status, bool cluster)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    for (;;) {
+        if (cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
             atomicOr(status, LORA_STATUS_TIMEOUT);
             return false;
         }
     }
 }
 
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status)
+{
+    return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, status, false);
+}
+
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint32_t *status)
 {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(status, LORA_STATUS_TIMEOUT);
-            return false;
-        }
-    }
+    return mbar_try_wait_cluster(bar, parity) || mbar_wait_slow(bar, parity, status, true);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -196,6 +199,23 @@ __device__ __forceinline__ uint32_t nclusters_x()
     uint32_t r;
     asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
     return r;
+}
+
+// Split cluster barrier: arrive (relaxed; pair with an explicit release fence when needed)
+// now, wait (acquire) later, so the barrier latency hides behind independent work.
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire()
+{
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bring a TMA tensor map into the descriptor cache ahead of its first use.
+__device__ __forceinline__ void prefetch_tensormap(const void *p)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(p) : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync_all()

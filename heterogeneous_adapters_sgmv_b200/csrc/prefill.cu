@@ -309,163 +309,259 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     if (warp == 1) tmem_dealloc(tmem, 64);
 }
 
-struct __align__(8) ExpandCtl {
-    uint64_t bar_b, bar_y, bar_mma;
-    uint32_t tmem_base;
-    int32_t info[6];   // valid, row0, rows, adapter, rank, scale bits
+// ----------------------------------------------------------------------------------------
+// Persistent expand: CTA b walks tiles [b * total / G, (b + 1) * total / G) of the
+// (128-token tile, 128-column tile) grid, columns fastest, so consecutive tiles share the
+// intermediate tile.  Warp roles:
+//   warp 0      producer: builds the bf16 hi + lo intermediate tile (double-buffered) when the
+//               token tile changes, and streams B_i and y tiles by TMA into a 3-stage ring;
+//   warp 1      MMA issuer (one thread) into two TMEM accumulators used alternately;
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 and columns
+//               64 ((w - 2) / 4) .. +63, adds s * acc to y in place in shared memory, then the
+//               eight warps store the tile's valid rows with coalesced 16-byte stores.
+constexpr int kEpiWarps = 8;
+constexpr int kThreadsEX = (2 + kEpiWarps) * 32;
+constexpr int kExStages = 3;
+constexpr int kExStageBytes = 16384 + 32768;           // B tile + y tile (two 64-column boxes)
+constexpr int kExVBytes = 32768;                       // hi + lo intermediate tile
+
+struct ExTileInfo {
+    int32_t row0, rows, col0, ncols, vb;
+    float scale;
 };
 
-__global__ void __launch_bounds__(kThreadsPF, 1) prefill_expand_kernel(const __grid_constant__ PrefillParams p)
+struct __align__(8) ExpandCtl {
+    uint64_t full[kExStages], empty[kExStages];
+    uint64_t vfull[2], vempty[2];
+    uint64_t accfull[2], accempty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int32_t total_m;
+    ExTileInfo info[kExStages];
+};
+
+__device__ int count_m_tiles(const PrefillParams &p)
+{
+    const int lane = threadIdx.x & 31;
+    const int nseg = min(*p.num_segs, p.max_segs);
+    int tot = 0;
+    for (int s0 = 0; s0 < nseg; s0 += 32) {
+        const int s = s0 + lane;
+        int len = 0;
+        if (s < nseg) len = max(0, min(p.seg_ptr[s + 1], p.T) - max(p.seg_ptr[s], 0));
+        int tiles = (len + kTileM - 1) / kTileM;
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, d);
+        tot += tiles;
+    }
+    return tot;
+}
+
+__global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __grid_constant__ PrefillParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *vhi = smem;                   // [128][128 B] swizzled, bf16 hi part of v
-    uint8_t *vlo = smem + 16384;           // bf16 lo part
-    uint8_t *bt = smem + 32768;            // B_i tile: 128 rows of o x 64 ranks, swizzled
-    uint8_t *yt = smem + 49152;            // y tile: two 64-column boxes [128][128 B], swizzled
-    ExpandCtl &ctl = *reinterpret_cast<ExpandCtl *>(smem + 81920);
+    uint8_t *vbuf = smem;                                    // [2][hi 16 KiB | lo 16 KiB]
+    uint8_t *ring = smem + 2 * kExVBytes;                    // [kExStages][B 16 KiB | y 32 KiB]
+    ExpandCtl &ctl = *reinterpret_cast<ExpandCtl *>(ring + kExStages * kExStageBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nt = blockIdx.x;
-    const int g = blockIdx.y;
-    const int col0 = nt * kTileN;
-    const int ncols = min(kTileN, p.o - col0);
+    const int NT = (p.o + kTileN - 1) / kTileN;
 
-    pdl_wait();
-    pdl_launch_dependents();
-
-    if (warp == 0) {
-        int s, row0 = 0, rows = 0, a = 0;
-        const bool ok = find_tile(p, g, &s, &row0, &rows, &a);
-        if (lane == 0) {
-            const bool good = ok && a >= 0 && a < p.n && rows > 0 && ncols > 0;
-            if (ok && !good && nt == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
-            ctl.info[0] = good ? 1 : 0;
-            ctl.info[1] = row0;
-            ctl.info[2] = rows;
-            ctl.info[3] = a;
-            ctl.info[4] = good ? p.desc[a].rank : 0;
-            ctl.info[5] = good ? __float_as_int(p.desc[a].scale) : 0;
-            mbar_init(smem_u32(&ctl.bar_b), 1);
-            mbar_init(smem_u32(&ctl.bar_y), 1);
-            mbar_init(smem_u32(&ctl.bar_mma), 1);
-            fence_mbar_init_cluster();
+    if (tid == 0) {
+        for (int i = 0; i < kExStages; ++i) {
+            mbar_init(smem_u32(&ctl.full[i]), 1);
+            mbar_init(smem_u32(&ctl.empty[i]), 1 + kEpiWarps);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&ctl.vfull[i]), 1);
+            mbar_init(smem_u32(&ctl.vempty[i]), 1);
+            mbar_init(smem_u32(&ctl.accfull[i]), 1);
+            mbar_init(smem_u32(&ctl.accempty[i]), kEpiWarps);
+        }
+        mbar_init(smem_u32(&ctl.mma_done), 1);
+        fence_mbar_init_cluster();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&ctl.tmem_base), 128);
+        tmem_alloc(smem_u32(&ctl.tmem_base), 256);
         tmem_relinquish();
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+    if (warp == 0) {
+        const int tm = count_m_tiles(p);
+        if (lane == 0) ctl.total_m = tm;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const bool valid = ctl.info[0] != 0;
-    const int row0 = ctl.info[1], rows = ctl.info[2], a = ctl.info[3], r = ctl.info[4];
-    const float sc = __int_as_float(ctl.info[5]);
     const uint32_t tmem = ctl.tmem_base;
+    const int total = ctl.total_m * NT;
+    const int t0 = (int)((int64_t)blockIdx.x * total / gridDim.x);
+    const int t1 = (int)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
     bool ok = true;
 
-    if (valid) {
-        if (tid == 0) {
-            const uint32_t bb = smem_u32(&ctl.bar_b), yb = smem_u32(&ctl.bar_y);
-            mbar_arrive_expect_tx(bb, 16384);
-            tma_load_2d(smem_u32(bt), p.tm_B + (size_t)a * 128, 0, col0, bb);
-            mbar_arrive_expect_tx(yb, 32768);
-            tma_load_2d(smem_u32(yt), &p.tmap_io, col0, row0, yb);
-            tma_load_2d(smem_u32(yt + 16384), &p.tmap_io, col0 + 64, row0, yb);
-        }
-        // ---- v tile: row m of the tile, split into bf16 hi + lo, 128-byte swizzle, zero past r
-        {
-            const int m = tid;
-            const bool rv = m < rows;
-            const float *vr = p.v + (int64_t)(row0 + m) * p.ldv;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int k = c * 8 + e;
-                    f[e] = (rv && k < r) ? vr[k] : 0.f;
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int cur_g = -1, vcount = 0, row0 = 0, rows = 0, a = 0, r = 0, vb = 0;
+        float sc = 0.f;
+        for (int t = t0; t < t1 && ok; ++t) {
+            const int i = t - t0, s = i % kExStages;
+            const int g = t / NT, nt = t - g * NT;
+            if (g != cur_g) {
+                int sg;
+                if (!find_tile(p, g, &sg, &row0, &rows, &a) || a < 0 || a >= p.n) {
+                    // a bad segment entry: keep the pipeline fed, store nothing for this tile
+                    if (lane == 0 && nt == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+                    row0 = 0;
+                    rows = 0;
+                    a = 0;
                 }
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(f[e], f[e + 1]);
-                    const float2 hf = __bfloat1622float2(h2);
-                    const __nv_bfloat162 l2 = __floats2bfloat162_rn(f[e] - hf.x, f[e + 1] - hf.y);
-                    hi[e / 2] = *reinterpret_cast<const uint32_t *>(&h2);
-                    lo[e / 2] = *reinterpret_cast<const uint32_t *>(&l2);
+                r = rows > 0 ? p.desc[a].rank : 0;
+                sc = p.desc[a].scale;
+                cur_g = g;
+                vb = vcount & 1;
+                if (vcount >= 2 && !mbar_wait(smem_u32(&ctl.vempty[vb]), ((vcount >> 1) - 1) & 1, p.status)) {
+                    ok = false;
+                    break;
                 }
-                *reinterpret_cast<uint4 *>(vhi + sw128_off(m, c)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(vlo + sw128_off(m, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                // intermediate tile: row m, 4 columns per lane-quarter, hi and lo bf16, swizzled
+                uint8_t *vhi = vbuf + vb * kExVBytes, *vlo = vhi + 16384;
+                for (int it2 = 0; it2 < kTileM / 2; ++it2) {
+                    const int m = it2 * 2 + (lane >> 4);
+                    const int k = (lane & 15) * 4;
+                    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (m < rows && k < r) f = *reinterpret_cast<const float4 *>(p.v + (int64_t)(row0 + m) * p.ldv + k);
+                    const __nv_bfloat162 h01 = __floats2bfloat162_rn(f.x, f.y);
+                    const __nv_bfloat162 h23 = __floats2bfloat162_rn(f.z, f.w);
+                    const float2 g01 = __bfloat1622float2(h01), g23 = __bfloat1622float2(h23);
+                    const __nv_bfloat162 l01 = __floats2bfloat162_rn(f.x - g01.x, f.y - g01.y);
+                    const __nv_bfloat162 l23 = __floats2bfloat162_rn(f.z - g23.x, f.w - g23.y);
+                    const uint32_t off = sw128_off(m, k >> 3) + ((k & 4) ? 8 : 0);
+                    *reinterpret_cast<uint2 *>(vhi + off) =
+                        make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
+                    *reinterpret_cast<uint2 *>(vlo + off) =
+                        make_uint2(*reinterpret_cast<const uint32_t *>(&l01), *reinterpret_cast<const uint32_t *>(&l23));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl.vfull[vb]));
+                ++vcount;
             }
+            if (i >= kExStages && !mbar_wait(smem_u32(&ctl.empty[s]), ((i / kExStages) - 1) & 1, p.status)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                ExTileInfo &inf = ctl.info[s];
+                inf.row0 = row0;
+                inf.rows = rows;
+                inf.col0 = nt * kTileN;
+                inf.ncols = min(kTileN, p.o - nt * kTileN);
+                inf.vb = vb;
+                inf.scale = sc;
+                uint8_t *st = ring + s * kExStageBytes;
+                const uint32_t fb = smem_u32(&ctl.full[s]);
+                mbar_arrive_expect_tx(fb, kExStageBytes);
+                tma_load_2d(smem_u32(st), p.tm_B + (size_t)a * 128, 0, nt * kTileN, fb);
+                tma_load_2d(smem_u32(st + 16384), &p.tmap_io, nt * kTileN, row0, fb);
+                tma_load_2d(smem_u32(st + 32768), &p.tmap_io, nt * kTileN + 64, row0, fb);
+            }
+            __syncwarp();
         }
-        fence_proxy_async_smem();   // generic-proxy writes of v become visible to the tensor core
-        __syncthreads();
-        if (tid == 32) {
-            // MMA issuer: acc[128 x 128] = vhi . B^T + vlo . B^T
-            if (mbar_wait(smem_u32(&ctl.bar_b), 0, p.status)) {
+        // drain: every TMA issued by this CTA has landed before shared memory is released
+        const int n = t1 - t0;
+        if (lane == 0)
+            for (int i = max(0, n - kExStages); i < n; ++i)
+                mbar_wait(smem_u32(&ctl.full[i % kExStages]), (i / kExStages) & 1, p.status);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kTileM, kTileN);
+            int vuse = 0, prev_vb = -1;
+            for (int t = t0; t < t1; ++t) {
+                const int i = t - t0, s = i % kExStages, ab = i & 1;
+                if (!mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status)) break;
+                const int vb = ctl.info[s].vb;
+                if (vb != prev_vb) {
+                    if (prev_vb >= 0) umma_commit(smem_u32(&ctl.vempty[prev_vb]));   // old tile may be rebuilt
+                    if (!mbar_wait(smem_u32(&ctl.vfull[vb]), (vuse >> 1) & 1, p.status)) break;
+                    ++vuse;
+                    prev_vb = vb;
+                }
+                if (i >= 2 && !mbar_wait(smem_u32(&ctl.accempty[ab]), ((i >> 1) - 1) & 1, p.status)) break;
                 tc_fence_after();
-                const uint32_t idesc = idesc_bf16(kTileM, kTileN);
-                const uint64_t dh = sw128_desc(smem_u32(vhi)), dl = sw128_desc(smem_u32(vlo));
-                const uint64_t db = sw128_desc(smem_u32(bt));
+                const uint8_t *st = ring + s * kExStageBytes;
+                const uint64_t dh = sw128_desc(smem_u32(vbuf + vb * kExVBytes));
+                const uint64_t dl = sw128_desc(smem_u32(vbuf + vb * kExVBytes + 16384));
+                const uint64_t db = sw128_desc(smem_u32(st));
+                const uint32_t acc = tmem + (uint32_t)(ab * kTileN);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) umma_bf16(tmem, dh + 2 * k, db + 2 * k, idesc, k != 0 ? 1u : 0u);
+                for (int k = 0; k < 4; ++k) umma_bf16(acc, dh + 2 * k, db + 2 * k, idesc, k != 0 ? 1u : 0u);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) umma_bf16(tmem, dl + 2 * k, db + 2 * k, idesc, 1u);
+                for (int k = 0; k < 4; ++k) umma_bf16(acc, dl + 2 * k, db + 2 * k, idesc, 1u);
+                umma_commit(smem_u32(&ctl.accfull[ab]));
+                umma_commit(smem_u32(&ctl.empty[s]));
             }
-            umma_commit(smem_u32(&ctl.bar_mma));
+            // every MMA of this CTA has completed before tensor memory is released
+            umma_commit(smem_u32(&ctl.mma_done));
+            mbar_wait(smem_u32(&ctl.mma_done), 0, p.status);
         }
         __syncwarp();
-        ok = mbar_wait(smem_u32(&ctl.bar_mma), 0, p.status);
-        ok = mbar_wait(smem_u32(&ctl.bar_y), 0, p.status) && ok;
-        tc_fence_after();
-        // ---- epilogue: thread m owns row m; y + s * acc, rounded once, written back in place
-        if (ok) {
-            const int m = tid;
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int half = (warp - 2) >> 2;       // column half of the tile
+        const int m = q * 32 + lane;            // row of the tile
+        const int ew = warp - 2;                // epilogue warp 0..7
+        for (int t = t0; t < t1; ++t) {
+            const int i = t - t0, s = i % kExStages, ab = i & 1;
+            if (!mbar_wait(smem_u32(&ctl.accfull[ab]), (i >> 1) & 1, p.status)) break;
+            if (!mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status)) break;
+            tc_fence_after();
+            const ExTileInfo inf = ctl.info[s];
+            uint8_t *yt = ring + s * kExStageBytes + 16384 + half * 16384;   // this half's 64-column box
 #pragma unroll 1
-            for (int c0 = 0; c0 < kTileN; c0 += 32) {
+            for (int c0 = 0; c0 < 64; c0 += 32) {
                 float acc[32];
-                tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, acc);
-                uint8_t *box = yt + (c0 >= 64 ? 16384 : 0);
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kTileN + half * 64 + c0), acc);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = ((c0 & 63) >> 3) + q;
-                    uint4 *pw = reinterpret_cast<uint4 *>(box + sw128_off(m, chunk));
+                for (int qq = 0; qq < 4; ++qq) {
+                    uint4 *pw = reinterpret_cast<uint4 *>(yt + sw128_off(m, (c0 >> 3) + qq));
                     uint4 w = *pw;
                     uint32_t *wv = reinterpret_cast<uint32_t *>(&w);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float y0 = fmaf(sc, acc[q * 8 + 2 * e], bf16_lo(wv[e]));
-                        const float y1 = fmaf(sc, acc[q * 8 + 2 * e + 1], bf16_hi(wv[e]));
+                        const float y0 = fmaf(inf.scale, acc[qq * 8 + 2 * e], bf16_lo(wv[e]));
+                        const float y1 = fmaf(inf.scale, acc[qq * 8 + 2 * e + 1], bf16_hi(wv[e]));
                         wv[e] = pack_bf16x2(y0, y1);
                     }
                     *pw = w;
                 }
             }
-        }
-        __syncthreads();
-        // ---- coalesced stores of the tile's valid rows and columns (two rows per warp step)
-        if (ok) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.accempty[ab]));
+            named_bar_sync(2, kEpiWarps * 32);   // the whole tile is updated in shared memory
+            // coalesced stores: epilogue warp ew stores rows 16 ew .. 16 ew + 15, two per step
             uint8_t *yg = static_cast<uint8_t *>(p.y);
-            for (int rr = warp * 32 + (lane >> 4); rr < warp * 32 + 32; rr += 2) {
-                const int chunk = lane & 15;
-                if (rr < rows && chunk * 8 < ncols) {
-                    const uint8_t *box = yt + (chunk >= 8 ? 16384 : 0);
+            const int chunk = lane & 15;
+#pragma unroll 1
+            for (int rr = ew * 16 + (lane >> 4); rr < ew * 16 + 16; rr += 2) {
+                if (rr < inf.rows && chunk * 8 < inf.ncols) {
+                    const uint8_t *box = ring + s * kExStageBytes + 16384 + (chunk >= 8 ? 16384 : 0);
                     const uint4 w = *reinterpret_cast<const uint4 *>(box + sw128_off(rr, chunk & 7));
-                    *reinterpret_cast<uint4 *>(yg + ((int64_t)(row0 + rr) * p.ldy + p.y_off + col0 + chunk * 8) * 2) = w;
+                    *reinterpret_cast<uint4 *>(
+                        yg + ((int64_t)(inf.row0 + rr) * p.ldy + p.y_off + inf.col0 + chunk * 8) * 2) = w;
                 }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
         }
-    }
-    if (!ok && tid == 0) {
-        // drain whatever may still be landing before shared memory is released
-        mbar_wait(smem_u32(&ctl.bar_b), 0, p.status);
-        mbar_wait(smem_u32(&ctl.bar_y), 0, p.status);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, 128);
+    if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
 // ------------------------------------------------------------------- host side
@@ -500,7 +596,7 @@ int encode_sw128(CUtensorMap *out, const void *base, uint64_t cols, uint64_t row
 }
 
 constexpr int kShrinkSmem = kStages * (kTileM * 128 + kMaxRankPF * 128) + 256 + 1024;
-constexpr int kExpandSmem = 81920 + 256 + 1024;
+constexpr int kExpandSmem = 2 * kExVBytes + kExStages * kExStageBytes + (int)sizeof(ExpandCtl) + 1024;
 static_assert(kStages * (kTileM * 128 + kMaxRankPF * 128) >= kTileM * (kMaxRankPF + 4) * 4, "partial fits ring");
 
 }  // namespace
@@ -592,14 +688,17 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
         cfg.numAttrs = na;
         if (cudaLaunchKernelEx(&cfg, prefill_shrink_kernel, p) != cudaSuccess) return LORA_ERR_CUDA;
     }
-    // expand: one CTA per (128-token tile, 128-column tile)
+    // expand: persistent, one CTA per SM over all (128-token tile, 128-column tile) pairs
     rc = encode_sw128(&p.tmap_io, static_cast<uint8_t *>(y) + (int64_t)y_off * 2, (uint64_t)t->o, (uint64_t)seg->T,
                       (uint64_t)ldy, kTileM);
     if (rc != LORA_OK) return rc;
     {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((t->o + kTileN - 1) / kTileN, mt_bound);
-        cfg.blockDim = dim3(kThreadsPF);
+        static int n_sms[64];
+        if (!n_sms[dev]) cudaDeviceGetAttribute(&n_sms[dev], cudaDevAttrMultiProcessorCount, dev);
+        const int tiles_bound = mt_bound * ((t->o + kTileN - 1) / kTileN);
+        cfg.gridDim = dim3(max(1, min(n_sms[dev], tiles_bound)));
+        cfg.blockDim = dim3(kThreadsEX);
         cfg.dynamicSmemBytes = kExpandSmem;
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
