@@ -426,6 +426,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         const int r = hdr.rank, L = hdr.L, flags = hdr.flags, len = hdr.len, off = hdr.off;
         const uint8_t *data = stage_base + (size_t)s * p.stage_bytes + kHeaderBytes;
         const int nch = len / EPC;   // 16-byte chunks per staged row
+        if (tid == 0 && u < 8 && kind == kTileShrink && (flags & kFlagFirst)) LORA_TRACE_MARK(32 + 4 * u);
 
         // Rows to stage while the TMA lands: x for a shrink tile, y for an expand tile (unless
         // the unit's first shrink tile already brought y along).  Element e = (row l, chunk c)
@@ -502,6 +503,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             }
             if (flags & kFlagLast) {
                 if (tid == 0) LORA_TRACE_MARK(15);
+                if (tid == 0 && u < 8) LORA_TRACE_MARK(33 + 4 * u);
                 named_bar_sync(1, kConsumers);
                 if (tid == 0) LORA_TRACE_MARK(16);
                 // ---- push the partial into every CTA of the cluster (this one included)
@@ -540,8 +542,9 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 if (tid == 0) LORA_TRACE_MARK(20);
                 named_bar_sync(1, kConsumers);
                 if (tid == 0) LORA_TRACE_MARK(21);
-                if (tid < kCluster) mbar_arrive_remote(smem_u32(&ctl.freed), tid);
+                if (tid < kCluster) mbar_arrive_remote_relaxed(smem_u32(&ctl.freed), tid);
                 if (tid == 0) LORA_TRACE_MARK(22);
+                if (tid == 0 && u < 8) LORA_TRACE_MARK(34 + 4 * u);
                 ++u;
             }
         } else {  // kTileExpand
@@ -600,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             }
         }
         if (tid == 0 && it < 2) LORA_TRACE_MARK(9 + 5 * it);
+        if (tid == 0 && kind == kTileExpand && (flags & kFlagLast) && u >= 1 && u <= 8) LORA_TRACE_MARK(35 + 4 * (u - 1));
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
     }

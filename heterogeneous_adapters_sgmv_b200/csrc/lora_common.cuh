@@ -86,6 +86,16 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar, uint32_t rank)
 // issue slots from the warps that are working.
 constexpr uint32_t kSuspendHintNs = 500000u;
 
+// Arrive on a peer's barrier without release semantics: for signals whose preceding accesses
+// are loads whose values have already been consumed (nothing left to order), this avoids a
+// cluster-scope fence behind unrelated outstanding stores.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar, uint32_t rank)
+{
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(bar), "r"(rank));
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
@@ -266,7 +276,7 @@ __device__ __forceinline__ void pdl_launch_dependents()
 
 #ifdef LORA_TRACE
 constexpr int kTraceCtas = 4096;
-constexpr int kTraceSlots = 32;
+constexpr int kTraceSlots = 64;
 // defined (once) by the translation unit that uses the marks
 #define LORA_TRACE_MARK(slot)                                                              \
     do {                                                                                   \

@@ -427,11 +427,20 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 }
                 // intermediate tile: row m, 4 columns per lane-quarter, hi and lo bf16, swizzled
                 uint8_t *vhi = vbuf + vb * kExVBytes, *vlo = vhi + 16384;
-                for (int it2 = 0; it2 < kTileM / 2; ++it2) {
-                    const int m = it2 * 2 + (lane >> 4);
-                    const int k = (lane & 15) * 4;
-                    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (m < rows && k < r) f = *reinterpret_cast<const float4 *>(p.v + (int64_t)(row0 + m) * p.ldv + k);
+                const int k = (lane & 15) * 4;
+                for (int b0 = 0; b0 < kTileM / 2; b0 += 16) {
+                    // 16 independent loads in flight, then convert: one round trip per batch
+                    float4 fb[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int m = (b0 + j) * 2 + (lane >> 4);
+                        fb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (m < rows && k < r) fb[j] = *reinterpret_cast<const float4 *>(p.v + (int64_t)(row0 + m) * p.ldv + k);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                    const int m = (b0 + j) * 2 + (lane >> 4);
+                    const float4 f = fb[j];
                     const __nv_bfloat162 h01 = __floats2bfloat162_rn(f.x, f.y);
                     const __nv_bfloat162 h23 = __floats2bfloat162_rn(f.z, f.w);
                     const float2 g01 = __bfloat1622float2(h01), g23 = __bfloat1622float2(h23);
@@ -442,6 +451,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                         make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
                     *reinterpret_cast<uint2 *>(vlo + off) =
                         make_uint2(*reinterpret_cast<const uint32_t *>(&l01), *reinterpret_cast<const uint32_t *>(&l23));
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
