@@ -4,11 +4,13 @@
 // "TGI Multi-LoRA" page, "Technical Foundation: LoRA").
 //
 // Design for sm_100a:
-//  * A cluster of 8 CTAs owns one work unit at a time: up to 16 tokens of one adapter (one
-//    SGMV segment chunk, or one group of equal ids in the per-token BGMV form).  CTA j of the
-//    cluster streams the j-th eighth of h for the shrink and the j-th eighth of o for the
-//    expand, so each adapter's A_i and B_i are read once per unit and every token of the unit
-//    reuses that read.
+//  * A cluster of CL CTAs (CL = 8, 4, 2 or 1, picked per launch from the number of work units)
+//    owns one work unit at a time: up to 16 tokens of one adapter (one SGMV segment chunk, or
+//    one group of equal ids in the per-token BGMV form).  CTA j of the cluster streams the j-th
+//    CL-th of h for the shrink and the j-th CL-th of o for the expand, so each adapter's A_i
+//    and B_i are read once per unit and every token of the unit reuses that read.  Few units
+//    (a small decode batch) take wide clusters so every SM streams; many units take narrow
+//    ones so units run side by side instead of one after another.
 //  * One producer warp per CTA runs ahead across units: it stages this CTA's slice of A_i with
 //    2-D tensor-map TMA loads (one or two instructions per unit) and its slice of B_i with one
 //    bulk copy, into a ring of shared-memory stages guarded by mbarriers, and hints the unit's
@@ -17,8 +19,9 @@
 //    warp-level split-K; a warp owns rank rows k = warp + 8 i, a lane 16 bytes at two places of
 //    each 1 KiB row; each dot product is folded across the warp with a 5-step butterfly.
 //  * Each CTA pushes its partial intermediate into every peer's shared memory with st.async
-//    (completion counted in bytes on the peer's mbarrier); every CTA then sums the 8 partials in
-//    fixed CTA order.  No atomics, no grid barrier: bit-identical run to run.
+//    (completion counted in bytes on the peer's mbarrier); every CTA then sums the CL partials
+//    in fixed CTA order.  No atomics, no grid barrier: bit-identical run to run.  A cluster of
+//    one keeps its own sum and exchanges nothing.
 //  * Expand: a thread owns two output columns (bf16) and walks the unit's tokens; one rounding
 //    (nearest-even) per output, coalesced 32-bit stores.
 //  * Short kernels like this one are dominated by instruction fetch, so the per-unit code is
@@ -41,7 +44,7 @@ __device__ unsigned long long lora_trace_buf[kTraceCtas * kTraceSlots];
 #endif
 namespace {
 
-constexpr int kCluster = 8;
+constexpr int kMaxCluster = 8;
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;   // + one producer warp
@@ -91,7 +94,7 @@ struct Layout {
 
 __host__ __device__ inline int row_bytes_for(int R) { return R > 64 ? kRowBytes / 2 : kRowBytes; }
 
-__host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int stages, int stage_bytes)
+__host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int stages, int stage_bytes, int CL)
 {
     Layout l;
     const int rowb = row_bytes_for(R);
@@ -102,8 +105,13 @@ __host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int 
     l.ys_off = l.xs_off + kTokChunk * rowb;
     l.vpart_off = l.ys_off + kTokChunk * rowb;
     l.recv_off = l.vpart_off + round_up(kTokChunk * l.RP * 4, 128);
-    l.vsum_off = l.recv_off + kCluster * kTokChunk * l.RP * 4;
-    l.stage_off = l.vsum_off + round_up(kTokChunk * l.RP * 4, 128);
+    if (CL > 1) {
+        l.vsum_off = l.recv_off + CL * kTokChunk * l.RP * 4;
+        l.stage_off = l.vsum_off + round_up(kTokChunk * l.RP * 4, 128);
+    } else {   // no exchange: the CTA's own partial is the unit's intermediate
+        l.recv_off = l.vsum_off = l.vpart_off;
+        l.stage_off = l.vpart_off + round_up(kTokChunk * l.RP * 4, 128);
+    }
     l.total = l.stage_off + stages * stage_bytes;
     return l;
 }
@@ -132,7 +140,7 @@ __device__ __forceinline__ float warp_sum(float v)
 
 __device__ __forceinline__ int ceil_log2(int v) { return v <= 1 ? 0 : 32 - __clz(v - 1); }
 
-template <typename E, int MODE, int SRC>
+template <typename E, int MODE, int SRC, int CL>
 __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_constant__ DecodeParams p)
 {
     using T_ = Tr<E>;
@@ -145,11 +153,11 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
 
     extern __shared__ __align__(128) uint8_t smem[];
     SmemCtl &ctl = *reinterpret_cast<SmemCtl *>(smem);
-    const Layout lay = make_layout(SRC, p.R, p.n, p.T, p.stages, p.stage_bytes);
+    const Layout lay = make_layout(SRC, p.R, p.n, p.T, p.stages, p.stage_bytes, CL);
     uint8_t *xs = smem + lay.xs_off;
     uint8_t *ys = smem + lay.ys_off;
     float *vpart = reinterpret_cast<float *>(smem + lay.vpart_off);   // [kTokChunk][RP] this CTA's partial
-    float *recv = reinterpret_cast<float *>(smem + lay.recv_off);     // [kCluster][kTokChunk][RP] from peers
+    float *recv = reinterpret_cast<float *>(smem + lay.recv_off);     // [CL][kTokChunk][RP] from peers
     float *vsum = reinterpret_cast<float *>(smem + lay.vsum_off);     // [kTokChunk][RP] the unit's intermediate
     uint8_t *stage_base = smem + lay.stage_off;
     const int RP = lay.RP;
@@ -169,11 +177,11 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             mbar_init(smem_u32(&ctl.empty[s]), kConsumerWarps);
         }
         mbar_init(smem_u32(&ctl.recv), 1);
-        mbar_init(smem_u32(&ctl.freed), kCluster);
+        mbar_init(smem_u32(&ctl.freed), CL);
         fence_mbar_init_cluster();
     }
     __syncthreads();            // barriers initialised for this CTA
-    cluster_arrive_relaxed();   // peers wait for this before their first remote access to us
+    if (CL > 1) cluster_arrive_relaxed();   // peers wait for this before their first remote access
 
     // Per-token ids: tokens with equal ids form one group.  With no more adapters than
     // clusters, cluster c owns adapter c and its producer scans the ids itself; otherwise a
@@ -223,10 +231,10 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
 
     // h and o ranges of this CTA, in 16-byte chunks of h and EPC-row groups of o
     const int hchunks = p.h / EPC, ogroups = p.o / EPC;
-    const int hc0 = (int)((int64_t)crank * hchunks / kCluster);
-    const int hc1 = (int)((int64_t)(crank + 1) * hchunks / kCluster);
-    const int og0 = (int)((int64_t)crank * ogroups / kCluster);
-    const int og1 = (int)((int64_t)(crank + 1) * ogroups / kCluster);
+    const int hc0 = (int)((int64_t)crank * hchunks / CL);
+    const int hc1 = (int)((int64_t)(crank + 1) * hchunks / CL);
+    const int og0 = (int)((int64_t)crank * ogroups / CL);
+    const int og1 = (int)((int64_t)(crank + 1) * ogroups / CL);
     const int n_shrink = (MODE == kModeExpand) ? 0 : max(1, (hc1 - hc0 + CHUNKS - 1) / CHUNKS);
     const int orows = (og1 - og0) * EPC;
     const int n_expand = (MODE == kModeShrink) ? 0 : (orows + W - 1) / W;
@@ -248,22 +256,51 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             __syncwarp();
         }
         // Walk this cluster's units; each yields (adapter, descriptor, tokens in lanes 0..L-1).
-        int seg = cid, q = 0, g = cid, base = -1, cnt = 0;
+        // Segment tables: units are the 16-token chunks of the segments, numbered segment by
+        // segment, and cluster c takes units c, c + G, ... so a long segment spreads over many
+        // clusters.  The warp holds a window of 32 segments (lane l: segment sb + l) with the
+        // inclusive prefix count of their units and slides it forward as units are taken.
+        const int nseg = (SRC == kSrcSegments) ? min(*p.num_segs, p.max_segs) : 0;
+        int sb = -32, ubase = 0, w_p0 = 0, w_p1 = 0, w_sa = -1, w_nu = 0, w_incl = 0, w_total = 0;
+        int un = cid;
+        int g = cid, base = -1, cnt = 0;
         for (;;) {
             int a = -1, my_tok = 0, L = 0;
             AdapterDesc d = {};
             if (SRC == kSrcSegments) {
-                const int nseg = min(*p.num_segs, p.max_segs);
-                while (seg < nseg && L == 0) {
-                    const int sa = p.seg_adapter[seg];
-                    const int p0 = p.seg_ptr[seg], p1 = p.seg_ptr[seg + 1];
-                    if (sa < 0 || sa >= p.n || p0 < 0 || p1 < p0 || p1 > p.T) {
-                        if (lane == 0 && crank == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
-                        seg += G;
-                        q = 0;
-                        continue;
+                while (L == 0) {
+                    while (un >= ubase + w_total && sb + 32 < nseg) {
+                        ubase += w_total;
+                        sb += 32;
+                        const int sg = sb + lane;
+                        w_nu = 0;
+                        w_sa = -1;
+                        w_p0 = w_p1 = 0;
+                        if (sg < nseg) {
+                            w_sa = p.seg_adapter[sg];
+                            w_p0 = p.seg_ptr[sg];
+                            w_p1 = p.seg_ptr[sg + 1];
+                            if (w_sa >= 0 && w_sa < p.n && w_p0 >= 0 && w_p1 >= w_p0 && w_p1 <= p.T)
+                                w_nu = (w_p1 - w_p0 + kTokChunk - 1) / kTokChunk;
+                            else if (cid == 0 && crank == 0)   // every cluster scans every segment
+                                atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+                        }
+                        w_incl = w_nu;
+#pragma unroll
+                        for (int dl = 1; dl < 32; dl <<= 1) {
+                            const int v = __shfl_up_sync(0xffffffffu, w_incl, dl);
+                            if (lane >= dl) w_incl += v;
+                        }
+                        w_total = __shfl_sync(0xffffffffu, w_incl, 31);
                     }
-                    const int start = p0 + q;
+                    if (un >= ubase + w_total) break;   // this cluster has no units left
+                    const int hl = __ffs(__ballot_sync(0xffffffffu, ubase + w_incl > un)) - 1;
+                    const int sa = __shfl_sync(0xffffffffu, w_sa, hl);
+                    const int p1 = __shfl_sync(0xffffffffu, w_p1, hl);
+                    const int first_unit = ubase + __shfl_sync(0xffffffffu, w_incl - w_nu, hl);
+                    const int start = __shfl_sync(0xffffffffu, w_p0, hl) + (un - first_unit) * kTokChunk;
+                    un += G;
+                    d = p.desc[sa];
                     const int L0 = min(kTokChunk, p1 - start);
                     int t = -1;
                     if (lane < L0) t = p.perm ? p.perm[start + lane] : start + lane;
@@ -279,13 +316,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     __syncwarp();
                     L = __popc(m);
                     a = sa;
-                    q += kTokChunk;
-                    if (p0 + q >= p1) {
-                        seg += G;
-                        q = 0;
-                    }
                 }
-                if (L > 0) d = p.desc[a];
             } else {
                 const int ng = direct_ids ? min(p.n, cid + 1) : ctl.n_groups;
                 while (g < ng && L == 0) {
@@ -411,16 +442,37 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     }
 
     // =================================== consumers ===================================
+    // The global rows a tile reads (x for a shrink tile, y for an expand tile) are loaded into
+    // registers while the previous tile computes, and written to shared memory once every
+    // consumer is done with that tile.  Element e = (row l, chunk c) with c < CHUNKS; four per
+    // thread at most (16 rows x CHUNKS chunks).
     int u = 0;   // units whose intermediate has been exchanged (fused / shrink modes)
     bool cluster_waited = false;
-    bool y_staged = false;   // ys already holds the rows of the unit's first expand tile
-    const int ylen = min(W, orows);   // length of the first expand tile of this CTA
-    for (int it = 0;; ++it) {
+    uint4 ld[4];
+    auto stage_header = [&](int i) -> const StageHeader & {
+        return *reinterpret_cast<const StageHeader *>(stage_base + (size_t)(i % S) * p.stage_bytes);
+    };
+    auto load_rows = [&](const StageHeader &h) {
+        const bool xr = h.kind == kTileShrink;
+        const int L = h.L, nch = h.len / EPC;
+        const uint8_t *src = xr ? static_cast<const uint8_t *>(p.x) + (int64_t)h.off * ESZ
+                                : static_cast<const uint8_t *>(p.y) + ((int64_t)p.y_off + h.off) * ESZ;
+        const int64_t ld_row = (xr ? p.ldx : p.ldy) * ESZ;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int e = tid + kConsumers * i;
+            const int l = e >> lgC, c = e & (CHUNKS - 1);
+            ld[i] = make_uint4(0, 0, 0, 0);
+            if (l < L && c < nch) ld[i] = *reinterpret_cast<const uint4 *>(src + h.tok[l] * ld_row + c * 16);
+        }
+    };
+    bool live = mbar_wait(smem_u32(&ctl.meta[0]), 0, p.status);
+    if (live && stage_header(0).kind != kTileEnd) load_rows(stage_header(0));
+    for (int it = 0; live; ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!mbar_wait(smem_u32(&ctl.meta[s]), ph, p.status)) break;
         if (tid == 0 && it < 2) LORA_TRACE_MARK(5 + 5 * it);
-        const StageHeader &hdr = *reinterpret_cast<const StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
+        const StageHeader &hdr = stage_header(it);
         const int kind = hdr.kind;
         if (kind == kTileEnd) break;
         const int r = hdr.rank, L = hdr.L, flags = hdr.flags, len = hdr.len, off = hdr.off;
@@ -428,42 +480,19 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         const int nch = len / EPC;   // 16-byte chunks per staged row
         if (tid == 0 && u < 8 && kind == kTileShrink && (flags & kFlagFirst)) LORA_TRACE_MARK(32 + 4 * u);
 
-        // Rows to stage while the TMA lands: x for a shrink tile, y for an expand tile (unless
-        // the unit's first shrink tile already brought y along).  Element e = (row l, chunk c)
-        // with c < CHUNKS; four elements per thread at most (16 rows x CHUNKS chunks).
-        const bool xy = kind == kTileShrink;
-        const bool also_y = (MODE == kModeFused) && xy && (flags & kFlagFirst) && ylen > 0;
-        const bool own = !(kind == kTileExpand && (flags & kFlagFirst) && y_staged);
-        uint4 ld[4], ldy[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int e = tid + kConsumers * i;
-            const int l = e >> lgC, c = e & (CHUNKS - 1);
-            ld[i] = ldy[i] = make_uint4(0, 0, 0, 0);
-            if (l < L) {
-                const int64_t t = hdr.tok[l];
-                if (own && c < nch)
-                    ld[i] = *reinterpret_cast<const uint4 *>(
-                        xy ? static_cast<const uint8_t *>(p.x) + (t * p.ldx + off) * ESZ + c * 16
-                           : static_cast<const uint8_t *>(p.y) + (t * p.ldy + p.y_off + off) * ESZ + c * 16);
-                if (also_y && c < ylen / EPC)
-                    ldy[i] = *reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.y) +
-                                                             (t * p.ldy + p.y_off + og0 * EPC) * ESZ + c * 16);
-            }
-        }
         named_bar_sync(1, kConsumers);   // every consumer is done with the previous tile's buffers
         if (tid == 0 && it < 2) LORA_TRACE_MARK(6 + 5 * it);
+        uint8_t *rows = kind == kTileShrink ? xs : ys;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int e = tid + kConsumers * i;
             const int l = e >> lgC, c = e & (CHUNKS - 1);
-            if (l < L) {
-                if (own && c < nch) *reinterpret_cast<uint4 *>((xy ? xs : ys) + l * rowb + c * 16) = ld[i];
-                if (also_y && c < ylen / EPC) *reinterpret_cast<uint4 *>(ys + l * rowb + c * 16) = ldy[i];
-            }
+            if (l < L && c < nch) *reinterpret_cast<uint4 *>(rows + l * rowb + c * 16) = ld[i];
         }
-        if (also_y) y_staged = true;
-        if (kind == kTileExpand) y_staged = false;
+        // next tile's rows (its stage was released S - 1 tiles ago, so its header comes
+        // without waiting on this tile)
+        if (!mbar_wait(smem_u32(&ctl.meta[(it + 1) % S]), ((it + 1) / S) & 1, p.status)) break;
+        if (stage_header(it + 1).kind != kTileEnd) load_rows(stage_header(it + 1));
         if (!mbar_wait(smem_u32(&ctl.full[s]), ph, p.status)) break;
         if (tid == 0 && it < 2) LORA_TRACE_MARK(7 + 5 * it);
         named_bar_sync(1, kConsumers);
@@ -506,44 +535,54 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 if (tid == 0 && u < 8) LORA_TRACE_MARK(33 + 4 * u);
                 named_bar_sync(1, kConsumers);
                 if (tid == 0) LORA_TRACE_MARK(16);
-                // ---- push the partial into every CTA of the cluster (this one included)
-                if (!cluster_waited) {
-                    cluster_wait_acquire();   // every peer has initialised its barriers
-                    cluster_waited = true;
-                }
-                if (u >= 1 && !mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status)) break;
-                if (tid == 0) LORA_TRACE_MARK(17);
-                const int nq = L * RP / 4;            // float4 quads of the partial
-                const int lgq = ceil_log2(nq);
-                const uint32_t my_slot = smem_u32(recv + crank * kTokChunk * RP);
-                const uint32_t rbar = smem_u32(&ctl.recv);
-                for (int e = tid; e < (kCluster << lgq); e += kConsumers) {
-                    const int peer = e >> lgq, qd = e & ((1 << lgq) - 1);
-                    if (qd < nq) {
-                        const float4 v = *reinterpret_cast<const float4 *>(vpart + qd * 4);
-                        st_async_v4(my_slot + qd * 16, rbar, peer, v);
+                if constexpr (CL == 1) {
+                    // ---- no peers: vpart (= vsum) already holds the unit's intermediate
+                    if (MODE == kModeShrink) {
+                        for (int e = tid; e < (L << lgRP); e += kConsumers) {
+                            const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
+                            if (k < r) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = vsum[l * RP + k];
+                        }
                     }
-                }
-                if (tid == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(kCluster * nq * 16));
-                if (tid == 0) LORA_TRACE_MARK(18);
-                if (!mbar_wait_cluster(rbar, u & 1, p.status)) break;
-                if (tid == 0) LORA_TRACE_MARK(19);
-                // ---- sum the 8 partials in CTA order (entries k >= r are never read)
-                for (int e = tid; e < (L << lgRP); e += kConsumers) {
-                    const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
-                    if (k < r) {
-                        float acc = 0.f;
+                } else {
+                    // ---- push the partial into every CTA of the cluster (this one included)
+                    if (!cluster_waited) {
+                        cluster_wait_acquire();   // every peer has initialised its barriers
+                        cluster_waited = true;
+                    }
+                    if (u >= 1 && !mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status)) break;
+                    if (tid == 0) LORA_TRACE_MARK(17);
+                    const int nq = L * RP / 4;            // float4 quads of the partial
+                    const int lgq = ceil_log2(nq);
+                    const uint32_t my_slot = smem_u32(recv + crank * kTokChunk * RP);
+                    const uint32_t rbar = smem_u32(&ctl.recv);
+                    for (int e = tid; e < (CL << lgq); e += kConsumers) {
+                        const int peer = e >> lgq, qd = e & ((1 << lgq) - 1);
+                        if (qd < nq) {
+                            const float4 v = *reinterpret_cast<const float4 *>(vpart + qd * 4);
+                            st_async_v4(my_slot + qd * 16, rbar, peer, v);
+                        }
+                    }
+                    if (tid == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(CL * nq * 16));
+                    if (tid == 0) LORA_TRACE_MARK(18);
+                    if (!mbar_wait_cluster(rbar, u & 1, p.status)) break;
+                    if (tid == 0) LORA_TRACE_MARK(19);
+                    // ---- sum the CL partials in CTA order (entries k >= r are never read)
+                    for (int e = tid; e < (L << lgRP); e += kConsumers) {
+                        const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
+                        if (k < r) {
+                            float acc = 0.f;
 #pragma unroll
-                        for (int j = 0; j < kCluster; ++j) acc += recv[(j * kTokChunk + l) * RP + k];
-                        vsum[l * RP + k] = acc;
-                        if (MODE == kModeShrink && crank == 0) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = acc;
+                            for (int j = 0; j < CL; ++j) acc += recv[(j * kTokChunk + l) * RP + k];
+                            vsum[l * RP + k] = acc;
+                            if (MODE == kModeShrink && crank == 0) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = acc;
+                        }
                     }
+                    if (tid == 0) LORA_TRACE_MARK(20);
+                    named_bar_sync(1, kConsumers);
+                    if (tid == 0) LORA_TRACE_MARK(21);
+                    if (tid < CL) mbar_arrive_remote_relaxed(smem_u32(&ctl.freed), tid);
+                    if (tid == 0) LORA_TRACE_MARK(22);
                 }
-                if (tid == 0) LORA_TRACE_MARK(20);
-                named_bar_sync(1, kConsumers);
-                if (tid == 0) LORA_TRACE_MARK(21);
-                if (tid < kCluster) mbar_arrive_remote_relaxed(smem_u32(&ctl.freed), tid);
-                if (tid == 0) LORA_TRACE_MARK(22);
                 if (tid == 0 && u < 8) LORA_TRACE_MARK(34 + 4 * u);
                 ++u;
             }
@@ -610,15 +649,19 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     if (tid == 0) LORA_TRACE_MARK(24);
     // No CTA may leave while a peer can still arrive on its barriers: wait until every peer
     // has released the partials of the last unit.
-    if (MODE != kModeExpand && u >= 1) mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status);
+    if (CL > 1 && MODE != kModeExpand && u >= 1) mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status);
     if (tid == 0) LORA_TRACE_MARK(25);
 }
 
-template <typename E, int MODE, int SRC>
-int launch_one(const DecodeParams &p0, cudaStream_t s)
+// Shared-memory size, pipeline depth and co-resident cluster count of one instantiation.
+struct LaunchShape {
+    int stages, stage_bytes, smem, clusters;
+};
+
+template <typename E, int MODE, int SRC, int CL>
+int launch_shape(const DecodeParams &p, LaunchShape &ls)
 {
-    auto kern = lora_decode_kernel<E, MODE, SRC>;
-    DecodeParams p = p0;
+    auto kern = lora_decode_kernel<E, MODE, SRC, CL>;
     const Options &opt = options();
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LORA_ERR_CUDA;
@@ -632,72 +675,124 @@ int launch_one(const DecodeParams &p0, cudaStream_t s)
     });
     // Pipeline depth: aim for two CTAs per SM unless told otherwise.
     const int stage_bytes = kHeaderBytes + p.R * row_bytes_for(p.R);
-    const int fixed = make_layout(SRC, p.R, p.n, p.T, 0, stage_bytes).total;
+    const int fixed = make_layout(SRC, p.R, p.n, p.T, 0, stage_bytes, CL).total;
     const int ctas_per_sm = opt.decode_ctas_per_sm > 0 ? (int)opt.decode_ctas_per_sm : 2;
     int stages = (int)opt.decode_stages;
     if (stages <= 0) {
         const int budget = (228 * 1024) / ctas_per_sm - 1024 - fixed;
         stages = max(2, min(kMaxStages, budget / stage_bytes));
     }
-    stages = max(1, min(kMaxStages, stages));
-    while (stages > 1 && make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes).total > max_optin[dev]) --stages;
-    const Layout lay = make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes);
+    // at least two stages: consumers read the next tile's header before releasing this one
+    stages = max(2, min(kMaxStages, stages));
+    while (stages > 2 && make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes, CL).total > max_optin[dev]) --stages;
+    const Layout lay = make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes, CL);
     if (lay.total > max_optin[dev]) return LORA_ERR_UNSUPPORTED;
-    p.stages = stages;
-    p.stage_bytes = stage_bytes;
     static int smem_set[64];
     if (smem_set[dev] < lay.total) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total) != cudaSuccess)
             return LORA_ERR_CUDA;
         smem_set[dev] = lay.total;
     }
+    // co-resident clusters for this shared-memory size (cached: a host query, not a stream op)
+    static int occ_smem[64], occ_clusters[64];
+    if (occ_smem[dev] != lay.total) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = CL;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.blockDim = dim3(kThreads);
+        cfg.gridDim = dim3(CL);
+        cfg.dynamicSmemBytes = (size_t)lay.total;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int mc = 0;
+        if (cudaOccupancyMaxActiveClusters(&mc, (void *)kern, &cfg) != cudaSuccess || mc < 1)
+            mc = max(1, n_sms[dev] / CL);
+        occ_clusters[dev] = mc;
+        occ_smem[dev] = lay.total;
+    }
+    ls.stages = stages;
+    ls.stage_bytes = stage_bytes;
+    ls.smem = lay.total;
+    ls.clusters = occ_clusters[dev];
+    return LORA_OK;
+}
 
+template <typename E, int MODE, int SRC, int CL>
+int launch_one(const DecodeParams &p0, int units, cudaStream_t s)
+{
+    auto kern = lora_decode_kernel<E, MODE, SRC, CL>;
+    LaunchShape ls;
+    const int rc = launch_shape<E, MODE, SRC, CL>(p0, ls);
+    if (rc != LORA_OK) return rc;
+    DecodeParams p = p0;
+    p.stages = ls.stages;
+    p.stage_bytes = ls.stage_bytes;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)lay.total;
+    cfg.dynamicSmemBytes = (size_t)ls.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     int na = 0;
     attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = kCluster;
+    attr[na].val.clusterDim.x = CL;
     attr[na].val.clusterDim.y = 1;
     attr[na].val.clusterDim.z = 1;
     ++na;
-    cfg.attrs = attr;
-    cfg.numAttrs = na;
-    cfg.gridDim = dim3(kCluster);
-    // co-resident clusters for this shared-memory size (cached: a host query, not a stream op)
-    static int occ_smem[64], occ_clusters[64];
-    if (occ_smem[dev] != lay.total) {
-        int mc = 0;
-        if (cudaOccupancyMaxActiveClusters(&mc, (void *)kern, &cfg) != cudaSuccess || mc < 1)
-            mc = max(1, n_sms[dev] / kCluster);
-        occ_clusters[dev] = mc;
-        occ_smem[dev] = lay.total;
-    }
-    const int max_clusters = occ_clusters[dev];
-    const int units_bound = max(1, min(p.T, (SRC == kSrcSegments) ? p.max_segs : p.n));
-    const int G = max(1, min(max_clusters, units_bound));
-    cfg.gridDim = dim3(G * kCluster);
-    if (opt.pdl) {
+    if (options().pdl) {
         attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[na].val.programmaticStreamSerializationAllowed = 1;
         ++na;
     }
+    cfg.attrs = attr;
     cfg.numAttrs = na;
+    const int G = max(1, min(ls.clusters, units));
+    cfg.gridDim = dim3(G * CL);
     if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return LORA_ERR_CUDA;
     return LORA_OK;
+}
+
+// Cluster width for a launch: 8 CTAs share each unit unless the "decode_cluster" option asks
+// for fewer (1, 2 or 4).  Narrow clusters run more units side by side but stream each unit's
+// weights through fewer SMs; measured on the decode workloads here, 8 was never slower.
+template <typename E, int MODE, int SRC>
+int launch_mode(const DecodeParams &p, cudaStream_t s)
+{
+    // units: an upper bound on the work units (16-token chunks of one adapter's tokens)
+    const int units = max(1, (SRC == kSrcSegments) ? min(p.T, p.max_segs + (p.T + kTokChunk - 1) / kTokChunk)
+                                                   : min(p.T, p.n));
+    const int64_t forced = options().decode_cluster;
+    int CL = (forced == 1 || forced == 2 || forced == 4) ? (int)forced : kMaxCluster;
+    // The widest width whose pipeline fits in shared memory (the partial-exchange buffers grow
+    // with the width).
+    for (;; CL >>= 1) {
+        LaunchShape ls;
+        int rc = LORA_OK;
+        if (CL == 8) rc = launch_shape<E, MODE, SRC, 8>(p, ls);
+        else if (CL == 4) rc = launch_shape<E, MODE, SRC, 4>(p, ls);
+        else if (CL == 2) rc = launch_shape<E, MODE, SRC, 2>(p, ls);
+        else rc = launch_shape<E, MODE, SRC, 1>(p, ls);
+        if (rc == LORA_OK || CL == 1 || rc != LORA_ERR_UNSUPPORTED) break;
+    }
+    switch (CL) {
+    case 8: return launch_one<E, MODE, SRC, 8>(p, units, s);
+    case 4: return launch_one<E, MODE, SRC, 4>(p, units, s);
+    case 2: return launch_one<E, MODE, SRC, 2>(p, units, s);
+    default: return launch_one<E, MODE, SRC, 1>(p, units, s);
+    }
 }
 
 template <typename E>
 int launch_typed(int mode, int src, const DecodeParams &p, cudaStream_t s)
 {
     if (src == kSrcSegments) {
-        if (mode == kModeFused) return launch_one<E, kModeFused, kSrcSegments>(p, s);
-        if (mode == kModeShrink) return launch_one<E, kModeShrink, kSrcSegments>(p, s);
-        return launch_one<E, kModeExpand, kSrcSegments>(p, s);
+        if (mode == kModeFused) return launch_mode<E, kModeFused, kSrcSegments>(p, s);
+        if (mode == kModeShrink) return launch_mode<E, kModeShrink, kSrcSegments>(p, s);
+        return launch_mode<E, kModeExpand, kSrcSegments>(p, s);
     }
-    if (mode == kModeFused) return launch_one<E, kModeFused, kSrcIds>(p, s);
+    if (mode == kModeFused) return launch_mode<E, kModeFused, kSrcIds>(p, s);
     return LORA_ERR_UNSUPPORTED;
 }
 

@@ -33,6 +33,22 @@ def assert_close(y_gpu, ref: np.ndarray, dtype: str, what: str = "") -> float:
     return worst
 
 
+class option:
+    """Set a runtime option of the library for the duration of a with-block."""
+
+    def __init__(self, key: str, value: int):
+        self.key, self.value = key, value
+
+    def __enter__(self):
+        self.old = L.lora_get_option(self.key)
+        L.lora_set_option(self.key, self.value)
+        return self
+
+    def __exit__(self, *exc):
+        L.lora_set_option(self.key, self.old)
+        return False
+
+
 @functools.lru_cache(maxsize=8)
 def workload(name: str, delta_only: bool = False, reading: str = "variance", **kw):
     return workloads.generate(name, delta_only=delta_only, reading=reading, **kw)

@@ -8,7 +8,7 @@ import torch
 import heterogeneous_adapters_sgmv_b200 as L
 import oracle
 import workloads
-from tests.gpu_util import DeviceProj, assert_close, reference, workload
+from tests.gpu_util import DeviceProj, assert_close, option, reference, workload
 from workloads import to_float64
 
 pytestmark = pytest.mark.gpu
@@ -21,6 +21,7 @@ def _cuda():
     yield
     L.lora_set_option("split", 0)
     L.lora_set_option("pdl", 1)
+    L.lora_set_option("decode_cluster", 0)
 
 
 # ------------------------------------------------------------------ full-size workloads
@@ -197,20 +198,20 @@ def test_zero_B_and_zero_scale_leave_y_bit_identical(path):
     assert torch.equal(y2, dp2.d.y0)
 
 
-def test_paths_agree_bit_for_bit():
-    """BGMV, SGMV (fused) and shrink-then-expand through the fp32 workspace perform the same
-    per-token arithmetic in the same order, so they agree exactly; repeated runs too."""
+@pytest.mark.parametrize("cluster", [1, 2, 4, 8])
+def test_paths_agree_bit_for_bit(cluster):
+    """At one cluster width, BGMV, SGMV (fused) and shrink-then-expand through the fp32
+    workspace perform the same per-token arithmetic in the same order, so they agree exactly;
+    repeated runs too."""
     wl = _small("multirank_decode")
     dp = DeviceProj(wl)
-    y_b = dp.bgmv(dp.y())
-    seg, _k = dp.segments()
-    y_s = dp.sgmv(dp.y(), seg)
-    L.lora_set_option("split", 1)
-    try:
-        y_x = dp.sgmv(dp.y(), seg)
-    finally:
-        L.lora_set_option("split", 0)
-    y_b2 = dp.bgmv(dp.y())
+    with option("decode_cluster", cluster):
+        y_b = dp.bgmv(dp.y())
+        seg, _k = dp.segments()
+        y_s = dp.sgmv(dp.y(), seg)
+        with option("split", 1):
+            y_x = dp.sgmv(dp.y(), seg)
+        y_b2 = dp.bgmv(dp.y())
     assert torch.equal(y_b, y_s)
     assert torch.equal(y_b, y_x)
     assert torch.equal(y_b, y_b2)
@@ -286,11 +287,33 @@ def test_ragged_shapes_and_odd_ranks(h, o, ranks, T):
     wl = workloads.generate("multirank_decode", T=T, n=9, shapes=(("q", h, o, 0),), ranks=ranks)
     dp = DeviceProj(wl)
     ref = oracle.workload_reference(wl)
-    y = dp.bgmv(dp.y())
-    assert_close(dp.to_np(y), ref, wl.dtype, "ragged bgmv")
     seg, _k = dp.segments()
-    y2 = dp.sgmv(dp.y(), seg)
-    assert torch.equal(y, y2)
+    for cluster in (1, 2, 4, 8):
+        with option("decode_cluster", cluster):
+            y = dp.bgmv(dp.y())
+            assert_close(dp.to_np(y), ref, wl.dtype, "ragged bgmv, cluster %d" % cluster)
+            y2 = dp.sgmv(dp.y(), seg)
+            assert torch.equal(y, y2)
+
+
+@pytest.mark.parametrize("cluster", [1, 2, 4])
+@pytest.mark.parametrize("name", ["decode_bgmv", "multirank_decode", "many_adapter_qkvo"])
+def test_every_cluster_width_matches_oracle(name, cluster):
+    """The decode kernel at each forced cluster width (8 is what the automatic choice takes
+    for the small batches elsewhere in this file), fused and split, at full size."""
+    wl = workload(name)
+    ref = reference(name)
+    dp = DeviceProj(wl)
+    seg, _k = dp.segments()
+    with option("decode_cluster", cluster):
+        y = dp.bgmv(dp.y())
+        assert_close(dp.to_np(y), ref, wl.dtype, "%s bgmv, cluster %d" % (name, cluster))
+        y2 = dp.sgmv(dp.y(), seg)
+        assert_close(dp.to_np(y2), ref, wl.dtype, "%s sgmv, cluster %d" % (name, cluster))
+        with option("split", 1):
+            y3 = dp.sgmv(dp.y(), seg)
+        assert_close(dp.to_np(y3), ref, wl.dtype, "%s split, cluster %d" % (name, cluster))
+    assert dp.status() == (0, 0)
 
 
 def test_long_segment_spans_many_units():
