@@ -127,17 +127,6 @@ __device__ __forceinline__ void cvt16(const uint4 w, float *o, float *)
     o[2] = __uint_as_float(w.z); o[3] = __uint_as_float(w.w);
 }
 
-// Sum over the 32 lanes of a warp (fixed butterfly order: deterministic).
-__device__ __forceinline__ float warp_sum(float v)
-{
-    v += __shfl_xor_sync(0xffffffffu, v, 16);
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    return v;
-}
-
 __device__ __forceinline__ int ceil_log2(int v) { return v <= 1 ? 0 : 32 - __clz(v - 1); }
 
 template <typename E, int MODE, int SRC, int CL>
@@ -183,6 +172,48 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     __syncthreads();            // barriers initialised for this CTA
     if (CL > 1) cluster_arrive_relaxed();   // peers wait for this before their first remote access
 
+    // h and o ranges of this CTA, in 16-byte chunks of h and EPC-row groups of o
+    const int hchunks = p.h / EPC, ogroups = p.o / EPC;
+    const int hc0 = (int)((int64_t)crank * hchunks / CL);
+    const int hc1 = (int)((int64_t)(crank + 1) * hchunks / CL);
+    const int og0 = (int)((int64_t)crank * ogroups / CL);
+    const int og1 = (int)((int64_t)(crank + 1) * ogroups / CL);
+    const int n_shrink = (MODE == kModeExpand) ? 0 : max(1, (hc1 - hc0 + CHUNKS - 1) / CHUNKS);
+    const int orows = (og1 - og0) * EPC;
+    const int n_expand = (MODE == kModeShrink) ? 0 : (orows + W - 1) / W;
+
+    // Geometry of tile j of a unit: shrink tiles first (a slice of h, A by TMA boxes), then
+    // expand tiles (W rows of o, one bulk copy of B).  Returns the bytes the tile brings in.
+    auto tile_geom = [&](int j, int r, int &off, int &len, int &nbox) -> uint32_t {
+        if (j < n_shrink) {
+            const int c0 = hc0 + j * CHUNKS;
+            const int c1 = min(hc1, c0 + CHUNKS);
+            off = c0 * EPC;
+            len = max(0, c1 - c0) * EPC;
+            nbox = (len + BOXW - 1) / BOXW;
+            return (uint32_t)(nbox * r * kBoxBytes);
+        }
+        const int jj = j - n_shrink;
+        off = og0 * EPC + jj * W;
+        len = min(W, orows - jj * W);
+        nbox = 0;
+        return (uint32_t)(len * r * ESZ);
+    };
+    // Producer lane 0: expect the bytes of tile j of adapter a on stage s and start its copies.
+    auto issue_tile = [&](int j, int a, const AdapterDesc &d, int s) {
+        int off, len, nbox;
+        const uint32_t bytes = tile_geom(j, d.rank, off, len, nbox);
+        const uint32_t data = smem_u32(stage_base + (size_t)s * p.stage_bytes + kHeaderBytes);
+        const uint32_t fb = smem_u32(&ctl.full[s]);
+        mbar_arrive_expect_tx(fb, bytes);
+        if (j < n_shrink) {
+            const char *tmapA = reinterpret_cast<const char *>(p.tmA) + (size_t)a * 128;
+            for (int b = 0; b < nbox; ++b) tma_load_2d(data + b * d.rank * kBoxBytes, tmapA, off + b * BOXW, 0, fb);
+        } else if (len > 0) {
+            bulk_g2s(data, static_cast<const uint8_t *>(d.B) + (int64_t)off * d.rank * ESZ, len * d.rank * ESZ, fb);
+        }
+    };
+
     // Per-token ids: tokens with equal ids form one group.  With no more adapters than
     // clusters, cluster c owns adapter c and its producer scans the ids itself; otherwise a
     // group is led by the first token carrying its id and groups are listed in leader order.
@@ -192,10 +223,20 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     const bool direct_ids = (SRC == kSrcIds) && p.n <= G;
     // The adapter table is immutable after creation: in direct mode this cluster's descriptor
     // and tensor map are fetched before waiting for the previous grid.
+    // The weights are immutable too, so the copies of the first stages of this cluster's
+    // adapter start here as well; the tiles are handed to the consumers (with no tokens if the
+    // adapter turns out to be unused) once the ids are known.
+    // A consumer thread starts them, so the producer warp goes straight on to the ids.
     AdapterDesc pre_desc = {};
-    if (direct_ids && warp == kConsumerWarps && cid < p.n) {
+    const int npre_all = (direct_ids && cid < p.n) ? min(n_shrink + n_expand, S) : 0;
+    int npre = 0;
+    if (npre_all > 0 && warp == kConsumerWarps) {
         pre_desc = p.desc[cid];
-        if (lane == 0) prefetch_tensormap(reinterpret_cast<const char *>(p.tmA) + (size_t)cid * 128);
+        npre = npre_all;
+    }
+    if (npre_all > 0 && tid == 0) {
+        const AdapterDesc d0 = p.desc[cid];
+        for (int j = 0; j < npre_all; ++j) issue_tile(j, cid, d0, j);
     }
     pdl_wait();
     pdl_launch_dependents();
@@ -229,19 +270,9 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     }
     if (tid == 0) LORA_TRACE_MARK(1);
 
-    // h and o ranges of this CTA, in 16-byte chunks of h and EPC-row groups of o
-    const int hchunks = p.h / EPC, ogroups = p.o / EPC;
-    const int hc0 = (int)((int64_t)crank * hchunks / CL);
-    const int hc1 = (int)((int64_t)(crank + 1) * hchunks / CL);
-    const int og0 = (int)((int64_t)crank * ogroups / CL);
-    const int og1 = (int)((int64_t)(crank + 1) * ogroups / CL);
-    const int n_shrink = (MODE == kModeExpand) ? 0 : max(1, (hc1 - hc0 + CHUNKS - 1) / CHUNKS);
-    const int orows = (og1 - og0) * EPC;
-    const int n_expand = (MODE == kModeShrink) ? 0 : (orows + W - 1) / W;
-
     if (warp == kConsumerWarps) {
         // ================================ producer warp ================================
-        int issued = 0;
+        int issued = 0, ps = 0, pround = 0;   // tiles issued; stage and round of the next one
         bool alive = true;
         if (direct_ids) {
             // stage the ids for this warp's scan; cluster 0 CTA 0 reports bad ids
@@ -355,39 +386,29 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     }
                 }
             }
-            if (L == 0 || !alive) break;
+            if (L == 0 && npre > 0) {   // copies already started: hand them over with no tokens
+                a = cid;
+                d = pre_desc;
+            } else if (L == 0 || !alive) {
+                break;
+            }
 
-            // ---- issue every tile of this unit
+            // ---- issue every tile of this unit (the first npre were started before the wait)
             const int r = d.rank;
-            const char *tmapA = reinterpret_cast<const char *>(p.tmA) + (size_t)a * 128;
-            const uint8_t *Bb = static_cast<const uint8_t *>(d.B);
             if (lane == 0) LORA_TRACE_MARK(2);
             const int ntiles = n_shrink + n_expand;
+            const int skip = npre;
+            npre = 0;
             for (int j = 0; j < ntiles; ++j) {
-                const int s = issued % S, m = issued / S;
+                const int s = ps, m = pround;
                 if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
                     alive = false;
                     break;
                 }
                 StageHeader *hdr = reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
-                const uint32_t data = smem_u32(stage_base + (size_t)s * p.stage_bytes + kHeaderBytes);
-                const uint32_t fb = smem_u32(&ctl.full[s]);
                 const bool shrink = j < n_shrink;
-                int off, len, nbox = 0;
-                uint32_t bytes;
-                if (shrink) {
-                    const int c0 = hc0 + j * CHUNKS;
-                    const int c1 = min(hc1, c0 + CHUNKS);
-                    off = c0 * EPC;
-                    len = max(0, c1 - c0) * EPC;
-                    nbox = (len + BOXW - 1) / BOXW;
-                    bytes = (uint32_t)(nbox * r * kBoxBytes);
-                } else {
-                    const int jj = j - n_shrink;
-                    off = og0 * EPC + jj * W;
-                    len = min(W, orows - jj * W);
-                    bytes = (uint32_t)(len * r * ESZ);
-                }
+                int off, len, nbox;
+                tile_geom(j, r, off, len, nbox);
                 if (lane < L) hdr->tok[lane] = my_tok;
                 if (lane == 0) {
                     hdr->kind = shrink ? kTileShrink : kTileExpand;
@@ -404,13 +425,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(smem_u32(&ctl.meta[s]));
-                    mbar_arrive_expect_tx(fb, bytes);
-                    if (shrink) {
-                        for (int b = 0; b < nbox; ++b)
-                            tma_load_2d(data + b * r * kBoxBytes, tmapA, off + b * BOXW, 0, fb);
-                    } else if (len > 0) {
-                        bulk_g2s(data, Bb + (int64_t)off * r * ESZ, len * r * ESZ, fb);
-                    }
+                    if (j >= skip) issue_tile(j, a, d, s);
                 }
                 // L2 hints for the rows the consumers load for this tile (lane l: row l)
                 if (lane < L) {
@@ -420,12 +435,16 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     for (int c = 0; c < len * ESZ; c += 128) prefetch_l2(row + c);
                 }
                 ++issued;
+                if (++ps == S) {
+                    ps = 0;
+                    ++pround;
+                }
                 if (lane == 0) LORA_TRACE_MARK(shrink ? 3 : 4);
             }
         }
         // end marker
         if (alive) {
-            const int s = issued % S, m = issued / S;
+            const int s = ps, m = pround;
             if (m < 1 || mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
                 if (lane == 0) {
                     reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes)->kind = kTileEnd;
@@ -449,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     int u = 0;   // units whose intermediate has been exchanged (fused / shrink modes)
     bool cluster_waited = false;
     uint4 ld[4];
-    auto stage_header = [&](int i) -> const StageHeader & {
-        return *reinterpret_cast<const StageHeader *>(stage_base + (size_t)(i % S) * p.stage_bytes);
+    auto stage_header = [&](int st) -> const StageHeader & {
+        return *reinterpret_cast<const StageHeader *>(stage_base + (size_t)st * p.stage_bytes);
     };
     auto load_rows = [&](const StageHeader &h) {
         const bool xr = h.kind == kTileShrink;
@@ -468,11 +487,13 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     };
     bool live = mbar_wait(smem_u32(&ctl.meta[0]), 0, p.status);
     if (live && stage_header(0).kind != kTileEnd) load_rows(stage_header(0));
+    int s = 0;          // stage of tile `it`
+    uint32_t ph = 0;    // its phase parity
     for (int it = 0; live; ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
+        const int s1 = s + 1 == S ? 0 : s + 1;        // stage of the next tile
+        const uint32_t ph1 = s1 == 0 ? ph ^ 1u : ph;
         if (tid == 0 && it < 2) LORA_TRACE_MARK(5 + 5 * it);
-        const StageHeader &hdr = stage_header(it);
+        const StageHeader &hdr = stage_header(s);
         const int kind = hdr.kind;
         if (kind == kTileEnd) break;
         const int r = hdr.rank, L = hdr.L, flags = hdr.flags, len = hdr.len, off = hdr.off;
@@ -491,8 +512,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         }
         // next tile's rows (its stage was released S - 1 tiles ago, so its header comes
         // without waiting on this tile)
-        if (!mbar_wait(smem_u32(&ctl.meta[(it + 1) % S]), ((it + 1) / S) & 1, p.status)) break;
-        if (stage_header(it + 1).kind != kTileEnd) load_rows(stage_header(it + 1));
+        if (!mbar_wait(smem_u32(&ctl.meta[s1]), ph1, p.status)) break;
+        if (stage_header(s1).kind != kTileEnd) load_rows(stage_header(s1));
         if (!mbar_wait(smem_u32(&ctl.full[s]), ph, p.status)) break;
         if (tid == 0 && it < 2) LORA_TRACE_MARK(7 + 5 * it);
         named_bar_sync(1, kConsumers);
@@ -502,29 +523,54 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             const bool first = flags & kFlagFirst;
             // ---- partial shrink over this CTA's slice of h: warp w owns rows w, w + 8, ...;
             // A is staged as [box][row][512 B] (box 1 after r rows of box 0), x as [token][row].
+            // Two tokens x two rows at a time: a lane forms the four partial dot products over
+            // its 16 elements, and one transposed butterfly folds all four across the warp.
             const bool okA = lane < nch, okB = lane + 32 < nch;
             const uint4 z = make_uint4(0, 0, 0, 0);
             if (warp < r) {
-                for (int l = 0; l < L; ++l) {
-                    const uint8_t *xr = xs + l * rowb;
-                    float xv[2 * EPC];
-                    cvt16(okA ? *reinterpret_cast<const uint4 *>(xr + lane * 16) : z, xv, (E *)nullptr);
-                    cvt16(okB ? *reinterpret_cast<const uint4 *>(xr + 512 + lane * 16) : z, xv + EPC, (E *)nullptr);
-                    for (int k = warp; k < r; k += kConsumerWarps) {
-                        const uint8_t *row = data + k * kBoxBytes;
-                        float av[2 * EPC];
-                        cvt16(okA ? *reinterpret_cast<const uint4 *>(row + lane * 16) : z, av, (E *)nullptr);
-                        cvt16(okB ? *reinterpret_cast<const uint4 *>(row + r * kBoxBytes + lane * 16) : z, av + EPC,
-                              (E *)nullptr);
-                        float s0 = 0.f, s1 = 0.f;
+                for (int l = 0; l < L; l += 2) {
+                    const bool l2 = l + 1 < L;
+                    const uint8_t *xr0 = xs + l * rowb, *xr1 = xr0 + rowb;
+                    float xv0[2 * EPC], xv1[2 * EPC];
+                    cvt16(okA ? *reinterpret_cast<const uint4 *>(xr0 + lane * 16) : z, xv0, (E *)nullptr);
+                    cvt16(okB ? *reinterpret_cast<const uint4 *>(xr0 + 512 + lane * 16) : z, xv0 + EPC, (E *)nullptr);
+                    cvt16(l2 && okA ? *reinterpret_cast<const uint4 *>(xr1 + lane * 16) : z, xv1, (E *)nullptr);
+                    cvt16(l2 && okB ? *reinterpret_cast<const uint4 *>(xr1 + 512 + lane * 16) : z, xv1 + EPC,
+                          (E *)nullptr);
+                    for (int k = warp; k < r; k += 2 * kConsumerWarps) {
+                        const bool k2 = k + kConsumerWarps < r;
+                        float p[4];   // (token l, row k), (l, k + 8), (l + 1, k), (l + 1, k + 8)
 #pragma unroll
-                        for (int e = 0; e < EPC; ++e) {
-                            s0 = fmaf(xv[e], av[e], s0);
-                            s1 = fmaf(xv[EPC + e], av[EPC + e], s1);
+                        for (int q = 0; q < 2; ++q) {
+                            const uint8_t *row = data + (k + q * kConsumerWarps) * kBoxBytes;
+                            const bool ok = q == 0 || k2;
+                            float av[2 * EPC];
+                            cvt16(ok && okA ? *reinterpret_cast<const uint4 *>(row + lane * 16) : z, av, (E *)nullptr);
+                            cvt16(ok && okB ? *reinterpret_cast<const uint4 *>(row + r * kBoxBytes + lane * 16) : z,
+                                  av + EPC, (E *)nullptr);
+                            float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
+#pragma unroll
+                            for (int e = 0; e < EPC; ++e) {
+                                s0 = fmaf(xv0[e], av[e], s0);
+                                s1 = fmaf(xv0[EPC + e], av[EPC + e], s1);
+                                t0 = fmaf(xv1[e], av[e], t0);
+                                t1 = fmaf(xv1[EPC + e], av[EPC + e], t1);
+                            }
+                            p[q] = s0 + s1;
+                            p[2 + q] = t0 + t1;
                         }
-                        const float tot = warp_sum(s0 + s1);
-                        if (lane == 0) {
-                            float *dst = vpart + l * RP + k;
+                        // lane ends with value j = (lane >> 3) & 3, summed over all 32 lanes
+                        const bool hi16 = lane & 16, hi8 = lane & 8;
+                        float k0 = hi16 ? p[2] : p[0], k1 = hi16 ? p[3] : p[1];
+                        k0 += __shfl_xor_sync(0xffffffffu, hi16 ? p[0] : p[2], 16);
+                        k1 += __shfl_xor_sync(0xffffffffu, hi16 ? p[1] : p[3], 16);
+                        float tot = hi8 ? k1 : k0;
+                        tot += __shfl_xor_sync(0xffffffffu, hi8 ? k0 : k1, 8);
+                        tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+                        tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+                        tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+                        if ((lane & 7) == 0 && (!hi16 || l2) && (!hi8 || k2)) {
+                            float *dst = vpart + (l + (hi16 ? 1 : 0)) * RP + k + (hi8 ? kConsumerWarps : 0);
                             *dst = first ? tot : *dst + tot;
                         }
                     }
@@ -597,19 +643,24 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             const float sc = hdr.scale;
             const int c = tid * CPT;   // first column of this thread within the tile
             if (c < len) {
+                // Two tokens per pass share each load of this thread's B rows; per output the
+                // products are still added in ascending k.
                 const uint8_t *brow = data + (size_t)c * r * ESZ;   // CPT consecutive rows of B
-                for (int l = 0; l < L; ++l) {
-                    const float *vr = vsum + l * RP;
-                    float acc[CPT];
+                for (int l = 0; l < L; l += 2) {
+                    const bool l2 = l + 1 < L;   // row l + 1 of vsum exists even when unused
+                    const float *vr0 = vsum + l * RP, *vr1 = vr0 + RP;
+                    float acc0[CPT], acc1[CPT];
 #pragma unroll
-                    for (int j = 0; j < CPT; ++j) acc[j] = 0.f;
+                    for (int j = 0; j < CPT; ++j) acc0[j] = acc1[j] = 0.f;
                     if ((r % EPC) == 0) {
                         for (int k = 0; k < r; k += EPC) {
-                            float vv[EPC];
+                            float v0[EPC], v1[EPC];
 #pragma unroll
                             for (int e = 0; e < EPC; e += 4) {
-                                const float4 t4 = *reinterpret_cast<const float4 *>(vr + k + e);
-                                vv[e] = t4.x; vv[e + 1] = t4.y; vv[e + 2] = t4.z; vv[e + 3] = t4.w;
+                                const float4 a4 = *reinterpret_cast<const float4 *>(vr0 + k + e);
+                                const float4 b4 = *reinterpret_cast<const float4 *>(vr1 + k + e);
+                                v0[e] = a4.x; v0[e + 1] = a4.y; v0[e + 2] = a4.z; v0[e + 3] = a4.w;
+                                v1[e] = b4.x; v1[e + 1] = b4.y; v1[e + 2] = b4.z; v1[e + 3] = b4.w;
                             }
 #pragma unroll
                             for (int j = 0; j < CPT; ++j) {
@@ -617,26 +668,37 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                                 cvt16(*reinterpret_cast<const uint4 *>(brow + ((size_t)j * r + k) * ESZ), b,
                                       (E *)nullptr);
 #pragma unroll
-                                for (int e = 0; e < EPC; ++e) acc[j] = fmaf(vv[e], b[e], acc[j]);
+                                for (int e = 0; e < EPC; ++e) {
+                                    acc0[j] = fmaf(v0[e], b[e], acc0[j]);
+                                    acc1[j] = fmaf(v1[e], b[e], acc1[j]);
+                                }
                             }
                         }
                     } else {
                         for (int k = 0; k < r; ++k) {
 #pragma unroll
-                            for (int j = 0; j < CPT; ++j)
-                                acc[j] = fmaf(vr[k], (float)reinterpret_cast<const E *>(brow)[j * r + k], acc[j]);
+                            for (int j = 0; j < CPT; ++j) {
+                                const float b = (float)reinterpret_cast<const E *>(brow)[j * r + k];
+                                acc0[j] = fmaf(vr0[k], b, acc0[j]);
+                                acc1[j] = fmaf(vr1[k], b, acc1[j]);
+                            }
                         }
                     }
-                    const uint8_t *yr = ys + l * rowb + c * ESZ;
-                    const int64_t gofs = (int64_t)hdr.tok[l] * p.ldy + p.y_off + off + c;
-                    if constexpr (CPT == 2) {
-                        const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
-                        const float y0 = fmaf(sc, acc[0], bf16_lo(w));
-                        const float y1 = fmaf(sc, acc[1], bf16_hi(w));
-                        *reinterpret_cast<uint32_t *>(static_cast<E *>(p.y) + gofs) = pack_bf16x2(y0, y1);
-                    } else {
-                        const float w = *reinterpret_cast<const float *>(yr);
-                        static_cast<float *>(p.y)[gofs] = fmaf(sc, acc[0], w);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        if (q == 1 && !l2) break;
+                        const float *acc = q == 0 ? acc0 : acc1;
+                        const uint8_t *yr = ys + (l + q) * rowb + c * ESZ;
+                        const int64_t gofs = (int64_t)hdr.tok[l + q] * p.ldy + p.y_off + off + c;
+                        if constexpr (CPT == 2) {
+                            const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
+                            const float y0 = fmaf(sc, acc[0], bf16_lo(w));
+                            const float y1 = fmaf(sc, acc[1], bf16_hi(w));
+                            *reinterpret_cast<uint32_t *>(static_cast<E *>(p.y) + gofs) = pack_bf16x2(y0, y1);
+                        } else {
+                            const float w = *reinterpret_cast<const float *>(yr);
+                            static_cast<float *>(p.y)[gofs] = fmaf(sc, acc[0], w);
+                        }
                     }
                 }
             }
@@ -645,6 +707,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         if (tid == 0 && kind == kTileExpand && (flags & kFlagLast) && u >= 1 && u <= 8) LORA_TRACE_MARK(35 + 4 * (u - 1));
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
+        s = s1;
+        ph = ph1;
     }
     if (tid == 0) LORA_TRACE_MARK(24);
     // No CTA may leave while a peer can still arrive on its barriers: wait until every peer
