@@ -76,8 +76,8 @@ def measured_peaks():
 
 
 def profile_traffic(workload: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if the
-    summary says it still matches the current kernel."""
+    """DRAM bytes per launch of the dominant kernel (per step for workloads timed as a whole
+    step) from the committed ncu summary, if the summary says it still matches the kernels."""
     path = os.path.join(ROOT, "profiles", "%s_ncu.md" % workload)
     if not os.path.exists(path):
         return None
@@ -89,7 +89,7 @@ def profile_traffic(workload: str):
     try:
         if vals.get("current", "yes").lower() != "yes":
             return None
-        return float(vals["dram_bytes_per_launch"])
+        return float(vals.get("dram_bytes_per_launch") or vals["dram_bytes_per_step"])
     except (KeyError, ValueError):
         return None
 
