@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a graph")
+    ap.add_argument("--grouped", action="store_true",
+                    help="many_adapter_qkvo: one lora_sgmv_grouped launch for q, k, v, o (q, k, v reading one x) "
+                         "instead of four lora_sgmv calls")
     return ap.parse_args()
 
 
@@ -178,10 +181,25 @@ class Copy:
         return tot
 
 
-def make_step(wl, L):
+def make_step(wl, L, grouped=False):
     """Returns (step(copy, stream_handle), launches per step, name of the dominant kernel)."""
     name = wl.name
     T = wl.T
+    if grouped:
+        if name != "many_adapter_qkvo":
+            raise SystemExit("--grouped applies to many_adapter_qkvo only")
+        grp = [g for (_n, _h, _o, g) in wl.spec.projections]
+        src = [grp.index(g) for g in grp]   # the first projection reading the same x
+
+        def step(c, s):
+            st = c.seg_t
+            L.lora_build_segments(c.tables[0].handle, c.ids, T, st["perm"], st["seg_ptr"], st["seg_adapter"],
+                                  st["num"], s)
+            xs = [c.projs[i].x for i in src]
+            L.lora_sgmv_grouped([t.handle for t in c.tables], c.seg, xs, [x.shape[1] for x in xs],
+                                [d.y0 for d in c.projs], [d.o for d in c.projs], [0] * len(c.projs), c.ws,
+                                c.ws.numel(), s)
+        return step, 2, "lora_decode_kernel (fused, segments, 4 projections per launch)"
 
     if name == "decode_bgmv":
         def step(c, s):
@@ -215,8 +233,8 @@ def run_ours(args, rank, world, local_rank):
     seed = workloads.SEED_BASE + workloads.WORKLOAD_NAMES.index(args.workload) + 1000 * rank
     wl = workloads.generate(args.workload, seed=seed)
     T = wl.T
-    step, launches_per_step, kname = make_step(wl, L)
-    bytes_step = accounting.workload_bytes(wl)
+    step, launches_per_step, kname = make_step(wl, L, args.grouped)
+    bytes_step = accounting.workload_bytes(wl, shared_x=args.grouped)
     flops_step = accounting.workload_flops(wl)
     distinct = int(accounting.distinct_adapters(wl.ids).size)
 
@@ -374,7 +392,9 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": codes[wl.dtype], "data": "synthetic (seeded; random adapter weights and activations)",
-        "config": {"workload": "%s: %s" % (args.workload, DESCRIPTIONS[args.workload]),
+        "config": {"workload": "%s: %s" % (args.workload, DESCRIPTIONS[args.workload] if not args.grouped else
+                                           DESCRIPTIONS[args.workload].replace(
+                                               "4 x lora_sgmv", "one lora_sgmv_grouped, q/k/v sharing x")),
                    "tokens_per_step": T, "distinct_adapters_per_step": distinct,
                    "algorithmic_bytes_per_step": bytes_step, "flops_per_step": flops_step,
                    "l2": "rotating %d input copies, %.0f MB in total against a 126 MB L2%s" % (

@@ -32,12 +32,13 @@ LORA_STATUS_BAD_SEGMENT = 4
 LORA_MAX_RANK = 128
 LORA_MAX_SEGMENT_TOKENS = 8192
 LORA_NOALLOC_SCRATCH_FLOATS = 262144
+LORA_MAX_GROUP = 4
 
 EXPORTS = (
     "lora_table_create", "lora_table_destroy", "lora_table_info", "lora_workspace_bytes",
     "lora_build_segments", "lora_shrink", "lora_expand", "lora_sgmv", "lora_bgmv",
     "lora_get_status", "lora_status_string", "lora_set_option", "lora_get_option",
-    "lora_sgmv_noalloc",
+    "lora_sgmv_noalloc", "lora_sgmv_grouped",
 )
 
 
@@ -84,6 +85,7 @@ def _load():
         "lora_sgmv": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
         "lora_bgmv": ([P, P, I32, P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
         "lora_sgmv_noalloc": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, I32, P], ctypes.c_int),
+        "lora_sgmv_grouped": ([P, I32, ctypes.POINTER(lora_segments), P, P, P, P, P, P, SZ, P], ctypes.c_int),
         "lora_get_status": ([P, ctypes.POINTER(ctypes.c_uint32), I32, P], ctypes.c_int),
         "lora_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "lora_set_option": ([ctypes.c_char_p, I64], ctypes.c_int),
@@ -176,6 +178,23 @@ def lora_sgmv(table: int, seg: lora_segments, x, ldx: int, y, ldy: int, y_offset
               ws_bytes: int = 0, stream=None) -> None:
     _check(_load().lora_sgmv(table, ctypes.byref(seg), _ptr(x), ldx, _ptr(y), ldy, y_offset, _ptr(ws), ws_bytes,
                              _stream(stream)), "lora_sgmv")
+
+
+def lora_sgmv_grouped(tables, seg: lora_segments, xs, ldxs, ys, ldys, y_offsets, ws=None, ws_bytes: int = 0,
+                      stream=None) -> None:
+    """One launch for several projections sharing a segment table: projection p applies
+    tables[p] to xs[p] and updates ys[p][:, y_offsets[p] : y_offsets[p] + o_p]."""
+    P = len(tables)
+    if not (len(xs) == len(ldxs) == len(ys) == len(ldys) == len(y_offsets) == P):
+        raise ValueError("lora_sgmv_grouped: every per-projection list needs one entry per table")
+    t_arr = (ctypes.c_void_p * P)(*tables)
+    x_arr = (ctypes.c_void_p * P)(*[_ptr(x) for x in xs])
+    y_arr = (ctypes.c_void_p * P)(*[_ptr(y) for y in ys])
+    ldx_arr = (ctypes.c_int64 * P)(*ldxs)
+    ldy_arr = (ctypes.c_int64 * P)(*ldys)
+    off_arr = (ctypes.c_int32 * P)(*y_offsets)
+    _check(_load().lora_sgmv_grouped(t_arr, P, ctypes.byref(seg), x_arr, ldx_arr, y_arr, ldy_arr, off_arr,
+                                     _ptr(ws), ws_bytes, _stream(stream)), "lora_sgmv_grouped")
 
 
 def lora_sgmv_noalloc(table: int, seg: lora_segments, x, ldx: int, y, ldy: int, y_offset: int, stream=None) -> None:

@@ -62,6 +62,7 @@ struct __align__(16) StageHeader {
     int32_t kind, flags, adapter, rank;
     float scale;
     int32_t L, off, len;   // tokens; first column of h (shrink) or row of o (expand); extent
+    int32_t proj;          // projection of a grouped launch
     int32_t tok[kTokChunk];
 };
 static_assert(sizeof(StageHeader) <= kHeaderBytes, "header");
@@ -172,42 +173,51 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     __syncthreads();            // barriers initialised for this CTA
     if (CL > 1) cluster_arrive_relaxed();   // peers wait for this before their first remote access
 
-    // h and o ranges of this CTA, in 16-byte chunks of h and EPC-row groups of o
-    const int hchunks = p.h / EPC, ogroups = p.o / EPC;
-    const int hc0 = (int)((int64_t)crank * hchunks / CL);
-    const int hc1 = (int)((int64_t)(crank + 1) * hchunks / CL);
-    const int og0 = (int)((int64_t)crank * ogroups / CL);
-    const int og1 = (int)((int64_t)(crank + 1) * ogroups / CL);
-    const int n_shrink = (MODE == kModeExpand) ? 0 : max(1, (hc1 - hc0 + CHUNKS - 1) / CHUNKS);
-    const int orows = (og1 - og0) * EPC;
-    const int n_expand = (MODE == kModeShrink) ? 0 : (orows + W - 1) / W;
-
+    // This CTA's share of projection pi: a range of h in 16-byte chunks (shrink) and a range
+    // of o in EPC-row groups (expand), and the tiles they make.
+    const int lgW = lgC + 4 - (ESZ == 2 ? 1 : 2);   // W = 2^lgW
+    struct Geo {
+        int hc0, hc1, og0, orows, n_shrink, n_expand;
+    };
+    auto geo_of = [&](int pi) -> Geo {
+        Geo g;
+        const int hchunks = p.pj[pi].h / EPC, ogroups = p.pj[pi].o / EPC;
+        g.hc0 = (int)((int64_t)crank * hchunks / CL);
+        g.hc1 = (int)((int64_t)(crank + 1) * hchunks / CL);
+        g.og0 = (int)((int64_t)crank * ogroups / CL);
+        const int og1 = (int)((int64_t)(crank + 1) * ogroups / CL);
+        g.n_shrink = (MODE == kModeExpand) ? 0 : max(1, (g.hc1 - g.hc0 + CHUNKS - 1) >> lgC);
+        g.orows = (og1 - g.og0) * EPC;
+        g.n_expand = (MODE == kModeShrink) ? 0 : (g.orows + W - 1) >> lgW;
+        return g;
+    };
     // Geometry of tile j of a unit: shrink tiles first (a slice of h, A by TMA boxes), then
     // expand tiles (W rows of o, one bulk copy of B).  Returns the bytes the tile brings in.
-    auto tile_geom = [&](int j, int r, int &off, int &len, int &nbox) -> uint32_t {
-        if (j < n_shrink) {
-            const int c0 = hc0 + j * CHUNKS;
-            const int c1 = min(hc1, c0 + CHUNKS);
+    auto tile_geom = [&](const Geo &g, int j, int r, int &off, int &len, int &nbox) -> uint32_t {
+        if (j < g.n_shrink) {
+            const int c0 = g.hc0 + j * CHUNKS;
+            const int c1 = min(g.hc1, c0 + CHUNKS);
             off = c0 * EPC;
             len = max(0, c1 - c0) * EPC;
             nbox = (len + BOXW - 1) / BOXW;
             return (uint32_t)(nbox * r * kBoxBytes);
         }
-        const int jj = j - n_shrink;
-        off = og0 * EPC + jj * W;
-        len = min(W, orows - jj * W);
+        const int jj = j - g.n_shrink;
+        off = g.og0 * EPC + jj * W;
+        len = min(W, g.orows - jj * W);
         nbox = 0;
         return (uint32_t)(len * r * ESZ);
     };
-    // Producer lane 0: expect the bytes of tile j of adapter a on stage s and start its copies.
-    auto issue_tile = [&](int j, int a, const AdapterDesc &d, int s) {
+    // One thread: expect the bytes of tile j of adapter a (projection pi) on stage s and start
+    // its copies.
+    auto issue_tile = [&](const Geo &g, int pi, int j, int a, const AdapterDesc &d, int s) {
         int off, len, nbox;
-        const uint32_t bytes = tile_geom(j, d.rank, off, len, nbox);
+        const uint32_t bytes = tile_geom(g, j, d.rank, off, len, nbox);
         const uint32_t data = smem_u32(stage_base + (size_t)s * p.stage_bytes + kHeaderBytes);
         const uint32_t fb = smem_u32(&ctl.full[s]);
         mbar_arrive_expect_tx(fb, bytes);
-        if (j < n_shrink) {
-            const char *tmapA = reinterpret_cast<const char *>(p.tmA) + (size_t)a * 128;
+        if (j < g.n_shrink) {
+            const char *tmapA = reinterpret_cast<const char *>(p.pj[pi].tmA) + (size_t)a * 128;
             for (int b = 0; b < nbox; ++b) tma_load_2d(data + b * d.rank * kBoxBytes, tmapA, off + b * BOXW, 0, fb);
         } else if (len > 0) {
             bulk_g2s(data, static_cast<const uint8_t *>(d.B) + (int64_t)off * d.rank * ESZ, len * d.rank * ESZ, fb);
@@ -228,15 +238,16 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     // adapter turns out to be unused) once the ids are known.
     // A consumer thread starts them, so the producer warp goes straight on to the ids.
     AdapterDesc pre_desc = {};
-    const int npre_all = (direct_ids && cid < p.n) ? min(n_shrink + n_expand, S) : 0;
+    const Geo geo0 = geo_of(0);
+    const int npre_all = (direct_ids && cid < p.n) ? min(geo0.n_shrink + geo0.n_expand, S) : 0;
     int npre = 0;
     if (npre_all > 0 && warp == kConsumerWarps) {
-        pre_desc = p.desc[cid];
+        pre_desc = p.pj[0].desc[cid];
         npre = npre_all;
     }
     if (npre_all > 0 && tid == 0) {
-        const AdapterDesc d0 = p.desc[cid];
-        for (int j = 0; j < npre_all; ++j) issue_tile(j, cid, d0, j);
+        const AdapterDesc d0 = p.pj[0].desc[cid];
+        for (int j = 0; j < npre_all; ++j) issue_tile(geo0, 0, j, cid, d0, j);
     }
     pdl_wait();
     pdl_launch_dependents();
@@ -331,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     const int first_unit = ubase + __shfl_sync(0xffffffffu, w_incl - w_nu, hl);
                     const int start = __shfl_sync(0xffffffffu, w_p0, hl) + (un - first_unit) * kTokChunk;
                     un += G;
-                    d = p.desc[sa];
+                    d = p.pj[0].desc[sa];
                     const int L0 = min(kTokChunk, p1 - start);
                     int t = -1;
                     if (lane < L0) t = p.perm ? p.perm[start + lane] : start + lane;
@@ -376,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         my_tok = ctl.pending[lane & (kTokChunk - 1)];
                         L = cnt;
                         a = ga;
-                        d = direct_ids ? pre_desc : p.desc[ga];
+                        d = direct_ids ? pre_desc : p.pj[0].desc[ga];
                     }
                     __syncwarp();
                     cnt = 0;
@@ -393,53 +404,60 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 break;
             }
 
-            // ---- issue every tile of this unit (the first npre were started before the wait)
-            const int r = d.rank;
+            // ---- issue every tile of this unit, once per projection (the first npre tiles of
+            // projection 0 were started before the grid dependency wait)
             if (lane == 0) LORA_TRACE_MARK(2);
-            const int ntiles = n_shrink + n_expand;
             const int skip = npre;
             npre = 0;
-            for (int j = 0; j < ntiles; ++j) {
-                const int s = ps, m = pround;
-                if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
-                    alive = false;
-                    break;
+            for (int pi = 0; pi < p.P && alive; ++pi) {
+                const ProjParams &pj = p.pj[pi];
+                if (pi > 0) d = pj.desc[a];
+                const Geo g = pi == 0 ? geo0 : geo_of(pi);
+                const int r = d.rank;
+                const int ntiles = g.n_shrink + g.n_expand;
+                for (int j = 0; j < ntiles; ++j) {
+                    const int s = ps, m = pround;
+                    if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
+                        alive = false;
+                        break;
+                    }
+                    StageHeader *hdr = reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
+                    const bool shrink = j < g.n_shrink;
+                    int off, len, nbox;
+                    tile_geom(g, j, r, off, len, nbox);
+                    if (lane < L) hdr->tok[lane] = my_tok;
+                    if (lane == 0) {
+                        hdr->kind = shrink ? kTileShrink : kTileExpand;
+                        const int first_j = shrink ? 0 : g.n_shrink;
+                        const int last_j = shrink ? g.n_shrink - 1 : ntiles - 1;
+                        hdr->flags = (j == first_j ? kFlagFirst : 0) | (j == last_j ? kFlagLast : 0);
+                        hdr->adapter = a;
+                        hdr->rank = r;
+                        hdr->scale = d.scale;
+                        hdr->L = L;
+                        hdr->off = off;
+                        hdr->len = len;
+                        hdr->proj = pi;
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(smem_u32(&ctl.meta[s]));
+                        if (pi > 0 || j >= skip) issue_tile(g, pi, j, a, d, s);
+                    }
+                    // L2 hints for the rows the consumers load for this tile (lane l: row l)
+                    if (lane < L) {
+                        const uint8_t *row =
+                            shrink ? static_cast<const uint8_t *>(pj.x) + ((int64_t)my_tok * pj.ldx + off) * ESZ
+                                   : static_cast<const uint8_t *>(pj.y) + ((int64_t)my_tok * pj.ldy + pj.y_off + off) * ESZ;
+                        for (int c = 0; c < len * ESZ; c += 128) prefetch_l2(row + c);
+                    }
+                    ++issued;
+                    if (++ps == S) {
+                        ps = 0;
+                        ++pround;
+                    }
+                    if (lane == 0) LORA_TRACE_MARK(shrink ? 3 : 4);
                 }
-                StageHeader *hdr = reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
-                const bool shrink = j < n_shrink;
-                int off, len, nbox;
-                tile_geom(j, r, off, len, nbox);
-                if (lane < L) hdr->tok[lane] = my_tok;
-                if (lane == 0) {
-                    hdr->kind = shrink ? kTileShrink : kTileExpand;
-                    const int first_j = shrink ? 0 : n_shrink;
-                    const int last_j = shrink ? n_shrink - 1 : ntiles - 1;
-                    hdr->flags = (j == first_j ? kFlagFirst : 0) | (j == last_j ? kFlagLast : 0);
-                    hdr->adapter = a;
-                    hdr->rank = r;
-                    hdr->scale = d.scale;
-                    hdr->L = L;
-                    hdr->off = off;
-                    hdr->len = len;
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_u32(&ctl.meta[s]));
-                    if (j >= skip) issue_tile(j, a, d, s);
-                }
-                // L2 hints for the rows the consumers load for this tile (lane l: row l)
-                if (lane < L) {
-                    const uint8_t *row =
-                        shrink ? static_cast<const uint8_t *>(p.x) + ((int64_t)my_tok * p.ldx + off) * ESZ
-                               : static_cast<const uint8_t *>(p.y) + ((int64_t)my_tok * p.ldy + p.y_off + off) * ESZ;
-                    for (int c = 0; c < len * ESZ; c += 128) prefetch_l2(row + c);
-                }
-                ++issued;
-                if (++ps == S) {
-                    ps = 0;
-                    ++pround;
-                }
-                if (lane == 0) LORA_TRACE_MARK(shrink ? 3 : 4);
             }
         }
         // end marker
@@ -474,9 +492,10 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     auto load_rows = [&](const StageHeader &h) {
         const bool xr = h.kind == kTileShrink;
         const int L = h.L, nch = h.len / EPC;
-        const uint8_t *src = xr ? static_cast<const uint8_t *>(p.x) + (int64_t)h.off * ESZ
-                                : static_cast<const uint8_t *>(p.y) + ((int64_t)p.y_off + h.off) * ESZ;
-        const int64_t ld_row = (xr ? p.ldx : p.ldy) * ESZ;
+        const ProjParams &pj = p.pj[h.proj];
+        const uint8_t *src = xr ? static_cast<const uint8_t *>(pj.x) + (int64_t)h.off * ESZ
+                                : static_cast<const uint8_t *>(pj.y) + ((int64_t)pj.y_off + h.off) * ESZ;
+        const int64_t ld_row = (xr ? pj.ldx : pj.ldy) * ESZ;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int e = tid + kConsumers * i;
@@ -641,6 +660,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 named_bar_sync(1, kConsumers);
             }
             const float sc = hdr.scale;
+            const ProjParams &pj = p.pj[hdr.proj];
             const int c = tid * CPT;   // first column of this thread within the tile
             if (c < len) {
                 // Two tokens per pass share each load of this thread's B rows; per output the
@@ -689,15 +709,15 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         if (q == 1 && !l2) break;
                         const float *acc = q == 0 ? acc0 : acc1;
                         const uint8_t *yr = ys + (l + q) * rowb + c * ESZ;
-                        const int64_t gofs = (int64_t)hdr.tok[l + q] * p.ldy + p.y_off + off + c;
+                        const int64_t gofs = (int64_t)hdr.tok[l + q] * pj.ldy + pj.y_off + off + c;
                         if constexpr (CPT == 2) {
                             const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
                             const float y0 = fmaf(sc, acc[0], bf16_lo(w));
                             const float y1 = fmaf(sc, acc[1], bf16_hi(w));
-                            *reinterpret_cast<uint32_t *>(static_cast<E *>(p.y) + gofs) = pack_bf16x2(y0, y1);
+                            *reinterpret_cast<uint32_t *>(static_cast<E *>(pj.y) + gofs) = pack_bf16x2(y0, y1);
                         } else {
                             const float w = *reinterpret_cast<const float *>(yr);
-                            static_cast<float *>(p.y)[gofs] = fmaf(sc, acc[0], w);
+                            static_cast<float *>(pj.y)[gofs] = fmaf(sc, acc[0], w);
                         }
                     }
                 }
@@ -864,7 +884,7 @@ int launch_typed(int mode, int src, const DecodeParams &p, cudaStream_t s)
 
 int launch_decode(int mode, int src, const DecodeParams &p, int dtype, cudaStream_t s)
 {
-    if (!p.tmA) return LORA_ERR_INVALID_ARG;
+    if (!p.pj[0].tmA || p.P < 1 || p.P > kMaxProj) return LORA_ERR_INVALID_ARG;
     if (dtype == LORA_BF16) return launch_typed<__nv_bfloat16>(mode, src, p, s);
     if (dtype == LORA_F32) return launch_typed<float>(mode, src, p, s);
     return LORA_ERR_UNSUPPORTED;

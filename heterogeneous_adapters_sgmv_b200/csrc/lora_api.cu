@@ -45,6 +45,7 @@ using namespace lora;
 
 namespace {
 
+static_assert(kMaxProj == LORA_MAX_GROUP, "grouped-call limit");
 constexpr int kBgmvMaxT = 1024;
 constexpr int kBgmvMaxN = 4096;
 
@@ -110,11 +111,12 @@ DecodeParams base_params(const lora_table *t)
 {
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
-    p.desc = t->d_desc;
-    p.tmA = t->d_tmaps;
+    p.pj[0].desc = t->d_desc;
+    p.pj[0].tmA = t->d_tmaps;
+    p.pj[0].h = t->h;
+    p.pj[0].o = t->o;
+    p.P = 1;
     p.n = t->n;
-    p.h = t->h;
-    p.o = t->o;
     p.R = t->max_rank;
     p.status = t->d_status;
     return p;
@@ -262,8 +264,8 @@ int lora_shrink(const lora_table *t, const lora_segments *seg, const void *x, in
     if (seg->T == 0 || seg->max_segs == 0) return LORA_OK;
     DecodeParams p = base_params(t);
     set_segments(p, seg);
-    p.x = x;
-    p.ldx = ldx;
+    p.pj[0].x = x;
+    p.pj[0].ldx = ldx;
     p.v = v;
     p.ldv = ldv;
     return launch_decode(kModeShrink, kSrcSegments, p, t->dtype, static_cast<cudaStream_t>(stream));
@@ -281,9 +283,9 @@ int lora_expand(const lora_table *t, const lora_segments *seg, const float *v, i
     if (seg->T == 0 || seg->max_segs == 0) return LORA_OK;
     DecodeParams p = base_params(t);
     set_segments(p, seg);
-    p.y = y;
-    p.ldy = ldy;
-    p.y_off = y_off;
+    p.pj[0].y = y;
+    p.pj[0].ldy = ldy;
+    p.pj[0].y_off = y_off;
     p.v = const_cast<float *>(v);
     p.ldv = ldv;
     return launch_decode(kModeExpand, kSrcSegments, p, t->dtype, static_cast<cudaStream_t>(stream));
@@ -312,12 +314,75 @@ int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int6
     }
     DecodeParams p = base_params(t);
     set_segments(p, seg);
-    p.x = x;
-    p.ldx = ldx;
-    p.y = y;
-    p.ldy = ldy;
-    p.y_off = y_off;
+    p.pj[0].x = x;
+    p.pj[0].ldx = ldx;
+    p.pj[0].y = y;
+    p.pj[0].ldy = ldy;
+    p.pj[0].y_off = y_off;
     return launch_decode(kModeFused, kSrcSegments, p, t->dtype, s);
+}
+
+int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_segments *seg,
+                      const void *const *x, const int64_t *ldx, void *const *y, const int64_t *ldy,
+                      const int32_t *y_off, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!tables || !x || !ldx || !y || !ldy || !y_off) return LORA_ERR_INVALID_ARG;
+    if (P < 1 || P > kMaxProj) return LORA_ERR_INVALID_ARG;
+    int rc;
+    if ((rc = check_segments(seg))) return rc;
+    for (int i = 0; i < P; ++i) {
+        if ((rc = check_table(tables[i]))) return rc;
+        if (tables[i]->n != tables[0]->n || tables[i]->dtype != tables[0]->dtype ||
+            tables[i]->device != tables[0]->device)
+            return LORA_ERR_INVALID_ARG;
+        if ((rc = check_io(tables[i], x[i], ldx[i], y[i], ldy[i], y_off[i], true, true))) return rc;
+    }
+    // The output slices must not overlap: the projections update y concurrently.
+    const int e = esz(tables[0]->dtype);
+    for (int i = 0; i < P; ++i)
+        for (int j = i + 1; j < P; ++j) {
+            const int64_t a0 = y_off[i], a1 = a0 + tables[i]->o, b0 = y_off[j], b1 = b0 + tables[j]->o;
+            if (y[i] == y[j] && ldy[i] == ldy[j]) {
+                if (a0 < b1 && b0 < a1) return LORA_ERR_INVALID_ARG;
+                continue;
+            }
+            const int64_t rows = seg->T > 0 ? seg->T - 1 : 0;
+            const uintptr_t pi0 = reinterpret_cast<uintptr_t>(y[i]) + (uintptr_t)(a0 * e);
+            const uintptr_t pi1 = reinterpret_cast<uintptr_t>(y[i]) + (uintptr_t)((rows * ldy[i] + a1) * e);
+            const uintptr_t pj0 = reinterpret_cast<uintptr_t>(y[j]) + (uintptr_t)(b0 * e);
+            const uintptr_t pj1 = reinterpret_cast<uintptr_t>(y[j]) + (uintptr_t)((rows * ldy[j] + b1) * e);
+            if (pi0 < pj1 && pj0 < pi1) return LORA_ERR_INVALID_ARG;
+        }
+    if (seg->T == 0 || seg->max_segs == 0) return LORA_OK;
+    const Options &opt = options();
+    bool separate = opt.split != 0;
+    for (int i = 0; i < P; ++i)
+        separate |= opt.prefill_min_seg_len > 0 && seg->max_seg_len >= opt.prefill_min_seg_len &&
+                    seg->perm == nullptr && prefill_supported(tables[i]);
+    if (separate) {   // long segments (tcgen05 path) or the split option: one call per table
+        for (int i = 0; i < P; ++i)
+            if ((rc = lora_sgmv(tables[i], seg, x[i], ldx[i], y[i], ldy[i], y_off[i], ws, ws_bytes, stream)))
+                return rc;
+        return LORA_OK;
+    }
+    DecodeParams p = base_params(tables[0]);
+    set_segments(p, seg);
+    p.P = P;
+    for (int i = 0; i < P; ++i) {
+        const lora_table *t = tables[i];
+        ProjParams &pj = p.pj[i];
+        pj.desc = t->d_desc;
+        pj.tmA = t->d_tmaps;
+        pj.h = t->h;
+        pj.o = t->o;
+        pj.x = x[i];
+        pj.ldx = ldx[i];
+        pj.y = y[i];
+        pj.ldy = ldy[i];
+        pj.y_off = y_off[i];
+        if (t->max_rank > p.R) p.R = t->max_rank;
+    }
+    return launch_decode(kModeFused, kSrcSegments, p, tables[0]->dtype, static_cast<cudaStream_t>(stream));
 }
 
 int lora_bgmv(const lora_table *t, const int32_t *d_ids, int32_t T, const void *x, int64_t ldx, void *y,
@@ -334,11 +399,11 @@ int lora_bgmv(const lora_table *t, const int32_t *d_ids, int32_t T, const void *
         DecodeParams p = base_params(t);
         p.ids = d_ids;
         p.T = T;
-        p.x = x;
-        p.ldx = ldx;
-        p.y = y;
-        p.ldy = ldy;
-        p.y_off = y_off;
+        p.pj[0].x = x;
+        p.pj[0].ldx = ldx;
+        p.pj[0].y = y;
+        p.pj[0].ldy = ldy;
+        p.pj[0].y_off = y_off;
         return launch_decode(kModeFused, kSrcIds, p, t->dtype, s);
     }
     // Larger batches: sort into the workspace, then run the segmented form.

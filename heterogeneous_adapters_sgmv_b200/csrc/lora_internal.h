@@ -19,15 +19,24 @@ enum DecodeMode : int { kModeFused = 0, kModeShrink = 1, kModeExpand = 2 };
 // Where the work units come from: a segment table, or per-token ids grouped on the device.
 enum UnitSource : int { kSrcSegments = 0, kSrcIds = 1 };
 
-struct DecodeParams {
+// One projection (one adapter table with its activations) of a decode launch.  A grouped
+// launch carries up to kMaxProj of them over one segment table.
+struct ProjParams {
     const AdapterDesc *desc;
     const void *tmA;       // device array of 128-byte tensor maps, one per adapter (A_i slices)
-    int32_t n, h, o, R;    // adapters, in/out features, max rank of the table
     const void *x;
-    int64_t ldx;
     void *y;
-    int64_t ldy;
+    int64_t ldx, ldy;
+    int32_t h, o;          // in/out features
     int32_t y_off;
+    int32_t pad_;
+};
+constexpr int kMaxProj = 4;
+
+struct DecodeParams {
+    ProjParams pj[kMaxProj];
+    int32_t P;             // projections in this launch (1 unless grouped)
+    int32_t n, R;          // adapters per table, max rank over the launch's tables
     int32_t ldv;
     float *v;
     const int32_t *perm, *seg_ptr, *seg_adapter, *num_segs;

@@ -144,6 +144,25 @@ int lora_expand(const lora_table *table, const lora_segments *seg, const float *
 int lora_sgmv(const lora_table *table, const lora_segments *seg, const void *x, int64_t ldx,
               void *y, int64_t ldy, int32_t y_offset, void *ws, size_t ws_bytes, void *stream);
 
+/* Grouped SGMV: P <= LORA_MAX_GROUP projections of one batch in one launch, e.g. the q, k and
+ * v (and o) projections of a layer, each with its own adapter table but one shared segment
+ * table (the same adapter id selects adapter i of every table).  Projection p computes
+ * y[p][t, y_offset[p] + n] += s_i * (x[p][t] . A_i^T) . B_i^T exactly as lora_sgmv with
+ * tables[p] would, and per output the arithmetic is the same as that call's, so results
+ * match it bit for bit (at the same "decode_cluster" width).  The per-call y_offset /
+ * y_slice_size of the pages' pseudocode ("Compress then Serve" review thread, add_lora_slice)
+ * is what lets q, k and v write their slices of one fused output.
+ * Arguments: host arrays of P entries (tables, x, ldx, y, ldy, y_offset); the tables must
+ * have the same n, dtype and device; x[p] may repeat (q, k and v share x); the output
+ * slices must not overlap (LORA_ERR_INVALID_ARG), because the projections update y
+ * concurrently.  Device errors latch into tables[0]'s status word.  When a table qualifies
+ * for the tcgen05 path (long contiguous segments) or the "split" option is set, the call
+ * runs lora_sgmv once per table instead (ws as for lora_sgmv). */
+#define LORA_MAX_GROUP 4
+int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_segments *seg,
+                      const void *const *x, const int64_t *ldx, void *const *y, const int64_t *ldy,
+                      const int32_t *y_offset, void *ws, size_t ws_bytes, void *stream);
+
 /* BGMV: the same update driven by per-token ids (d_ids[T], device) without a caller-built
  * segment table, as the per-token "indices" of the pseudocode.  Tokens sharing an adapter
  * are grouped on the device so each adapter's weights are read once per group.  For

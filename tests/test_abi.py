@@ -34,6 +34,18 @@ def test_host_only_calls():
     assert lib.lora_table_info(None, None, None, None, None, None) == L.LORA_ERR_INVALID_ARG
     assert lib.lora_workspace_bytes(None, 5) == 256
     assert lib.lora_table_destroy(None) == L.LORA_OK
+    # grouped call: argument checks that need no table
+    arr = (ctypes.c_void_p * 5)()
+    i64 = (ctypes.c_int64 * 5)()
+    i32 = (ctypes.c_int32 * 5)()
+    seg = L.lora_segments()
+    for P in (0, 5, -1):
+        assert lib.lora_sgmv_grouped(arr, P, ctypes.byref(seg), arr, i64, arr, i64, i32, None, 0,
+                                     None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_sgmv_grouped(None, 1, ctypes.byref(seg), arr, i64, arr, i64, i32, None, 0,
+                                 None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_sgmv_grouped(arr, 1, ctypes.byref(seg), arr, i64, arr, i64, i32, None, 0,
+                                 None) == L.LORA_ERR_INVALID_ARG   # null segment pointers / table
     old = L.lora_get_option("split")
     L.lora_set_option("split", 1)
     assert L.lora_get_option("split") == 1
@@ -51,7 +63,7 @@ def test_header_constants_match_binding():
     for name in ("LORA_F32", "LORA_BF16", "LORA_OK", "LORA_ERR_INVALID_ARG", "LORA_ERR_UNSUPPORTED",
                  "LORA_ERR_WORKSPACE", "LORA_ERR_CUDA", "LORA_ERR_TIMEOUT", "LORA_ERR_DEVICE_STATUS",
                  "LORA_STATUS_BAD_ID", "LORA_STATUS_TIMEOUT", "LORA_STATUS_BAD_SEGMENT", "LORA_MAX_RANK",
-                 "LORA_MAX_SEGMENT_TOKENS", "LORA_NOALLOC_SCRATCH_FLOATS"):
+                 "LORA_MAX_SEGMENT_TOKENS", "LORA_NOALLOC_SCRATCH_FLOATS", "LORA_MAX_GROUP"):
         m = re.search(r"#define %s \(?(-?\d+)u?\)?" % name, txt)
         assert m, name
         assert int(m.group(1)) == getattr(L, name), name

@@ -35,14 +35,21 @@ def projection_flops(ids: np.ndarray, ranks: np.ndarray, h: int, o: int) -> int:
     return int(2 * (r * h).sum() + 2 * (r * o).sum())
 
 
-def workload_bytes(wl) -> int:
-    """Algorithmic bytes of one step of a workload (all projections)."""
+def workload_bytes(wl, shared_x: bool = False) -> int:
+    """Algorithmic bytes of one step of a workload (all projections).  With ``shared_x`` the
+    projections that read the same activations (q, k and v) count x once, as one grouped
+    launch reads it."""
     e = ELEM_BYTES[wl.dtype]
     d = distinct_adapters(wl.ids)
     T_valid = int((np.asarray(wl.ids) >= 0).sum())
     tot = 0
-    for p in wl.projections:
+    seen = set()
+    groups = [g for (_n, _h, _o, g) in wl.spec.projections] if shared_x else range(len(wl.projections))
+    for p, g in zip(wl.projections, groups):
         tot += projection_bytes(T_valid, p.h, p.o, (p.ranks[i] for i in d), e)
+        if g in seen:
+            tot -= T_valid * p.h * e
+        seen.add(g)
     return tot
 
 
