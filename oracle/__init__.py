@@ -13,6 +13,9 @@ Two independent implementations live here:
   Foundation: LoRA") and the add_lora_slice pseudocode of the "Compress then Serve"
   review thread (authors' rebuttal on Punica).  Also the stable segment bookkeeping that
   SGMV's grouping of same-adapter requests implies.
+  The same file holds the three-stage form of that thread's add_lora_slice_with_sigma
+  pseudocode (A with scale 1, then the adapter's small Sigma_i, full or diagonal, with
+  scale 1, then B with the scale).
 * ``brute.py``: numpy fp64 matrix products per adapter group (a different evaluation
   order), used to cross-check the loop.
 
@@ -62,6 +65,12 @@ def bind(path: str):
     lib.oracle_lora_expand.argtypes = [ctypes.c_int, i64, i64, P, i64, P, i64, i64, P, i32,
                                        P, P, P, P, ctypes.c_int]
     lib.oracle_lora_expand.restype = ctypes.c_int
+    lib.oracle_lora_delta_sigma.argtypes = [ctypes.c_int, i64, i64, i64, P, i64, P, i64, i64,
+                                            P, i32, P, P, P, P, ctypes.c_int, P, P, ctypes.c_int]
+    lib.oracle_lora_delta_sigma.restype = ctypes.c_int
+    lib.oracle_lora_shrink_sigma.argtypes = [ctypes.c_int, i64, i64, P, i64, P, i32, P, P, ctypes.c_int, P, P,
+                                             i64, ctypes.c_int]
+    lib.oracle_lora_shrink_sigma.restype = ctypes.c_int
     lib.oracle_build_segments.argtypes = [i64, P, i32, P, P, P, P]
     lib.oracle_build_segments.restype = ctypes.c_int64
     lib.oracle_max_threads.argtypes = []
@@ -168,6 +177,75 @@ def lora_expand(dtype: str, v: np.ndarray, y0: np.ndarray, ids: np.ndarray,
     if rc != 0:
         raise OracleError("adapter id out of range")
     return out
+
+
+SIGMA_NONE, SIGMA_FULL, SIGMA_DIAG = 0, 1, 2
+
+
+def _sigma_arrays(sigma_kind: int, sigma, ranks: np.ndarray):
+    if sigma_kind not in (SIGMA_NONE, SIGMA_FULL, SIGMA_DIAG):
+        raise ValueError("sigma_kind")
+    if sigma_kind == SIGMA_NONE:
+        return [], None
+    Ss = [np.ascontiguousarray(sg, dtype=np.float32) for sg in sigma]
+    for sg, r in zip(Ss, ranks):
+        want = (r, r) if sigma_kind == SIGMA_FULL else (r,)
+        if sg.shape != want:
+            raise ValueError("Sigma shape %s, want %s" % (sg.shape, want))
+    return Ss, (ctypes.c_void_p * max(len(Ss), 1))(*[_ptr(sg) for sg in Ss])
+
+
+def lora_delta_sigma(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray,
+                     A: Sequence[np.ndarray], B: Sequence[np.ndarray], scales: Sequence[float],
+                     sigma_kind: int, sigma: Sequence[np.ndarray], y_offset: int = 0,
+                     o: Optional[int] = None, threads: int = 0) -> np.ndarray:
+    """Three-stage form: fp64 y_ref = y0 + s_i B_i (Sigma_i (A_i x[t])) -- Sigma_i full
+    (r_i x r_i) or diagonal (r_i values), fp32 values."""
+    x = _check_store(x, dtype)
+    y0 = _check_store(y0, dtype)
+    T, h = x.shape
+    if o is None:
+        o = y0.shape[1] - y_offset
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    n = len(A)
+    As = [_check_store(a, dtype) for a in A]
+    Bs = [_check_store(b, dtype) for b in B]
+    ranks = np.array([a.shape[0] for a in As], dtype=np.int32)
+    for a, b, r in zip(As, Bs, ranks):
+        if a.shape != (r, h) or b.shape != (o, r):
+            raise ValueError("adapter shapes %s / %s do not match h=%d o=%d" % (a.shape, b.shape, h, o))
+    Ss, Sp = _sigma_arrays(sigma_kind, sigma, ranks)
+    Ap = (ctypes.c_void_p * max(n, 1))(*[_ptr(a) for a in As])
+    Bp = (ctypes.c_void_p * max(n, 1))(*[_ptr(b) for b in Bs])
+    sc = np.ascontiguousarray(np.asarray(scales, dtype=np.float32).astype(np.float64))
+    out = np.empty((T, o), dtype=np.float64)
+    rc = _load().oracle_lora_delta_sigma(_dtype_code(dtype), T, h, o, _ptr(x), x.shape[1], _ptr(y0),
+                                         y0.shape[1], y_offset, _ptr(ids), n, Ap, Bp, _ptr(ranks),
+                                         _ptr(sc), sigma_kind, Sp, _ptr(out), threads)
+    if rc != 0:
+        raise OracleError("adapter id out of range")
+    return out
+
+
+def lora_shrink_sigma(dtype: str, x: np.ndarray, ids: np.ndarray, A: Sequence[np.ndarray],
+                      sigma_kind: int, sigma: Sequence[np.ndarray], ldv: Optional[int] = None,
+                      threads: int = 0) -> np.ndarray:
+    """Steps 1 and 2 of the three-stage form: fp64 v[t, :r_i] = Sigma_i (A_i x[t])."""
+    x = _check_store(x, dtype)
+    T, h = x.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    As = [_check_store(a, dtype) for a in A]
+    ranks = np.array([a.shape[0] for a in As], dtype=np.int32)
+    if ldv is None:
+        ldv = int(ranks.max()) if len(ranks) else 1
+    Ss, Sp = _sigma_arrays(sigma_kind, sigma, ranks)
+    Ap = (ctypes.c_void_p * max(len(As), 1))(*[_ptr(a) for a in As])
+    v = np.empty((T, ldv), dtype=np.float64)
+    rc = _load().oracle_lora_shrink_sigma(_dtype_code(dtype), T, h, _ptr(x), x.shape[1], _ptr(ids), len(As), Ap,
+                                          _ptr(ranks), sigma_kind, Sp, _ptr(v), ldv, threads)
+    if rc != 0:
+        raise OracleError("adapter id out of range")
+    return v
 
 
 def build_segments(ids: np.ndarray, n_adapters: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:

@@ -203,6 +203,132 @@ int oracle_lora_expand(int dtype, int64_t T, int64_t o,
 }
 
 /*
+ * Three-stage form of the "Compress then Serve" review thread (authors' rebuttal on Punica,
+ * pseudocode of add_lora_slice_with_sigma): step 1 applies A_i to x with scale 1 into a
+ * buffer of width R, step 2 applies the adapter's small matrix Sigma_i to that buffer with
+ * scale 1, step 3 applies B_i with the adapter scale and updates the y slice:
+ *
+ *   u[k]        = sum_j x[t, j] * A_i[k, j]                       k < r_i
+ *   w[k]        = sum_m Sigma_i[k, m] * u[m]        (sigma_kind 1: r_i x r_i, row-major)
+ *               = Sigma_i[k] * u[k]                 (sigma_kind 2: diagonal, r_i values)
+ *               = u[k]                              (sigma_kind 0: no Sigma)
+ *   y_ref[t, n] = y0[t, y_offset + n] + s_i * sum_k B_i[n, k] * w[k]
+ *
+ * Sigma[i] points to fp32 values (widened exactly).  The pages name the two Sigma shapes
+ * JD-Full and JD-Diag; where the adapters of one cluster share A and B, the caller passes
+ * the same A / B pointer for each of them.  Other arguments as oracle_lora_delta.
+ */
+static void sigma_step(int sigma_kind, const float *S, int32_t r, const double *u, double *w)
+{
+    for (int32_t k = 0; k < r; ++k) {
+        if (sigma_kind == 1) {
+            double acc = 0.0;
+            for (int32_t m = 0; m < r; ++m)
+                acc += (double)S[(int64_t)k * r + m] * u[m];
+            w[k] = acc;
+        } else if (sigma_kind == 2) {
+            w[k] = (double)S[k] * u[k];
+        } else {
+            w[k] = u[k];
+        }
+    }
+}
+
+int oracle_lora_delta_sigma(int dtype, int64_t T, int64_t h, int64_t o,
+                            const void *x, int64_t ldx,
+                            const void *y0, int64_t ldy, int64_t y_offset,
+                            const int32_t *ids, int32_t n_adapters,
+                            const void *const *A, const void *const *B,
+                            const int32_t *ranks, const double *scales,
+                            int sigma_kind, const float *const *Sigma,
+                            double *y_ref, int n_threads)
+{
+    if (!ids_valid(T, ids, n_adapters) || sigma_kind < 0 || sigma_kind > 2)
+        return -1;
+    set_threads(n_threads);
+#pragma omp parallel
+    {
+        double *u = NULL, *w = NULL;
+        int32_t cap = 0;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < T; ++t) {
+            double *yr = y_ref + t * o;
+            for (int64_t n = 0; n < o; ++n)
+                yr[n] = widen(y0, dtype, t * ldy + y_offset + n);
+            int32_t i = ids[t];
+            if (i < 0)
+                continue;
+            int32_t r = ranks[i];
+            if (r > cap) {
+                free(u);
+                free(w);
+                u = (double *)malloc((size_t)r * sizeof(double));
+                w = (double *)malloc((size_t)r * sizeof(double));
+                cap = r;
+            }
+            /* step 1: u = A_i x, scale 1 */
+            for (int32_t k = 0; k < r; ++k) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < h; ++j)
+                    acc += widen(x, dtype, t * ldx + j) * widen(A[i], dtype, (int64_t)k * h + j);
+                u[k] = acc;
+            }
+            /* step 2: w = Sigma_i u, scale 1 */
+            sigma_step(sigma_kind, sigma_kind ? Sigma[i] : NULL, r, u, w);
+            /* step 3: y += s_i * B_i w */
+            for (int64_t n = 0; n < o; ++n) {
+                double acc = 0.0;
+                for (int32_t k = 0; k < r; ++k)
+                    acc += widen(B[i], dtype, n * r + k) * w[k];
+                yr[n] += scales[i] * acc;
+            }
+        }
+        free(u);
+        free(w);
+    }
+    return 0;
+}
+
+/*
+ * Steps 1 and 2 of the three-stage form: v[t, k] = (Sigma_i (A_i x[t]))[k] for k < r_i;
+ * v is [T, ldv] doubles, other entries 0.  Arguments as oracle_lora_shrink plus Sigma.
+ */
+int oracle_lora_shrink_sigma(int dtype, int64_t T, int64_t h,
+                             const void *x, int64_t ldx,
+                             const int32_t *ids, int32_t n_adapters,
+                             const void *const *A, const int32_t *ranks,
+                             int sigma_kind, const float *const *Sigma,
+                             double *v, int64_t ldv, int n_threads)
+{
+    if (!ids_valid(T, ids, n_adapters) || sigma_kind < 0 || sigma_kind > 2)
+        return -1;
+    set_threads(n_threads);
+#pragma omp parallel
+    {
+        double *u = (double *)malloc((size_t)(ldv > 0 ? ldv : 1) * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < T; ++t) {
+            double *vr = v + t * ldv;
+            for (int64_t k = 0; k < ldv; ++k)
+                vr[k] = 0.0;
+            int32_t i = ids[t];
+            if (i < 0)
+                continue;
+            int32_t r = ranks[i];
+            for (int32_t k = 0; k < r; ++k) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < h; ++j)
+                    acc += widen(x, dtype, t * ldx + j) * widen(A[i], dtype, (int64_t)k * h + j);
+                u[k] = acc;
+            }
+            sigma_step(sigma_kind, sigma_kind ? Sigma[i] : NULL, r, u, vr);
+        }
+        free(u);
+    }
+    return 0;
+}
+
+/*
  * Segment bookkeeping: a stable counting sort of the tokens by adapter id.
  *   perm[p]          token index at sorted position p (p < number of tokens with an adapter)
  *   seg_ptr[s]       first sorted position of segment s; seg_ptr[num_segs] = valid tokens

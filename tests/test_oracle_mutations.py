@@ -19,20 +19,35 @@ MUTATIONS = {
     "transposed_A": ("acc += xrow[j] * widen(A[i], dtype, (int64_t)k * h + j)",
                      "acc += xrow[j] * widen(A[i], dtype, (int64_t)j * r + k)"),
     "transposed_B": ("widen(B[i], dtype, n * r + k) * v[k]", "widen(B[i], dtype, (int64_t)k * o + n) * v[k]"),
-    "dropped_y0": ("yr[n] = widen(y0, dtype, t * ldy + y_offset + n);\n            int32_t i",
-                   "yr[n] = 0.0;\n            int32_t i"),
+    "dropped_y0": ("yr[n] = widen(y0, dtype, t * ldy + y_offset + n);\n            int32_t i = ids[t];\n"
+                   "            if (i < 0)\n                continue;\n            int32_t r = ranks[i];\n"
+                   "            if (r > vcap)",
+                   "yr[n] = 0.0;\n            int32_t i = ids[t];\n"
+                   "            if (i < 0)\n                continue;\n            int32_t r = ranks[i];\n"
+                   "            if (r > vcap)"),
     "scale_squared": ("yr[n] += scales[i] * acc;\n            }\n        }\n        free(v);",
                       "yr[n] += scales[i] * scales[i] * acc;\n            }\n        }\n        free(v);"),
     "scale_dropped": ("yr[n] += scales[i] * acc;\n            }\n        }\n        free(v);",
                       "yr[n] += acc;\n            }\n        }\n        free(v);"),
-    "neighbour_id": ("int32_t i = ids[t];\n            if (i < 0)\n                continue;\n            int32_t r",
-                     "int32_t i = ids[(t + 1) % T];\n            if (i < 0)\n                continue;\n            int32_t r"),
+    "neighbour_id": ("int32_t i = ids[t];\n            if (i < 0)\n                continue;\n"
+                     "            int32_t r = ranks[i];\n            if (r > vcap)",
+                     "int32_t i = ids[(t + 1) % T];\n            if (i < 0)\n                continue;\n"
+                     "            int32_t r = ranks[i];\n            if (r > vcap)"),
     "rank_off_by_one": ("for (int32_t k = 0; k < r; ++k) {\n                double acc = 0.0;\n                for (int64_t j = 0; j < h; ++j)\n                    acc += xrow[j]",
                         "for (int32_t k = 0; k < r - 1; ++k) {\n                double acc = 0.0;\n                for (int64_t j = 0; j < h; ++j)\n                    acc += xrow[j]"),
     "unstable_segments": ("for (int64_t t = 0; t < T; ++t)\n        if (ids[t] >= 0)\n            perm[next[ids[t]]++]",
                           "for (int64_t t = T - 1; t >= 0; --t)\n        if (ids[t] >= 0)\n            perm[next[ids[t]]++]"),
-    "offset_ignored": ("widen(y0, dtype, t * ldy + y_offset + n);\n            int32_t i",
-                       "widen(y0, dtype, t * ldy + n);\n            int32_t i"),
+    "offset_ignored": ("widen(y0, dtype, t * ldy + y_offset + n);\n            int32_t i = ids[t];\n"
+                       "            if (i < 0)\n                continue;\n            int32_t r = ranks[i];\n"
+                       "            if (r > vcap)",
+                       "widen(y0, dtype, t * ldy + n);\n            int32_t i = ids[t];\n"
+                       "            if (i < 0)\n                continue;\n            int32_t r = ranks[i];\n"
+                       "            if (r > vcap)"),
+    "sigma_transposed": ("acc += (double)S[(int64_t)k * r + m] * u[m];", "acc += (double)S[(int64_t)m * r + k] * u[m];"),
+    "sigma_full_skipped": ("            w[k] = acc;\n        } else if", "            w[k] = u[k];\n        } else if"),
+    "sigma_diag_skipped": ("w[k] = (double)S[k] * u[k];", "w[k] = u[k];"),
+    "sigma_scale_dropped": ("yr[n] += scales[i] * acc;\n            }\n        }\n        free(u);",
+                            "yr[n] += acc;\n            }\n        }\n        free(u);"),
 }
 
 PIN_TESTS = [
@@ -47,6 +62,10 @@ PIN_TESTS = [
     pins.test_output_slice_offset,
     pins.test_exhaustive_tiny_against_outer_products,
     lambda: [pins.test_segments_equal_stable_argsort(s) for s in (1, 2)],
+    lambda: [pins.test_sigma_identity_is_the_plain_delta(k) for k in ("full", "diag")],
+    pins.test_sigma_diagonal_of_powers_of_two_folds_into_B,
+    lambda: [pins.test_sigma_equals_merged_three_factor_weight(k) for k in ("full", "diag")],
+    pins.test_sigma_shrink_is_sigma_times_shrink,
 ]
 
 

@@ -328,3 +328,116 @@ def test_recipe_is_deterministic_and_rounded():
     assert counts[0] == counts.max() and set(z.projections[0].ranks) <= {8, 16, 32, 64}
     pf = workloads.generate("prefill_sgmv", shapes=[("up", 8, 8, 0)])
     assert np.array_equal(pf.ids, np.repeat(np.arange(8), 512))
+
+
+# ------------------------------------------------------------------ three-stage form (Sigma)
+# "Compress then Serve" review thread, add_lora_slice_with_sigma pseudocode: A with scale 1,
+# then the adapter's Sigma with scale 1, then B with the scale into the y slice.
+
+def _sigma_case(dtype="bf16"):
+    if dtype == "f32":
+        wl = workloads.generate("tiny_sgmv", T=30, n=5)
+    else:
+        wl = workloads.generate("multirank_decode", T=40, n=7, shapes=[("q", 192, 136, 0)], ranks=(3, 8, 16))
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    return wl, p, A, B
+
+
+@pytest.mark.parametrize("kind", ["full", "diag"])
+def test_sigma_identity_is_the_plain_delta(kind):
+    """Sigma_i = I (full) or all ones (diagonal) multiplies by exactly 1 and adds exact zeros,
+    so the three-stage result equals the two-stage one bit for bit."""
+    wl, p, A, B = _sigma_case()
+    sig = [np.eye(a.shape[0], dtype=np.float32) if kind == "full" else np.ones(a.shape[0], np.float32) for a in A]
+    plain = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    three = oracle.lora_delta_sigma(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales,
+                                    oracle.SIGMA_FULL if kind == "full" else oracle.SIGMA_DIAG, sig)
+    assert np.array_equal(plain, three)
+
+
+def test_sigma_diagonal_of_powers_of_two_folds_into_B():
+    """A diagonal Sigma of powers of two can be folded into B exactly (B' = B diag(d), every
+    product exact in fp32): the three-stage result equals the plain one with B'."""
+    wl, p, A, B = _sigma_case("f32")
+    rng = np.random.default_rng(3)
+    d = [np.ldexp(1.0, rng.integers(-3, 4, size=a.shape[0])).astype(np.float32) for a in A]
+    Bf = [(b * di[None, :]).astype(np.float32) for b, di in zip(B, d)]
+    plain = oracle.lora_delta("f32", p.x, p.y0, wl.ids, A, Bf, p.scales)
+    three = oracle.lora_delta_sigma("f32", p.x, p.y0, wl.ids, A, B, p.scales, oracle.SIGMA_DIAG, d)
+    assert np.array_equal(plain, three)
+
+
+@pytest.mark.parametrize("kind", ["full", "diag"])
+def test_sigma_equals_merged_three_factor_weight(kind):
+    """Per token, y = y0 + s_i (B_i Sigma_i A_i) x with the o x h product formed first in
+    fp64 (a different evaluation order); a non-symmetric Sigma catches a transposed Sigma."""
+    wl, p, A, B = _sigma_case()
+    sig = workloads.draw_sigma(p.ranks, kind, seed=11)
+    got = oracle.lora_delta_sigma(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales,
+                                  oracle.SIGMA_FULL if kind == "full" else oracle.SIGMA_DIAG, sig)
+    x = to_float64(p.x, wl.dtype)
+    want = to_float64(p.y0, wl.dtype).copy()
+    for i in range(wl.n):
+        S = sig[i].astype(np.float64)
+        S = S if kind == "full" else np.diag(S)
+        W = float(p.scales[i]) * (to_float64(B[i], wl.dtype) @ S @ to_float64(A[i], wl.dtype))
+        rows = wl.ids == i
+        want[rows] += x[rows] @ W.T
+    scale = np.abs(want).max()
+    assert np.abs(got - want).max() <= 1e-12 * scale
+
+
+def test_sigma_delta_linear_in_sigma():
+    """Doubling every Sigma_i doubles the delta exactly (delta-only: y0 = 0)."""
+    wl = workloads.generate("multirank_decode", delta_only=True, T=24, n=5, shapes=[("q", 128, 96, 0)])
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    sig = workloads.draw_sigma(p.ranks, "full", seed=2)
+    one = oracle.lora_delta_sigma(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales, oracle.SIGMA_FULL, sig)
+    two = oracle.lora_delta_sigma(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales, oracle.SIGMA_FULL,
+                                  [2 * s for s in sig])
+    assert np.array_equal(2 * one, two)
+
+
+def test_sigma_shrink_is_sigma_times_shrink():
+    """Steps 1 and 2 alone: v = Sigma_i (A_i x), against numpy applying Sigma to the plain
+    shrink (closed form); tokens without an adapter give zero rows."""
+    wl, p, A, B = _sigma_case()
+    ids = wl.ids.copy()
+    ids[::7] = -1
+    sig = workloads.draw_sigma(p.ranks, "full", seed=4)
+    R = int(p.ranks.max())
+    got = oracle.lora_shrink_sigma(wl.dtype, p.x, ids, A, oracle.SIGMA_FULL, sig, ldv=R)
+    x = to_float64(p.x, wl.dtype)
+    for t in range(wl.T):
+        i = ids[t]
+        if i < 0:
+            assert not got[t].any()
+            continue
+        r = A[i].shape[0]
+        u = to_float64(A[i], wl.dtype) @ x[t]
+        w = sig[i].astype(np.float64) @ u
+        assert np.abs(got[t, :r] - w).max() <= 1e-12 * max(np.abs(w).max(), 1e-30)
+        assert not got[t, r:].any()
+
+
+def test_sigma_shared_cluster_weights():
+    """Compressed serving shares A and B inside a cluster: adapters that point at the same
+    A_c, B_c and differ only in Sigma_i give, per token, y0 + s (B_c Sigma_i A_c) x."""
+    wl, p, A, B = _sigma_case()
+    cl = workloads.jd_clusters(wl.n, 2)
+    # members use their leader's weights (same rank inside a cluster by construction here)
+    ranks = np.array([A[c].shape[0] for c in cl])
+    A2 = [A[c] for c in cl]
+    B2 = [B[c] for c in cl]
+    sig = workloads.draw_sigma(ranks, "full", seed=8)
+    got = oracle.lora_delta_sigma(wl.dtype, p.x, p.y0, wl.ids, A2, B2, p.scales, oracle.SIGMA_FULL, sig)
+    x = to_float64(p.x, wl.dtype)
+    want = to_float64(p.y0, wl.dtype).copy()
+    for i in range(wl.n):
+        W = float(p.scales[i]) * (to_float64(B2[i], wl.dtype) @ sig[i].astype(np.float64) @
+                                  to_float64(A2[i], wl.dtype))
+        rows = wl.ids == i
+        want[rows] += x[rows] @ W.T
+    assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max()

@@ -258,3 +258,30 @@ def random_intermediate(T: int, R: int, seed: int) -> np.ndarray:
     """A seeded fp32 rank-space intermediate ``v[T, R]`` for expand-only runs."""
     rng = np.random.default_rng(seed)
     return rng.standard_normal((T, R)).astype(np.float32)
+
+
+SIGMA_KINDS = ("none", "full", "diag")
+
+
+def draw_sigma(ranks: np.ndarray, kind: str, seed: int) -> List[np.ndarray]:
+    """Seeded fp32 Sigma_i for the three-stage (compressed) form, one per adapter: "full" is
+    r_i x r_i with entries of variance 1/r_i (so Sigma_i u keeps the scale of u), "diag" is
+    r_i entries of variance 1.  Values are drawn in fp64 and rounded to fp32."""
+    if kind not in ("full", "diag"):
+        raise ValueError(kind)
+    rng = np.random.default_rng(seed)
+    out = []
+    for r in np.asarray(ranks, dtype=np.int64):
+        r = int(r)
+        if kind == "full":
+            out.append((rng.standard_normal((r, r)) * np.sqrt(1.0 / r)).astype(np.float32))
+        else:
+            out.append(rng.standard_normal(r).astype(np.float32))
+    return out
+
+
+def jd_clusters(n: int, clusters: int) -> np.ndarray:
+    """Cluster of each adapter for compressed serving with shared A and B: adapter i belongs
+    to cluster i mod clusters, and every member uses its cluster leader's (adapter c's)
+    A and B."""
+    return (np.arange(n) % max(1, clusters)).astype(np.int32)
