@@ -61,6 +61,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a graph")
+    ap.add_argument("--sigma", default="none", choices=["none", "full", "diag"],
+                    help="three-stage (compressed) form: a per-adapter Sigma_i between the A and B steps")
+    ap.add_argument("--jd-clusters", type=int, default=0,
+                    help="with --sigma: adapters share the A and B of adapter (i mod K), as compressed clusters do")
     ap.add_argument("--grouped", action="store_true",
                     help="many_adapter_qkvo: one lora_sgmv_grouped launch for q, k, v, o (q, k, v reading one x) "
                          "instead of four lora_sgmv calls")
@@ -145,14 +149,24 @@ class ClockSampler:
 class Copy:
     """One replica of the workload's inputs on the device plus its adapter tables."""
 
-    def __init__(self, wl, L, torch, shared_ids=None):
+    def __init__(self, wl, L, torch, sigma="none", clusters=0):
         from workloads.device import upload_projection
         self.projs = []
         self.tables = []
-        for p in wl.projections:
+        self.sigma = []
+        for pi, p in enumerate(wl.projections):
             d = upload_projection(p, wl.dtype)
-            t = L.AdapterTable(d.A_ptrs, d.B_ptrs, d.ranks, d.scales, p.h, p.o,
+            A, B, ranks = d.A_ptrs, d.B_ptrs, d.ranks
+            if clusters > 0:   # compressed clusters: members use their leader's A and B
+                cl = workloads.jd_clusters(wl.n, clusters)
+                A, B, ranks = [A[c] for c in cl], [B[c] for c in cl], [ranks[c] for c in cl]
+            t = L.AdapterTable(A, B, ranks, d.scales, p.h, p.o,
                                L.LORA_BF16 if wl.dtype == "bf16" else L.LORA_F32, keep=d)
+            if sigma != "none":
+                sg = [torch.from_numpy(a).cuda()
+                      for a in workloads.draw_sigma(np.asarray(ranks), sigma, seed=wl.seed + 77 + pi)]
+                t.set_sigma(L.LORA_SIGMA_FULL if sigma == "full" else L.LORA_SIGMA_DIAG, sg)
+                self.sigma.append(sg)
             self.projs.append(d)
             self.tables.append(t)
         self.ids = torch.from_numpy(wl.ids).cuda()
@@ -234,14 +248,16 @@ def run_ours(args, rank, world, local_rank):
     wl = workloads.generate(args.workload, seed=seed)
     T = wl.T
     step, launches_per_step, kname = make_step(wl, L, args.grouped)
-    bytes_step = accounting.workload_bytes(wl, shared_x=args.grouped)
+    if args.jd_clusters and args.sigma == "none":
+        raise SystemExit("--jd-clusters needs --sigma")
+    bytes_step = accounting.workload_bytes(wl, shared_x=args.grouped, sigma=args.sigma, clusters=args.jd_clusters)
     flops_step = accounting.workload_flops(wl)
     distinct = int(accounting.distinct_adapters(wl.ids).size)
 
-    first = Copy(wl, L, torch)
+    first = Copy(wl, L, torch, args.sigma, args.jd_clusters)
     ws_bytes = first.nbytes()
     C = args.copies or max(1, min(256, -(-4 * L2_BYTES // ws_bytes)))
-    copies = [first] + [Copy(wl, L, torch) for _ in range(C - 1)]
+    copies = [first] + [Copy(wl, L, torch, args.sigma, args.jd_clusters) for _ in range(C - 1)]
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
@@ -386,6 +402,8 @@ def run_ours(args, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_seconds)
+        if args.sigma != "none":
+            cpu["sample"] += "; two-stage oracle (the r x r Sigma step adds under 1 % of the work)"
 
     codes = {"bf16": "bf16", "f32": "f32"}
     out = {
@@ -400,6 +418,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "rotating %d input copies, %.0f MB in total against a 126 MB L2%s" % (
                        C, C * ws_bytes / 1e6, "" if C * ws_bytes >= 4 * L2_BYTES else " (copy count capped)"),
                    "graph": not args.no_graph, "pdl": bool(L.lora_get_option("pdl")),
+                   "sigma": args.sigma, "jd_clusters": args.jd_clusters,
                    "parallelism": "replicas x%d (independent token batches, no collective)" % world},
         "roofline": roofline,
         "cpu_baseline": cpu,

@@ -33,12 +33,15 @@ LORA_MAX_RANK = 128
 LORA_MAX_SEGMENT_TOKENS = 8192
 LORA_NOALLOC_SCRATCH_FLOATS = 262144
 LORA_MAX_GROUP = 4
+LORA_SIGMA_NONE = 0
+LORA_SIGMA_FULL = 1
+LORA_SIGMA_DIAG = 2
 
 EXPORTS = (
     "lora_table_create", "lora_table_destroy", "lora_table_info", "lora_workspace_bytes",
     "lora_build_segments", "lora_shrink", "lora_expand", "lora_sgmv", "lora_bgmv",
     "lora_get_status", "lora_status_string", "lora_set_option", "lora_get_option",
-    "lora_sgmv_noalloc", "lora_sgmv_grouped",
+    "lora_sgmv_noalloc", "lora_sgmv_grouped", "lora_table_set_sigma",
 )
 
 
@@ -77,6 +80,7 @@ def _load():
     sig = {
         "lora_table_create": ([ctypes.POINTER(P), I32, I32, I32, I32, P, P, P, P, P], ctypes.c_int),
         "lora_table_destroy": ([P], ctypes.c_int),
+        "lora_table_set_sigma": ([P, I32, P, P], ctypes.c_int),
         "lora_table_info": ([P, P, P, P, P, P], ctypes.c_int),
         "lora_workspace_bytes": ([P, I32], SZ),
         "lora_build_segments": ([P, P, I32, P, P, P, P, P], ctypes.c_int),
@@ -228,6 +232,13 @@ def lora_get_option(key: str) -> int:
     return int(v.value)
 
 
+def lora_table_set_sigma(table: int, kind: int, sigma: Optional[Sequence] = None, stream=None) -> None:
+    arr = None
+    if sigma is not None:
+        arr = (ctypes.c_void_p * len(sigma))(*[_ptr(sg) for sg in sigma])
+    _check(_load().lora_table_set_sigma(table, kind, arr, _stream(stream)), "lora_table_set_sigma")
+
+
 class AdapterTable:
     """Owns one ``lora_table`` and keeps the weight tensors it points to alive."""
 
@@ -252,3 +263,9 @@ class AdapterTable:
 
     def workspace_bytes(self, T: int) -> int:
         return lora_workspace_bytes(self.handle, T)
+
+    def set_sigma(self, kind: int, sigma: Optional[Sequence] = None, stream=None) -> None:
+        """Three-stage form: register Sigma_i per adapter (device fp32 tensors, [r_i, r_i] for
+        LORA_SIGMA_FULL or [r_i] for LORA_SIGMA_DIAG); LORA_SIGMA_NONE removes it."""
+        lora_table_set_sigma(self.handle, kind, sigma, stream)
+        self._sigma = list(sigma) if sigma is not None else None

@@ -63,6 +63,8 @@ struct __align__(16) StageHeader {
     float scale;
     int32_t L, off, len;   // tokens; first column of h (shrink) or row of o (expand); extent
     int32_t proj;          // projection of a grouped launch
+    int32_t skind;         // LORA_SIGMA_*: the unit's Sigma_i (three-stage form)
+    const float *sigma;
     int32_t tok[kTokChunk];
 };
 static_assert(sizeof(StageHeader) <= kHeaderBytes, "header");
@@ -248,6 +250,10 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     if (npre_all > 0 && tid == 0) {
         const AdapterDesc d0 = p.pj[0].desc[cid];
         for (int j = 0; j < npre_all; ++j) issue_tile(geo0, 0, j, cid, d0, j);
+        if (p.pj[0].sigma_kind != LORA_SIGMA_NONE) {
+            const int sbytes = (p.pj[0].sigma_kind == LORA_SIGMA_FULL ? d0.rank * d0.rank : d0.rank) * 4;
+            for (int c = 0; c < sbytes; c += 128) prefetch_l2(reinterpret_cast<const uint8_t *>(d0.sigma) + c);
+        }
     }
     pdl_wait();
     pdl_launch_dependents();
@@ -415,6 +421,11 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 const Geo g = pi == 0 ? geo0 : geo_of(pi);
                 const int r = d.rank;
                 const int ntiles = g.n_shrink + g.n_expand;
+                if (pj.sigma_kind != LORA_SIGMA_NONE) {   // the consumers read Sigma_i after the shrink
+                    const int sbytes = (pj.sigma_kind == LORA_SIGMA_FULL ? r * r : r) * 4;
+                    for (int c = lane * 128; c < sbytes; c += 32 * 128)
+                        prefetch_l2(reinterpret_cast<const uint8_t *>(d.sigma) + c);
+                }
                 for (int j = 0; j < ntiles; ++j) {
                     const int s = ps, m = pround;
                     if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
@@ -438,6 +449,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         hdr->off = off;
                         hdr->len = len;
                         hdr->proj = pi;
+                        hdr->skind = pj.sigma_kind;
+                        hdr->sigma = d.sigma;
                     }
                     __syncwarp();
                     if (lane == 0) {
@@ -540,6 +553,11 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
 
         if (kind == kTileShrink) {
             const bool first = flags & kFlagFirst;
+            if (first && hdr.skind != LORA_SIGMA_NONE) {   // Sigma_i is read after the exchange
+                const int sbytes = (hdr.skind == LORA_SIGMA_FULL ? r * r : r) * 4;
+                for (int c = tid * 128; c < sbytes; c += kConsumers * 128)
+                    prefetch_l1(reinterpret_cast<const uint8_t *>(hdr.sigma) + c);
+            }
             // ---- partial shrink over this CTA's slice of h: warp w owns rows w, w + 8, ...;
             // A is staged as [box][row][512 B] (box 1 after r rows of box 0), x as [token][row].
             // Two tokens x two rows at a time: a lane forms the four partial dot products over
@@ -600,15 +618,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 if (tid == 0 && u < 8) LORA_TRACE_MARK(33 + 4 * u);
                 named_bar_sync(1, kConsumers);
                 if (tid == 0) LORA_TRACE_MARK(16);
-                if constexpr (CL == 1) {
-                    // ---- no peers: vpart (= vsum) already holds the unit's intermediate
-                    if (MODE == kModeShrink) {
-                        for (int e = tid; e < (L << lgRP); e += kConsumers) {
-                            const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
-                            if (k < r) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = vsum[l * RP + k];
-                        }
-                    }
-                } else {
+                if constexpr (CL > 1) {
                     // ---- push the partial into every CTA of the cluster (this one included)
                     if (!cluster_waited) {
                         cluster_wait_acquire();   // every peer has initialised its barriers
@@ -639,7 +649,6 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
 #pragma unroll
                             for (int j = 0; j < CL; ++j) acc += recv[(j * kTokChunk + l) * RP + k];
                             vsum[l * RP + k] = acc;
-                            if (MODE == kModeShrink && crank == 0) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = acc;
                         }
                     }
                     if (tid == 0) LORA_TRACE_MARK(20);
@@ -647,6 +656,70 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     if (tid == 0) LORA_TRACE_MARK(21);
                     if (tid < CL) mbar_arrive_remote_relaxed(smem_u32(&ctl.freed), tid);
                     if (tid == 0) LORA_TRACE_MARK(22);
+                }
+                // (with CL == 1 vpart is vsum and already complete)
+                if (hdr.skind == LORA_SIGMA_FULL) {
+                    // ---- three-stage form, full Sigma_i: v[l] <- Sigma_i v[l] in fp32.  Thread
+                    // (k, g) forms output row k for tokens g, g + G, ...: each load of Sigma_i's
+                    // row k serves all of them; products are added in ascending m.
+                    const float *S = hdr.sigma;
+                    const int lgR = ceil_log2(r);
+                    const int G = kConsumers >> lgR;    // token groups (>= 2: r <= 128)
+                    const int k = tid & ((1 << lgR) - 1), g = tid >> lgR;
+                    float w[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) w[jj] = 0.f;
+                    if (k < r) {
+                        const float *Sk = S + (size_t)k * r;
+                        if ((r & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0) {
+                            for (int m = 0; m < r; m += 4) {
+                                const float4 s4 = __ldg(reinterpret_cast<const float4 *>(Sk + m));
+#pragma unroll
+                                for (int jj = 0; jj < 8; ++jj) {
+                                    const int l = g + G * jj;
+                                    if (l < L) {
+                                        const float4 v4 = *reinterpret_cast<const float4 *>(vsum + l * RP + m);
+                                        w[jj] = fmaf(s4.x, v4.x, w[jj]);
+                                        w[jj] = fmaf(s4.y, v4.y, w[jj]);
+                                        w[jj] = fmaf(s4.z, v4.z, w[jj]);
+                                        w[jj] = fmaf(s4.w, v4.w, w[jj]);
+                                    }
+                                }
+                            }
+                        } else {
+                            for (int m = 0; m < r; ++m) {
+                                const float sv = __ldg(Sk + m);
+#pragma unroll
+                                for (int jj = 0; jj < 8; ++jj) {
+                                    const int l = g + G * jj;
+                                    if (l < L) w[jj] = fmaf(sv, vsum[l * RP + m], w[jj]);
+                                }
+                            }
+                        }
+                    }
+                    named_bar_sync(1, kConsumers);
+                    if (k < r) {
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj) {
+                            const int l = g + G * jj;
+                            if (l < L) vsum[l * RP + k] = w[jj];
+                        }
+                    }
+                    if (MODE == kModeShrink) named_bar_sync(1, kConsumers);
+                } else if (hdr.skind == LORA_SIGMA_DIAG) {
+                    // ---- diagonal Sigma_i: v[l][k] <- Sigma_i[k] v[l][k], in place
+                    const float *S = hdr.sigma;
+                    for (int e = tid; e < (L << lgRP); e += kConsumers) {
+                        const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
+                        if (k < r) vsum[l * RP + k] = __ldg(S + k) * vsum[l * RP + k];
+                    }
+                    if (MODE == kModeShrink) named_bar_sync(1, kConsumers);
+                }
+                if (MODE == kModeShrink && (CL == 1 || crank == 0)) {
+                    for (int e = tid; e < (L << lgRP); e += kConsumers) {
+                        const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
+                        if (k < r) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = vsum[l * RP + k];
+                    }
                 }
                 if (tid == 0 && u < 8) LORA_TRACE_MARK(34 + 4 * u);
                 ++u;

@@ -115,6 +115,7 @@ DecodeParams base_params(const lora_table *t)
     p.pj[0].tmA = t->d_tmaps;
     p.pj[0].h = t->h;
     p.pj[0].o = t->o;
+    p.pj[0].sigma_kind = t->sigma_kind;
     p.P = 1;
     p.n = t->n;
     p.R = t->max_rank;
@@ -165,6 +166,7 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
     t->d_tmaps = nullptr;
     t->d_tmaps_pfA = nullptr;
     t->d_tmaps_pfB = nullptr;
+    t->sigma_kind = LORA_SIGMA_NONE;
     if (cudaGetDevice(&t->device) != cudaSuccess) {
         delete t;
         return LORA_ERR_CUDA;
@@ -183,6 +185,7 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
         h_desc[i].B = B[i];
         h_desc[i].rank = ranks[i];
         h_desc[i].scale = scales[i];
+        h_desc[i].sigma = nullptr;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int rc = LORA_OK;
@@ -203,6 +206,38 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
         return rc;
     }
     *out = t;
+    return LORA_OK;
+}
+
+int lora_table_set_sigma(lora_table *t, int32_t kind, const float *const *sigma, void *stream)
+{
+    if (!t || !t->d_desc) return LORA_ERR_INVALID_ARG;
+    if (kind != LORA_SIGMA_NONE && kind != LORA_SIGMA_FULL && kind != LORA_SIGMA_DIAG) return LORA_ERR_INVALID_ARG;
+    if (kind != LORA_SIGMA_NONE) {
+        if (!sigma) return LORA_ERR_INVALID_ARG;
+        for (int i = 0; i < t->n; ++i) {
+            if (!sigma[i]) return LORA_ERR_INVALID_ARG;
+            if (reinterpret_cast<uintptr_t>(sigma[i]) & 3u) return LORA_ERR_UNSUPPORTED;
+        }
+    }
+    std::vector<AdapterDesc> h_desc(t->n);
+    for (int i = 0; i < t->n; ++i) {
+        h_desc[i].A = t->A[i];
+        h_desc[i].B = t->B[i];
+        h_desc[i].rank = t->ranks[i];
+        h_desc[i].scale = t->scales[i];
+        h_desc[i].sigma = kind == LORA_SIGMA_NONE ? nullptr : sigma[i];
+    }
+    int prev = 0;
+    if (cudaGetDevice(&prev) != cudaSuccess || cudaSetDevice(t->device) != cudaSuccess) return LORA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool ok = cudaMemcpyAsync(t->d_desc, h_desc.data(), sizeof(AdapterDesc) * t->n, cudaMemcpyHostToDevice,
+                                    s) == cudaSuccess &&
+                    cudaStreamSynchronize(s) == cudaSuccess;
+    cudaSetDevice(prev);
+    if (!ok) return LORA_ERR_CUDA;
+    t->sigma_kind = kind;
+    t->sigma.assign(kind == LORA_SIGMA_NONE ? nullptr : sigma, kind == LORA_SIGMA_NONE ? nullptr : sigma + t->n);
     return LORA_OK;
 }
 
@@ -380,6 +415,7 @@ int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_seg
         pj.y = y[i];
         pj.ldy = ldy[i];
         pj.y_off = y_off[i];
+        pj.sigma_kind = t->sigma_kind;
         if (t->max_rank > p.R) p.R = t->max_rank;
     }
     return launch_decode(kModeFused, kSrcSegments, p, tables[0]->dtype, static_cast<cudaStream_t>(stream));

@@ -17,11 +17,13 @@ namespace lora {
 
 // One adapter of a table, as the kernels see it.
 struct __align__(32) AdapterDesc {
-    const void *A;   // [rank, h] row-major
-    const void *B;   // [o, rank] row-major
+    const void *A;        // [rank, h] row-major
+    const void *B;        // [o, rank] row-major
     int32_t rank;
     float scale;
+    const float *sigma;   // three-stage form: Sigma_i (rank x rank or rank values, fp32), else null
 };
+static_assert(sizeof(AdapterDesc) == 32, "descriptor size");
 
 // Upper bound of a bounded wait: about two seconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -173,6 +175,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
 __device__ __forceinline__ void prefetch_l2(const void *p)
 {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Hint: bring a 128-byte line into this SM's L1.
+__device__ __forceinline__ void prefetch_l1(const void *p)
+{
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
 // Asynchronous store of 16 bytes into cluster CTA `rank`'s shared memory at the same offset as

@@ -29,7 +29,7 @@ struct ProjParams {
     int64_t ldx, ldy;
     int32_t h, o;          // in/out features
     int32_t y_off;
-    int32_t pad_;
+    int32_t sigma_kind;    // LORA_SIGMA_* of the table
 };
 constexpr int kMaxProj = 4;
 
@@ -82,4 +82,7 @@ struct lora_table {
     void *d_tmaps;
     // prefill path (bf16, ranks multiple of 8 and <= 64): 128-byte-swizzled maps of A_i, B_i
     void *d_tmaps_pfA, *d_tmaps_pfB;
+    // three-stage form: LORA_SIGMA_* and the per-adapter Sigma_i pointers (device, fp32)
+    int32_t sigma_kind;
+    std::vector<const float *> sigma;
 };

@@ -611,7 +611,10 @@ static_assert(kStages * (kTileM * 128 + kMaxRankPF * 128) >= kTileM * (kMaxRankP
 
 }  // namespace
 
-bool prefill_supported(const lora_table *t) { return t && t->d_tmaps_pfA && t->d_tmaps_pfB; }
+bool prefill_supported(const lora_table *t)
+{
+    return t && t->d_tmaps_pfA && t->d_tmaps_pfB && t->sigma_kind == LORA_SIGMA_NONE;
+}
 
 // Tensor maps of every adapter for the prefill path (bf16 tables, ranks multiple of 8, <= 64).
 int prefill_build_maps(lora_table *t)

@@ -103,6 +103,24 @@ int lora_table_create(lora_table **out, int32_t n_adapters, int32_t h_in, int32_
                       int32_t dtype, const void *const *A, const void *const *B,
                       const int32_t *ranks, const float *scales, void *stream);
 
+/* Three-stage (compressed) form, "Compress then Serve" review thread, authors' rebuttal on
+ * Punica, pseudocode of add_lora_slice_with_sigma: between the A step (scale 1) and the B
+ * step (scale s_i) each token's intermediate passes through its adapter's small matrix:
+ *   LORA_SIGMA_FULL: sigma[i] is [ranks[i], ranks[i]] row-major, v'[k] = sum_m sigma[i][k, m] v[m]
+ *   LORA_SIGMA_DIAG: sigma[i] holds ranks[i] values,              v'[k] = sigma[i][k] * v[k]
+ * (the pages' JD-Full and JD-Diag).  sigma is a HOST array of n DEVICE pointers to fp32 values
+ * (4-byte aligned), kept alive by the caller while the table uses them; LORA_SIGMA_NONE
+ * (sigma may be NULL) returns to the plain form.  Adapters of one compression cluster share
+ * A_c and B_c simply by passing the same A / B pointers to lora_table_create.  Every compute
+ * call then applies Sigma in fp32 on chip; lora_shrink writes v' (steps 1 and 2) and
+ * lora_expand takes v' as given.  Tables with Sigma use the decode kernels (no tcgen05 path).
+ * The descriptor update is copied on `stream` and synchronised; do not call it while calls
+ * that use the table are in flight. */
+#define LORA_SIGMA_NONE 0
+#define LORA_SIGMA_FULL 1
+#define LORA_SIGMA_DIAG 2
+int lora_table_set_sigma(lora_table *table, int32_t kind, const float *const *sigma, void *stream);
+
 /* Free the table's device memory (synchronises the device first).  NULL is accepted. */
 int lora_table_destroy(lora_table *table);
 

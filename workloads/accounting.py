@@ -35,21 +35,29 @@ def projection_flops(ids: np.ndarray, ranks: np.ndarray, h: int, o: int) -> int:
     return int(2 * (r * h).sum() + 2 * (r * o).sum())
 
 
-def workload_bytes(wl, shared_x: bool = False) -> int:
+def workload_bytes(wl, shared_x: bool = False, sigma: str = "none", clusters: int = 0) -> int:
     """Algorithmic bytes of one step of a workload (all projections).  With ``shared_x`` the
     projections that read the same activations (q, k and v) count x once, as one grouped
-    launch reads it."""
+    launch reads it.  For the three-stage form, ``sigma`` ("full" / "diag") adds each
+    touched adapter's fp32 Sigma_i (r^2 or r values), and ``clusters`` > 0 shares A and B
+    inside clusters (adapter i uses adapter i mod clusters' weights), so the weights of each
+    touched cluster count once."""
     e = ELEM_BYTES[wl.dtype]
     d = distinct_adapters(wl.ids)
     T_valid = int((np.asarray(wl.ids) >= 0).sum())
+    leaders = np.unique(d % clusters) if clusters > 0 else d
     tot = 0
     seen = set()
     groups = [g for (_n, _h, _o, g) in wl.spec.projections] if shared_x else range(len(wl.projections))
     for p, g in zip(wl.projections, groups):
-        tot += projection_bytes(T_valid, p.h, p.o, (p.ranks[i] for i in d), e)
+        tot += projection_bytes(T_valid, p.h, p.o, (p.ranks[i] for i in leaders), e)
         if g in seen:
             tot -= T_valid * p.h * e
         seen.add(g)
+        if sigma == "full":
+            tot += int(sum(4 * int(p.ranks[i]) ** 2 for i in d))
+        elif sigma == "diag":
+            tot += int(sum(4 * int(p.ranks[i]) for i in d))
     return tot
 
 
