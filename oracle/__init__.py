@@ -71,6 +71,9 @@ def bind(path: str):
     lib.oracle_lora_shrink_sigma.argtypes = [ctypes.c_int, i64, i64, P, i64, P, i32, P, P, ctypes.c_int, P, P,
                                              i64, ctypes.c_int]
     lib.oracle_lora_shrink_sigma.restype = ctypes.c_int
+    lib.oracle_lora_delta_merged.argtypes = [ctypes.c_int, i64, i64, i64, P, i64, P, i64, i64, i32, P, P, i32,
+                                             P, P, P, P, P, ctypes.c_int]
+    lib.oracle_lora_delta_merged.restype = ctypes.c_int
     lib.oracle_build_segments.argtypes = [i64, P, i32, P, P, P, P]
     lib.oracle_build_segments.restype = ctypes.c_int64
     lib.oracle_max_threads.argtypes = []
@@ -246,6 +249,40 @@ def lora_shrink_sigma(dtype: str, x: np.ndarray, ids: np.ndarray, A: Sequence[np
     if rc != 0:
         raise OracleError("adapter id out of range")
     return v
+
+
+def lora_delta_merged(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray, w: np.ndarray,
+                      A: Sequence[np.ndarray], B: Sequence[np.ndarray], scales: Sequence[float],
+                      y_offset: int = 0, o: Optional[int] = None, threads: int = 0) -> np.ndarray:
+    """Several adapters per token: fp64 y_ref = y0 + sum_j w[t, j] s_i B_i (A_i x[t]) over the
+    K slots of ids[t, :] (-1 = empty); ids and w are [T, K]."""
+    x = _check_store(x, dtype)
+    y0 = _check_store(y0, dtype)
+    T, h = x.shape
+    if o is None:
+        o = y0.shape[1] - y_offset
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    if ids.ndim != 2 or ids.shape[0] != T or w.shape != ids.shape:
+        raise ValueError("ids and w must both be [T, K]")
+    K = ids.shape[1]
+    n = len(A)
+    As = [_check_store(a, dtype) for a in A]
+    Bs = [_check_store(b, dtype) for b in B]
+    ranks = np.array([a.shape[0] for a in As], dtype=np.int32)
+    for a, b, r in zip(As, Bs, ranks):
+        if a.shape != (r, h) or b.shape != (o, r):
+            raise ValueError("adapter shapes %s / %s do not match h=%d o=%d" % (a.shape, b.shape, h, o))
+    Ap = (ctypes.c_void_p * max(n, 1))(*[_ptr(a) for a in As])
+    Bp = (ctypes.c_void_p * max(n, 1))(*[_ptr(b) for b in Bs])
+    sc = np.ascontiguousarray(np.asarray(scales, dtype=np.float32).astype(np.float64))
+    out = np.empty((T, o), dtype=np.float64)
+    rc = _load().oracle_lora_delta_merged(_dtype_code(dtype), T, h, o, _ptr(x), x.shape[1], _ptr(y0), y0.shape[1],
+                                          y_offset, K, _ptr(ids), _ptr(w), n, Ap, Bp, _ptr(ranks), _ptr(sc),
+                                          _ptr(out), threads)
+    if rc != 0:
+        raise OracleError("adapter id out of range")
+    return out
 
 
 def build_segments(ids: np.ndarray, n_adapters: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:

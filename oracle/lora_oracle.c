@@ -329,6 +329,67 @@ int oracle_lora_shrink_sigma(int dtype, int64_t T, int64_t h,
 }
 
 /*
+ * Several adapters merged per token ("Lorax" pages: adapters merged per request into an
+ * ensemble with weighted merge strategies).  Reading: the merge is the weighted sum of the
+ * adapters' deltas,
+ *
+ *   y_ref[t, n] = y0[t, y_offset + n] + sum_{j < K, i = ids[t, j] >= 0} w[t, j] * s_i * (B_i (A_i x[t]))[n]
+ *
+ * ids and w are [T, K] row-major (K slots per token, id -1 = empty slot); w is fp32,
+ * widened exactly.  Other arguments as oracle_lora_delta.  Returns -1 for an id outside
+ * [-1, n_adapters).
+ */
+int oracle_lora_delta_merged(int dtype, int64_t T, int64_t h, int64_t o,
+                             const void *x, int64_t ldx,
+                             const void *y0, int64_t ldy, int64_t y_offset,
+                             int32_t K, const int32_t *ids, const float *w, int32_t n_adapters,
+                             const void *const *A, const void *const *B,
+                             const int32_t *ranks, const double *scales,
+                             double *y_ref, int n_threads)
+{
+    if (K < 1 || !ids_valid(T * K, ids, n_adapters))
+        return -1;
+    set_threads(n_threads);
+#pragma omp parallel
+    {
+        double *v = NULL;
+        int32_t cap = 0;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < T; ++t) {
+            double *yr = y_ref + t * o;
+            for (int64_t n = 0; n < o; ++n)
+                yr[n] = widen(y0, dtype, t * ldy + y_offset + n);
+            for (int32_t j = 0; j < K; ++j) {
+                int32_t i = ids[t * K + j];
+                if (i < 0)
+                    continue;
+                int32_t r = ranks[i];
+                if (r > cap) {
+                    free(v);
+                    v = (double *)malloc((size_t)r * sizeof(double));
+                    cap = r;
+                }
+                for (int32_t k = 0; k < r; ++k) {
+                    double acc = 0.0;
+                    for (int64_t jj = 0; jj < h; ++jj)
+                        acc += widen(x, dtype, t * ldx + jj) * widen(A[i], dtype, (int64_t)k * h + jj);
+                    v[k] = acc;
+                }
+                double wt = (double)w[t * K + j];
+                for (int64_t n = 0; n < o; ++n) {
+                    double acc = 0.0;
+                    for (int32_t k = 0; k < r; ++k)
+                        acc += widen(B[i], dtype, n * r + k) * v[k];
+                    yr[n] += wt * (scales[i] * acc);
+                }
+            }
+        }
+        free(v);
+    }
+    return 0;
+}
+
+/*
  * Segment bookkeeping: a stable counting sort of the tokens by adapter id.
  *   perm[p]          token index at sorted position p (p < number of tokens with an adapter)
  *   seg_ptr[s]       first sorted position of segment s; seg_ptr[num_segs] = valid tokens

@@ -18,7 +18,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "lora_oracle.c")
 MUTATIONS = {
     "transposed_A": ("acc += xrow[j] * widen(A[i], dtype, (int64_t)k * h + j)",
                      "acc += xrow[j] * widen(A[i], dtype, (int64_t)j * r + k)"),
-    "transposed_B": ("widen(B[i], dtype, n * r + k) * v[k]", "widen(B[i], dtype, (int64_t)k * o + n) * v[k]"),
+    "transposed_B": ("widen(B[i], dtype, n * r + k) * v[k];\n                yr[n] += scales[i] * acc;",
+                     "widen(B[i], dtype, (int64_t)k * o + n) * v[k];\n                yr[n] += scales[i] * acc;"),
     "dropped_y0": ("yr[n] = widen(y0, dtype, t * ldy + y_offset + n);\n            int32_t i = ids[t];\n"
                    "            if (i < 0)\n                continue;\n            int32_t r = ranks[i];\n"
                    "            if (r > vcap)",
@@ -43,6 +44,10 @@ MUTATIONS = {
                        "widen(y0, dtype, t * ldy + n);\n            int32_t i = ids[t];\n"
                        "            if (i < 0)\n                continue;\n            int32_t r = ranks[i];\n"
                        "            if (r > vcap)"),
+    "merge_weight_dropped": ("yr[n] += wt * (scales[i] * acc);", "yr[n] += scales[i] * acc;"),
+    "merge_first_slot_only": ("for (int32_t j = 0; j < K; ++j) {\n                int32_t i = ids[t * K + j];",
+                              "for (int32_t j = 0; j < 1; ++j) {\n                int32_t i = ids[t * K + j];"),
+    "merge_wrong_weight": ("double wt = (double)w[t * K + j];", "double wt = (double)w[t * K];"),
     "sigma_transposed": ("acc += (double)S[(int64_t)k * r + m] * u[m];", "acc += (double)S[(int64_t)m * r + k] * u[m];"),
     "sigma_full_skipped": ("            w[k] = acc;\n        } else if", "            w[k] = u[k];\n        } else if"),
     "sigma_diag_skipped": ("w[k] = (double)S[k] * u[k];", "w[k] = u[k];"),
@@ -66,6 +71,9 @@ PIN_TESTS = [
     pins.test_sigma_diagonal_of_powers_of_two_folds_into_B,
     lambda: [pins.test_sigma_equals_merged_three_factor_weight(k) for k in ("full", "diag")],
     pins.test_sigma_shrink_is_sigma_times_shrink,
+    pins.test_merged_single_slot_unit_weight_is_the_plain_delta,
+    pins.test_merged_equals_merged_weight_closed_form,
+    pins.test_merged_slot_order_and_duplicate_slots,
 ]
 
 

@@ -441,3 +441,77 @@ def test_sigma_shared_cluster_weights():
         rows = wl.ids == i
         want[rows] += x[rows] @ W.T
     assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max()
+
+
+# ------------------------------------------------------------------ merged adapters per token
+# "Lorax" pages: adapters merged per request into a weighted ensemble.  Reading: the merge is
+# the weighted sum of the adapters' deltas, y = y0 + sum_j w_j s_j B_j A_j x.
+
+def _merge_case(K=3, empty=0.25, seed=1):
+    wl = workloads.generate("multirank_decode", T=36, n=9, shapes=[("q", 160, 96, 0)], ranks=(4, 8, 16))
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    ids, w = workloads.draw_merge(wl.ids, wl.n, K, seed, empty=empty)
+    return wl, p, A, B, ids, w
+
+
+def test_merged_single_slot_unit_weight_is_the_plain_delta():
+    wl, p, A, B, _ids, _w = _merge_case()
+    ids = wl.ids.reshape(-1, 1).astype(np.int32)
+    w = np.ones_like(ids, dtype=np.float32)
+    plain = oracle.lora_delta(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales)
+    merged = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids, w, A, B, p.scales)
+    assert np.array_equal(plain, merged)
+
+
+def test_merged_zero_weights_leave_y_unchanged():
+    wl, p, A, B, ids, w = _merge_case()
+    got = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids, np.zeros_like(w), A, B, p.scales)
+    assert np.array_equal(got, to_float64(p.y0, wl.dtype))
+
+
+def test_merged_equals_merged_weight_closed_form():
+    """Per token, y0 + x (sum_j w_j s_j B_j A_j)^T with the o x h ensemble weight formed first
+    in fp64: pins the per-slot adapter, weight and scale."""
+    wl, p, A, B, ids, w = _merge_case()
+    got = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids, w, A, B, p.scales)
+    x = to_float64(p.x, wl.dtype)
+    want = to_float64(p.y0, wl.dtype).copy()
+    Wd = [float(p.scales[i]) * (to_float64(B[i], wl.dtype) @ to_float64(A[i], wl.dtype)) for i in range(wl.n)]
+    for t in range(wl.T):
+        W = np.zeros_like(Wd[0])
+        for j in range(ids.shape[1]):
+            if ids[t, j] >= 0:
+                W += float(w[t, j]) * Wd[ids[t, j]]
+        want[t] += W @ x[t]
+    assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max()
+
+
+def test_merged_slot_order_and_duplicate_slots():
+    """Permuting a token's slots, or splitting one slot's weight over two slots of the same
+    adapter, changes nothing beyond fp64 rounding."""
+    wl, p, A, B, ids, w = _merge_case(K=2, empty=0.0)
+    base = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids, w, A, B, p.scales)
+    swapped = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids[:, ::-1].copy(), w[:, ::-1].copy(), A, B, p.scales)
+    scale = np.abs(base).max()
+    assert np.abs(base - swapped).max() <= 1e-13 * scale
+    ids3 = np.concatenate([ids, ids[:, :1]], axis=1)
+    w3 = np.concatenate([w, np.zeros_like(w[:, :1])], axis=1)
+    w3[:, 2] = np.float32(0.5) * w3[:, 0]
+    w3[:, 0] = w3[:, 0] - w3[:, 2]   # exact in fp32: halving, then subtracting the half
+    split = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids3, w3, A, B, p.scales)
+    assert np.abs(base - split).max() <= 1e-13 * scale
+
+
+def test_merged_empty_slots_and_bad_ids():
+    wl, p, A, B, ids, w = _merge_case()
+    only0 = ids.copy()
+    only0[:, 1:] = -1
+    got = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, only0, w, A, B, p.scales)
+    w0 = np.where(only0 >= 0, w, 0).astype(np.float32)
+    again = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, only0, w0, A, B, p.scales)
+    assert np.array_equal(got, again)
+    bad = ids.copy()
+    bad[3, 1] = wl.n
+    with pytest.raises(oracle.OracleError):
+        oracle.lora_delta_merged(wl.dtype, p.x, p.y0, bad, w, A, B, p.scales)

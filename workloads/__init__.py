@@ -285,3 +285,24 @@ def jd_clusters(n: int, clusters: int) -> np.ndarray:
     to cluster i mod clusters, and every member uses its cluster leader's (adapter c's)
     A and B."""
     return (np.arange(n) % max(1, clusters)).astype(np.int32)
+
+
+def draw_merge(ids: np.ndarray, n: int, K: int, seed: int, empty: float = 0.0):
+    """Per-token adapter ensembles for the merged form: slot 0 keeps the batch's ids, slots
+    1..K-1 draw adapters uniformly from [0, n) (a fraction ``empty`` of them left empty, -1),
+    and each token's weights are uniform on (0, 1] normalised to sum to 1 over its filled
+    slots.  Returns (ids [T, K] int32, w [T, K] fp32)."""
+    rng = np.random.default_rng(seed)
+    T = len(ids)
+    out = np.empty((T, K), dtype=np.int32)
+    out[:, 0] = ids
+    if K > 1:
+        out[:, 1:] = rng.integers(0, n, size=(T, K - 1))
+        if empty > 0:
+            drop = rng.random((T, K - 1)) < empty
+            out[:, 1:][drop] = -1
+    w = rng.uniform(1e-3, 1.0, size=(T, K))
+    w[out < 0] = 0.0
+    tot = w.sum(axis=1, keepdims=True)
+    w = np.where(tot > 0, w / np.where(tot > 0, tot, 1.0), 0.0)
+    return out, w.astype(np.float32)
