@@ -65,6 +65,8 @@ def parse():
                     help="three-stage (compressed) form: a per-adapter Sigma_i between the A and B steps")
     ap.add_argument("--jd-clusters", type=int, default=0,
                     help="with --sigma: adapters share the A and B of adapter (i mod K), as compressed clusters do")
+    ap.add_argument("--merge", type=int, default=1,
+                    help="decode_bgmv: K adapters merged per token (weighted ensembles, lora_bgmv_merged)")
     ap.add_argument("--grouped", action="store_true",
                     help="many_adapter_qkvo: one lora_sgmv_grouped launch for q, k, v, o (q, k, v reading one x) "
                          "instead of four lora_sgmv calls")
@@ -149,7 +151,7 @@ class ClockSampler:
 class Copy:
     """One replica of the workload's inputs on the device plus its adapter tables."""
 
-    def __init__(self, wl, L, torch, sigma="none", clusters=0):
+    def __init__(self, wl, L, torch, sigma="none", clusters=0, merge=1):
         from workloads.device import upload_projection
         self.projs = []
         self.tables = []
@@ -170,6 +172,10 @@ class Copy:
             self.projs.append(d)
             self.tables.append(t)
         self.ids = torch.from_numpy(wl.ids).cuda()
+        if merge > 1:
+            m_ids, m_w = workloads.draw_merge(wl.ids, wl.n, merge, seed=wl.seed + 99)
+            self.m_ids = torch.from_numpy(m_ids).cuda()
+            self.m_w = torch.from_numpy(m_w).cuda()
         n, T = wl.n, wl.T
         self.seg_t = dict(perm=torch.empty(T, dtype=torch.int32, device="cuda"),
                           seg_ptr=torch.empty(n + 1, dtype=torch.int32, device="cuda"),
@@ -195,10 +201,18 @@ class Copy:
         return tot
 
 
-def make_step(wl, L, grouped=False):
+def make_step(wl, L, grouped=False, merge=1):
     """Returns (step(copy, stream_handle), launches per step, name of the dominant kernel)."""
     name = wl.name
     T = wl.T
+    if merge > 1:
+        if name != "decode_bgmv":
+            raise SystemExit("--merge applies to decode_bgmv only")
+
+        def step(c, s):
+            d, t = c.projs[0], c.tables[0]
+            L.lora_bgmv_merged(t.handle, c.m_ids, c.m_w, T, merge, d.x, d.h, d.y0, d.o, 0, c.ws, c.ws.numel(), s)
+        return step, merge, "lora_decode_kernel (fused, per-token ids, one pass per merged slot)"
     if grouped:
         if name != "many_adapter_qkvo":
             raise SystemExit("--grouped applies to many_adapter_qkvo only")
@@ -247,17 +261,20 @@ def run_ours(args, rank, world, local_rank):
     seed = workloads.SEED_BASE + workloads.WORKLOAD_NAMES.index(args.workload) + 1000 * rank
     wl = workloads.generate(args.workload, seed=seed)
     T = wl.T
-    step, launches_per_step, kname = make_step(wl, L, args.grouped)
+    step, launches_per_step, kname = make_step(wl, L, args.grouped, args.merge)
     if args.jd_clusters and args.sigma == "none":
         raise SystemExit("--jd-clusters needs --sigma")
     bytes_step = accounting.workload_bytes(wl, shared_x=args.grouped, sigma=args.sigma, clusters=args.jd_clusters)
+    if args.merge > 1:   # x and y once, every adapter any slot touches once
+        m_ids, _m_w = workloads.draw_merge(wl.ids, wl.n, args.merge, seed=wl.seed + 99)
+        bytes_step = accounting.merged_bytes(wl, m_ids)
     flops_step = accounting.workload_flops(wl)
     distinct = int(accounting.distinct_adapters(wl.ids).size)
 
-    first = Copy(wl, L, torch, args.sigma, args.jd_clusters)
+    first = Copy(wl, L, torch, args.sigma, args.jd_clusters, args.merge)
     ws_bytes = first.nbytes()
     C = args.copies or max(1, min(256, -(-4 * L2_BYTES // ws_bytes)))
-    copies = [first] + [Copy(wl, L, torch, args.sigma, args.jd_clusters) for _ in range(C - 1)]
+    copies = [first] + [Copy(wl, L, torch, args.sigma, args.jd_clusters, args.merge) for _ in range(C - 1)]
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
@@ -418,7 +435,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "rotating %d input copies, %.0f MB in total against a 126 MB L2%s" % (
                        C, C * ws_bytes / 1e6, "" if C * ws_bytes >= 4 * L2_BYTES else " (copy count capped)"),
                    "graph": not args.no_graph, "pdl": bool(L.lora_get_option("pdl")),
-                   "sigma": args.sigma, "jd_clusters": args.jd_clusters,
+                   "sigma": args.sigma, "jd_clusters": args.jd_clusters, "merge_slots": args.merge,
                    "parallelism": "replicas x%d (independent token batches, no collective)" % world},
         "roofline": roofline,
         "cpu_baseline": cpu,

@@ -36,12 +36,13 @@ LORA_MAX_GROUP = 4
 LORA_SIGMA_NONE = 0
 LORA_SIGMA_FULL = 1
 LORA_SIGMA_DIAG = 2
+LORA_MAX_MERGE = 8
 
 EXPORTS = (
     "lora_table_create", "lora_table_destroy", "lora_table_info", "lora_workspace_bytes",
     "lora_build_segments", "lora_shrink", "lora_expand", "lora_sgmv", "lora_bgmv",
     "lora_get_status", "lora_status_string", "lora_set_option", "lora_get_option",
-    "lora_sgmv_noalloc", "lora_sgmv_grouped", "lora_table_set_sigma",
+    "lora_sgmv_noalloc", "lora_sgmv_grouped", "lora_table_set_sigma", "lora_bgmv_merged",
 )
 
 
@@ -88,6 +89,7 @@ def _load():
         "lora_expand": ([P, ctypes.POINTER(lora_segments), P, I32, P, I64, I32, P], ctypes.c_int),
         "lora_sgmv": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
         "lora_bgmv": ([P, P, I32, P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
+        "lora_bgmv_merged": ([P, P, P, I32, I32, P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
         "lora_sgmv_noalloc": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, I32, P], ctypes.c_int),
         "lora_sgmv_grouped": ([P, I32, ctypes.POINTER(lora_segments), P, P, P, P, P, P, SZ, P], ctypes.c_int),
         "lora_get_status": ([P, ctypes.POINTER(ctypes.c_uint32), I32, P], ctypes.c_int),
@@ -199,6 +201,14 @@ def lora_sgmv_grouped(tables, seg: lora_segments, xs, ldxs, ys, ldys, y_offsets,
     off_arr = (ctypes.c_int32 * P)(*y_offsets)
     _check(_load().lora_sgmv_grouped(t_arr, P, ctypes.byref(seg), x_arr, ldx_arr, y_arr, ldy_arr, off_arr,
                                      _ptr(ws), ws_bytes, _stream(stream)), "lora_sgmv_grouped")
+
+
+def lora_bgmv_merged(table: int, ids, w, T: int, K: int, x, ldx: int, y, ldy: int, y_offset: int, ws=None,
+                     ws_bytes: int = 0, stream=None) -> None:
+    """Several adapters per token: ids and w are [T, K] device tensors (int32 / fp32, -1 =
+    empty slot); y[t] += sum_j w[t, j] s_i B_i A_i x[t]."""
+    _check(_load().lora_bgmv_merged(table, _ptr(ids), _ptr(w), T, K, _ptr(x), ldx, _ptr(y), ldy, y_offset, _ptr(ws),
+                                    ws_bytes, _stream(stream)), "lora_bgmv_merged")
 
 
 def lora_sgmv_noalloc(table: int, seg: lora_segments, x, ldx: int, y, ldy: int, y_offset: int, stream=None) -> None:

@@ -53,7 +53,7 @@ constexpr int kRowBytes = 1024;             // h-subtile row (shrink) / o-subtil
                                             // 512 for ranks above 64 (smaller stages)
 constexpr int kBoxBytes = 512;              // one TMA box row of A
 constexpr int kMaxStages = 4;
-constexpr int kHeaderBytes = 128;
+constexpr int kHeaderBytes = 256;
 
 enum : int32_t { kTileShrink = 1, kTileExpand = 2, kTileEnd = 3 };
 enum : int32_t { kFlagFirst = 1, kFlagLast = 2 };
@@ -66,6 +66,7 @@ struct __align__(16) StageHeader {
     int32_t skind;         // LORA_SIGMA_*: the unit's Sigma_i (three-stage form)
     const float *sigma;
     int32_t tok[kTokChunk];
+    float tw[kTokChunk];   // per-token weight of a merged ensemble slot (1 otherwise)
 };
 static_assert(sizeof(StageHeader) <= kHeaderBytes, "header");
 
@@ -103,7 +104,7 @@ __host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int 
     const int rowb = row_bytes_for(R);
     l.RP = round_up(R, 8);
     l.ids_off = kCtlBytes;
-    const int ids_bytes = (src == kSrcIds) ? round_up(4 * (2 * T + n), 128) : 0;
+    const int ids_bytes = (src == kSrcIds) ? round_up(4 * (3 * T + n), 128) : 0;   // ids, first, leaders, weights
     l.xs_off = l.ids_off + ids_bytes;
     l.ys_off = l.xs_off + kTokChunk * rowb;
     l.vpart_off = l.ys_off + kTokChunk * rowb;
@@ -232,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     int32_t *ids_s = reinterpret_cast<int32_t *>(smem + lay.ids_off);
     int32_t *first = ids_s + p.T;
     int32_t *leaders = first + p.n;
+    float *w_s = reinterpret_cast<float *>(leaders + p.T);   // per-token merge weights (ids form)
     const bool direct_ids = (SRC == kSrcIds) && p.n <= G;
     // The adapter table is immutable after creation: in direct mode this cluster's descriptor
     // and tensor map are fetched before waiting for the previous grid.
@@ -259,10 +261,24 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     pdl_launch_dependents();
     if (SRC == kSrcIds && !direct_ids) {
         bool bad = false;
-        for (int t = tid; t < p.T; t += kThreads) {
-            const int32_t a = p.ids[t];
-            ids_s[t] = a;
-            bad |= (a < -1 || a >= p.n);
+        for (int t0 = tid; t0 < p.T; t0 += 4 * kThreads) {
+            int32_t v[4];
+            float wv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int t = t0 + kThreads * q;
+                v[q] = t < p.T ? p.ids[(int64_t)t * p.ids_stride] : -1;
+                wv[q] = (t < p.T && p.tok_w) ? p.tok_w[(int64_t)t * p.w_stride] : 1.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int t = t0 + kThreads * q;
+                if (t < p.T) {
+                    ids_s[t] = v[q];
+                    w_s[t] = wv[q];
+                    bad |= (v[q] < -1 || v[q] >= p.n);
+                }
+            }
         }
         for (int i = tid; i < p.n; i += kThreads) first[i] = INT_MAX;
         if (__syncthreads_or(bad) && tid == 0 && crank == 0 && cid == 0) atomicOr(p.status, LORA_STATUS_BAD_ID);
@@ -293,11 +309,26 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         bool alive = true;
         if (direct_ids) {
             // stage the ids for this warp's scan; cluster 0 CTA 0 reports bad ids
+            // (loads issued four at a time per lane: the ids are on every unit's critical path)
             bool bad = false;
-            for (int t = lane; t < p.T; t += 32) {
-                const int32_t v = p.ids[t];
-                ids_s[t] = v;
-                bad |= (v < -1 || v >= p.n);
+            for (int t0 = lane; t0 < p.T; t0 += 4 * 32) {
+                int32_t v[4];
+                float wv[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int t = t0 + 32 * q;
+                    v[q] = t < p.T ? p.ids[(int64_t)t * p.ids_stride] : -1;
+                    wv[q] = (t < p.T && p.tok_w) ? p.tok_w[(int64_t)t * p.w_stride] : 1.f;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int t = t0 + 32 * q;
+                    if (t < p.T) {
+                        ids_s[t] = v[q];
+                        w_s[t] = wv[q];
+                        bad |= (v[q] < -1 || v[q] >= p.n);
+                    }
+                }
             }
             if (__any_sync(0xffffffffu, bad) && lane == 0 && crank == 0 && cid == 0)
                 atomicOr(p.status, LORA_STATUS_BAD_ID);
@@ -436,7 +467,12 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     const bool shrink = j < g.n_shrink;
                     int off, len, nbox;
                     tile_geom(g, j, r, off, len, nbox);
-                    if (lane < L) hdr->tok[lane] = my_tok;
+                    if (lane < L) {
+                        hdr->tok[lane] = my_tok;
+                        hdr->tw[lane] = SRC == kSrcIds ? w_s[my_tok]
+                                        : !p.tok_w ? 1.f
+                                                   : p.tok_w[(int64_t)my_tok * p.w_stride];
+                    }
                     if (lane == 0) {
                         hdr->kind = shrink ? kTileShrink : kTileExpand;
                         const int first_j = shrink ? 0 : g.n_shrink;
@@ -781,16 +817,17 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     for (int q = 0; q < 2; ++q) {
                         if (q == 1 && !l2) break;
                         const float *acc = q == 0 ? acc0 : acc1;
+                        const float sl = sc * hdr.tw[l + q];   // exact when the weight is 1
                         const uint8_t *yr = ys + (l + q) * rowb + c * ESZ;
                         const int64_t gofs = (int64_t)hdr.tok[l + q] * pj.ldy + pj.y_off + off + c;
                         if constexpr (CPT == 2) {
                             const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
-                            const float y0 = fmaf(sc, acc[0], bf16_lo(w));
-                            const float y1 = fmaf(sc, acc[1], bf16_hi(w));
+                            const float y0 = fmaf(sl, acc[0], bf16_lo(w));
+                            const float y1 = fmaf(sl, acc[1], bf16_hi(w));
                             *reinterpret_cast<uint32_t *>(static_cast<E *>(pj.y) + gofs) = pack_bf16x2(y0, y1);
                         } else {
                             const float w = *reinterpret_cast<const float *>(yr);
-                            static_cast<float *>(pj.y)[gofs] = fmaf(sc, acc[0], w);
+                            static_cast<float *>(pj.y)[gofs] = fmaf(sl, acc[0], w);
                         }
                     }
                 }

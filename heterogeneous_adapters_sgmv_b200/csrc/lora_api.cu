@@ -117,6 +117,8 @@ DecodeParams base_params(const lora_table *t)
     p.pj[0].o = t->o;
     p.pj[0].sigma_kind = t->sigma_kind;
     p.P = 1;
+    p.ids_stride = 1;
+    p.w_stride = 1;
     p.n = t->n;
     p.R = t->max_rank;
     p.status = t->d_status;
@@ -461,6 +463,66 @@ int lora_bgmv(const lora_table *t, const int32_t *d_ids, int32_t T, const void *
                                   stream)))
         return rc;
     return lora_sgmv(t, &seg, x, ldx, y, ldy, y_off, ws, ws_bytes, stream);
+}
+
+int lora_bgmv_merged(const lora_table *t, const int32_t *d_ids, const float *d_w, int32_t T, int32_t K,
+                     const void *x, int64_t ldx, void *y, int64_t ldy, int32_t y_off, void *ws, size_t ws_bytes,
+                     void *stream)
+{
+    int rc = check_table(t);
+    if (rc) return rc;
+    if (T < 0 || K < 1 || K > LORA_MAX_MERGE) return LORA_ERR_INVALID_ARG;
+    if ((rc = check_io(t, x, ldx, y, ldy, y_off, true, true))) return rc;
+    if (T == 0) return LORA_OK;
+    if (!d_ids || !d_w) return LORA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool direct = T <= kBgmvMaxT && t->n <= kBgmvMaxN;
+    if (!direct && T > LORA_MAX_SEGMENT_TOKENS) return LORA_ERR_UNSUPPORTED;
+    const WsLayout w = ws_layout(t, T);
+    if (!direct && (!ws || ws_bytes < w.total)) return LORA_ERR_WORKSPACE;
+    if (!direct && !al16(ws)) return LORA_ERR_UNSUPPORTED;
+    // One pass per slot, in slot order: each pass is the BGMV update of that slot's adapters
+    // with the per-token weight folded into the scale; y is rounded after each pass.
+    for (int k = 0; k < K; ++k) {
+        DecodeParams p = base_params(t);
+        p.pj[0].x = x;
+        p.pj[0].ldx = ldx;
+        p.pj[0].y = y;
+        p.pj[0].ldy = ldy;
+        p.pj[0].y_off = y_off;
+        p.tok_w = d_w + k;
+        p.w_stride = K;
+        if (direct) {
+            p.ids = d_ids + k;
+            p.ids_stride = K;
+            p.T = T;
+            rc = launch_decode(kModeFused, kSrcIds, p, t->dtype, s);
+        } else {
+            // slot k's ids into the workspace (the intermediate area, unused by the fused
+            // kernel), then the segment bookkeeping and the segmented kernel
+            uint8_t *b = static_cast<uint8_t *>(ws);
+            int32_t *col = reinterpret_cast<int32_t *>(b + w.v);
+            if (cudaMemcpy2DAsync(col, sizeof(int32_t), d_ids + k, sizeof(int32_t) * K, sizeof(int32_t), T,
+                                  cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+                return LORA_ERR_CUDA;
+            lora_segments seg;
+            std::memset(&seg, 0, sizeof seg);
+            seg.perm = reinterpret_cast<int32_t *>(b + w.perm);
+            seg.seg_ptr = reinterpret_cast<int32_t *>(b + w.seg_ptr);
+            seg.seg_adapter = reinterpret_cast<int32_t *>(b + w.seg_adapter);
+            seg.num_segs = reinterpret_cast<int32_t *>(b + w.num_segs);
+            seg.T = T;
+            seg.max_segs = t->n;
+            if ((rc = lora_build_segments(t, col, T, const_cast<int32_t *>(seg.perm),
+                                          const_cast<int32_t *>(seg.seg_ptr), const_cast<int32_t *>(seg.seg_adapter),
+                                          const_cast<int32_t *>(seg.num_segs), stream)))
+                return rc;
+            set_segments(p, &seg);
+            rc = launch_decode(kModeFused, kSrcSegments, p, t->dtype, s);
+        }
+        if (rc) return rc;
+    }
+    return LORA_OK;
 }
 
 int lora_get_status(const lora_table *t, uint32_t *h_status, int32_t reset, void *stream)

@@ -42,6 +42,9 @@ struct DecodeParams {
     const int32_t *perm, *seg_ptr, *seg_adapter, *num_segs;
     int32_t max_segs;
     const int32_t *ids;
+    int32_t ids_stride;    // element stride of ids (slot k of a [T, K] ensemble: ids + k, stride K)
+    const float *tok_w;    // per-token weights (merged ensembles), or null for weight 1
+    int32_t w_stride;
     int32_t T;
     uint32_t *status;
     int32_t stages;        // pipeline depth

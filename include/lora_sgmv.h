@@ -190,6 +190,19 @@ int lora_bgmv(const lora_table *table, const int32_t *d_ids, int32_t T, const vo
               int64_t ldx, void *y, int64_t ldy, int32_t y_offset, void *ws, size_t ws_bytes,
               void *stream);
 
+/* Several adapters merged per token (the Lorax pages' per-request weighted ensembles):
+ *   y[t, y_offset + n] += sum_{j < K, ids[t, j] >= 0} w[t, j] * s_i * (B_i (A_i x[t]))[n]
+ * d_ids and d_w are [T, K] row-major DEVICE arrays (int32 ids, -1 = empty slot; fp32
+ * weights), 1 <= K <= LORA_MAX_MERGE.  Runs one BGMV pass per slot, in slot order, with the
+ * weight folded into the scale, so y is rounded to its type after each slot (K roundings
+ * instead of one).  Batches above 1024 tokens or 4096 adapters sort each slot into the
+ * workspace (ws_bytes >= lora_workspace_bytes(table, T)); otherwise ws may be NULL.  The
+ * "split" option does not apply. */
+#define LORA_MAX_MERGE 8
+int lora_bgmv_merged(const lora_table *table, const int32_t *d_ids, const float *d_w, int32_t T,
+                     int32_t K, const void *x, int64_t ldx, void *y, int64_t ldy, int32_t y_offset,
+                     void *ws, size_t ws_bytes, void *stream);
+
 /* Read (and with reset != 0, clear) the table's device status word into *h_status.
  * Synchronises `stream`.  Returns LORA_OK when the word is 0, LORA_ERR_TIMEOUT when the
  * timeout bit is set, otherwise LORA_ERR_DEVICE_STATUS. */

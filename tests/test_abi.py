@@ -63,7 +63,8 @@ def test_header_constants_match_binding():
     for name in ("LORA_F32", "LORA_BF16", "LORA_OK", "LORA_ERR_INVALID_ARG", "LORA_ERR_UNSUPPORTED",
                  "LORA_ERR_WORKSPACE", "LORA_ERR_CUDA", "LORA_ERR_TIMEOUT", "LORA_ERR_DEVICE_STATUS",
                  "LORA_STATUS_BAD_ID", "LORA_STATUS_TIMEOUT", "LORA_STATUS_BAD_SEGMENT", "LORA_MAX_RANK",
-                 "LORA_MAX_SEGMENT_TOKENS", "LORA_NOALLOC_SCRATCH_FLOATS", "LORA_MAX_GROUP"):
+                 "LORA_MAX_SEGMENT_TOKENS", "LORA_NOALLOC_SCRATCH_FLOATS", "LORA_MAX_GROUP",
+                 "LORA_SIGMA_NONE", "LORA_SIGMA_FULL", "LORA_SIGMA_DIAG", "LORA_MAX_MERGE"):
         m = re.search(r"#define %s \(?(-?\d+)u?\)?" % name, txt)
         assert m, name
         assert int(m.group(1)) == getattr(L, name), name

@@ -61,6 +61,17 @@ def workload_bytes(wl, shared_x: bool = False, sigma: str = "none", clusters: in
     return tot
 
 
+def merged_bytes(wl, ids2d: np.ndarray) -> int:
+    """Algorithmic bytes of one call of the merged form on projection 0: x read and y read and
+    written once, and every adapter any slot touches once."""
+    e = ELEM_BYTES[wl.dtype]
+    p = wl.projections[0]
+    ids2d = np.asarray(ids2d)
+    d = distinct_adapters(ids2d.ravel())
+    T_valid = int((ids2d >= 0).any(axis=1).sum())
+    return projection_bytes(T_valid, p.h, p.o, (p.ranks[i] for i in d), e)
+
+
 def workload_flops(wl) -> int:
     return sum(projection_flops(wl.ids, p.ranks, p.h, p.o) for p in wl.projections)
 
