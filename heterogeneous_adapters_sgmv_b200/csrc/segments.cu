@@ -2,12 +2,17 @@
 // the grouping of same-adapter requests that SGMV multiplies segment by segment ("Compress
 // then Serve" review thread, authors' rebuttal on Punica).
 //
-// One CTA of 1024 threads sorts up to LORA_MAX_SEGMENT_TOKENS keys in shared memory with a
-// least-significant-digit radix sort (8-bit digits, as many passes as the adapter count
-// needs).  Every pass is stable: each warp owns a contiguous run of the input, counts its
-// digits into a private histogram row, the rows are scanned digit-major / warp-minor, and
-// each warp scatters its run in order.  No atomics decide positions, so the output is the
-// unique stable order and is bit-identical run to run.
+// Two single-CTA (1024-thread) kernels, both giving the unique stable order, bit-identical
+// run to run:
+//  * counting sort, for decode-sized batches (T <= 2048, n < 8192): one histogram of the
+//    adapter ids in shared memory (warp-aggregated atomics: counts only, not positions), one
+//    exclusive scan giving each adapter's first position and one giving segment indices,
+//    then one warp walks the tokens in batch order and places them (ties inside a warp
+//    broken by lane order), so positions never depend on timing;
+//  * least-significant-digit radix sort for the rest (8-bit digits, as many passes as the
+//    adapter count needs).  Every pass is stable: each warp owns a contiguous run of the
+//    input, counts its digits into a private histogram row, the rows are scanned digit-major
+//    / warp-minor, and each warp scatters its run in order.
 #include <climits>
 
 #include "lora_common.cuh"
@@ -158,17 +163,96 @@ build_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int
     }
 }
 
+// Counting sort (see above).  Shared memory: cnt[n + 1], flag[n], key[T].
+__global__ void __launch_bounds__(kSegThreads, 1)
+count_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int32_t *__restrict__ perm,
+                      int32_t *__restrict__ seg_ptr, int32_t *__restrict__ seg_adapter,
+                      int32_t *__restrict__ num_segs, uint32_t *__restrict__ status)
+{
+    pdl_wait();
+    pdl_launch_dependents();
+
+    extern __shared__ __align__(16) int32_t sm[];
+    int32_t *cnt = sm, *flag = sm + (n + 1), *key_s = flag + n;
+    __shared__ int32_t warp_sums[kSegWarps];
+    __shared__ int32_t total, segs;
+    __shared__ uint32_t bad;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) bad = 0;
+    for (int i = tid; i <= n; i += kSegThreads) cnt[i] = 0;
+    __syncthreads();
+    // keys (out-of-range ids and -1 get the sentinel n) and their histogram
+    for (int t0 = 0; t0 < T; t0 += kSegThreads) {
+        const int t = t0 + tid;
+        const bool ok = t < T;
+        int32_t key = n;
+        if (ok) {
+            const int32_t id = ids[t];
+            if (id >= 0 && id < n)
+                key = id;
+            else if (id != -1)
+                bad = 1;
+            key_s[t] = key;
+        }
+        const uint32_t peers = __match_any_sync(0xffffffffu, ok ? key : -1);
+        if (ok && lane == __ffs(peers) - 1) atomicAdd(&cnt[key], __popc(peers));
+    }
+    __syncthreads();
+    if (tid == 0 && bad) atomicOr(status, LORA_STATUS_BAD_ID);
+    for (int i = tid; i < n; i += kSegThreads) flag[i] = cnt[i] > 0 ? 1 : 0;
+    __syncthreads();
+    block_exclusive_scan(cnt, n + 1, warp_sums, &total);   // cnt[i]: first position of adapter i
+    block_exclusive_scan(flag, n, warp_sums, &segs);       // flag[i]: segment index of adapter i
+    const int32_t valid = cnt[n];
+    for (int i = tid; i < n; i += kSegThreads) {
+        if (cnt[i + 1] > cnt[i]) {
+            seg_ptr[flag[i]] = cnt[i];
+            seg_adapter[flag[i]] = i;
+        }
+    }
+    if (tid == 0) {
+        seg_ptr[segs] = valid;
+        *num_segs = segs;
+    }
+    __syncthreads();   // every thread has read cnt[] before warp 0 advances it
+    if (warp == 0) {
+        for (int t0 = 0; t0 < T; t0 += 32) {
+            const int t = t0 + lane;
+            const bool ok = t < T;
+            const int32_t key = ok ? key_s[t] : -1;
+            const uint32_t peers = __match_any_sync(0xffffffffu, key);
+            const int leader = __ffs(peers) - 1;
+            int32_t base = 0;
+            if (ok && lane == leader && key < n) {
+                base = cnt[key];
+                cnt[key] = base + __popc(peers);
+            }
+            base = __shfl_sync(0xffffffffu, base, leader);
+            if (ok && key < n) perm[base + __popc(peers & ((1u << lane) - 1u))] = t;
+            __syncwarp();
+        }
+    }
+}
+
+constexpr int kCountMaxT = 2048;
+constexpr int kCountMaxN = 8191;
+
 }  // namespace
 
 int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *perm, int32_t *seg_ptr,
                           int32_t *seg_adapter, int32_t *num_segs, uint32_t *status, cudaStream_t s)
 {
-    const size_t smem = (size_t)(4 * T + kHistEntries) * sizeof(int32_t);
+    const bool counting = T <= kCountMaxT && n <= kCountMaxN;
+    const size_t smem = counting ? (size_t)(2 * n + 1 + T) * sizeof(int32_t)
+                                 : (size_t)(4 * T + kHistEntries) * sizeof(int32_t);
     static bool attr_set = false;
     if (!attr_set) {
         const int max_smem = (4 * LORA_MAX_SEGMENT_TOKENS + kHistEntries) * (int)sizeof(int32_t);
+        const int max_count = (2 * kCountMaxN + 1 + kCountMaxT) * (int)sizeof(int32_t);
         if (cudaFuncSetAttribute(build_segments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 max_smem) != cudaSuccess)
+                                 max_smem) != cudaSuccess ||
+            cudaFuncSetAttribute(count_segments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 max_count) != cudaSuccess)
             return LORA_ERR_CUDA;
         attr_set = true;
     }
@@ -186,8 +270,8 @@ int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *per
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    if (cudaLaunchKernelEx(&cfg, build_segments_kernel, ids, T, n, perm, seg_ptr, seg_adapter, num_segs,
-                           status) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, counting ? count_segments_kernel : build_segments_kernel, ids, T, n, perm,
+                           seg_ptr, seg_adapter, num_segs, status) != cudaSuccess)
         return LORA_ERR_CUDA;
     return LORA_OK;
 }
