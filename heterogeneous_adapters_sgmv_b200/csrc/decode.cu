@@ -80,6 +80,10 @@ struct __align__(8) SmemCtl {
     int32_t pending[kTokChunk];   // producer's token list while grouping ids
 };
 constexpr int kCtlBytes = 256;
+#ifndef LORA_TRACE_TILE0
+#define LORA_TRACE_TILE0 0
+#endif
+constexpr int kTraceTile0 = LORA_TRACE_TILE0;   // instrumented builds: first of the two traced tiles
 static_assert(sizeof(SmemCtl) <= kCtlBytes, "ctl");
 
 template <typename E> struct Tr;
@@ -560,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     for (int it = 0; live; ++it) {
         const int s1 = s + 1 == S ? 0 : s + 1;        // stage of the next tile
         const uint32_t ph1 = s1 == 0 ? ph ^ 1u : ph;
-        if (tid == 0 && it < 2) LORA_TRACE_MARK(5 + 5 * it);
+        if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(5 + 5 * (it - kTraceTile0));
         const StageHeader &hdr = stage_header(s);
         const int kind = hdr.kind;
         if (kind == kTileEnd) break;
@@ -570,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         if (tid == 0 && u < 8 && kind == kTileShrink && (flags & kFlagFirst)) LORA_TRACE_MARK(32 + 4 * u);
 
         named_bar_sync(1, kConsumers);   // every consumer is done with the previous tile's buffers
-        if (tid == 0 && it < 2) LORA_TRACE_MARK(6 + 5 * it);
+        if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(6 + 5 * (it - kTraceTile0));
         uint8_t *rows = kind == kTileShrink ? xs : ys;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -583,9 +587,9 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         if (!mbar_wait(smem_u32(&ctl.meta[s1]), ph1, p.status)) break;
         if (stage_header(s1).kind != kTileEnd) load_rows(stage_header(s1));
         if (!mbar_wait(smem_u32(&ctl.full[s]), ph, p.status)) break;
-        if (tid == 0 && it < 2) LORA_TRACE_MARK(7 + 5 * it);
+        if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(7 + 5 * (it - kTraceTile0));
         named_bar_sync(1, kConsumers);
-        if (tid == 0 && it < 2) LORA_TRACE_MARK(8 + 5 * it);
+        if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(8 + 5 * (it - kTraceTile0));
 
         if (kind == kTileShrink) {
             const bool first = flags & kFlagFirst;
@@ -833,7 +837,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 }
             }
         }
-        if (tid == 0 && it < 2) LORA_TRACE_MARK(9 + 5 * it);
+        if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(9 + 5 * (it - kTraceTile0));
         if (tid == 0 && kind == kTileExpand && (flags & kFlagLast) && u >= 1 && u <= 8) LORA_TRACE_MARK(35 + 4 * (u - 1));
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
@@ -942,7 +946,8 @@ int launch_one(const DecodeParams &p0, int units, cudaStream_t s)
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    const int G = max(1, min(ls.clusters, units));
+    int G = max(1, min(ls.clusters, units));
+    if (options().decode_max_clusters > 0) G = min(G, (int)options().decode_max_clusters);
     cfg.gridDim = dim3(G * CL);
     if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return LORA_ERR_CUDA;
     return LORA_OK;

@@ -28,6 +28,7 @@ Options &options()
         o.decode_stages = env_or("LORA_DECODE_STAGES", o.decode_stages);
         o.decode_ctas_per_sm = env_or("LORA_DECODE_CTAS_PER_SM", o.decode_ctas_per_sm);
         o.decode_cluster = env_or("LORA_DECODE_CLUSTER", o.decode_cluster);
+        o.decode_max_clusters = env_or("LORA_DECODE_MAX_CLUSTERS", o.decode_max_clusters);
         o.prefill_min_seg_len = env_or("LORA_PREFILL_MIN_SEG_LEN", o.prefill_min_seg_len);
         o.split = env_or("LORA_SPLIT", o.split);
     });
@@ -563,6 +564,7 @@ int lora_set_option(const char *key, int64_t value)
     else if (!std::strcmp(key, "decode_stages")) o.decode_stages = value;
     else if (!std::strcmp(key, "decode_ctas_per_sm")) o.decode_ctas_per_sm = value;
     else if (!std::strcmp(key, "decode_cluster")) o.decode_cluster = value;
+    else if (!std::strcmp(key, "decode_max_clusters")) o.decode_max_clusters = value;
     else if (!std::strcmp(key, "prefill_min_seg_len")) o.prefill_min_seg_len = value;
     else if (!std::strcmp(key, "split")) o.split = value;
     else return LORA_ERR_INVALID_ARG;
@@ -577,6 +579,7 @@ int lora_get_option(const char *key, int64_t *value)
     else if (!std::strcmp(key, "decode_stages")) *value = o.decode_stages;
     else if (!std::strcmp(key, "decode_ctas_per_sm")) *value = o.decode_ctas_per_sm;
     else if (!std::strcmp(key, "decode_cluster")) *value = o.decode_cluster;
+    else if (!std::strcmp(key, "decode_max_clusters")) *value = o.decode_max_clusters;
     else if (!std::strcmp(key, "prefill_min_seg_len")) *value = o.prefill_min_seg_len;
     else if (!std::strcmp(key, "split")) *value = o.split;
     else return LORA_ERR_INVALID_ARG;

@@ -57,6 +57,7 @@ struct Options {
     int64_t decode_stages = 0;       // 0: automatic
     int64_t decode_ctas_per_sm = 0;  // 0: automatic
     int64_t decode_cluster = 0;      // 0: automatic; else 1, 2, 4 or 8 CTAs per cluster
+    int64_t decode_max_clusters = 0; // 0: as many as are co-resident
     int64_t prefill_min_seg_len = 256;
     int64_t split = 0;
 };
