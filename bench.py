@@ -357,7 +357,9 @@ def run_ours(args, rank, world, local_rank):
     kernel_ms = ms_step if launches_per_step == 1 else None
     achieved = bytes_step / (ms_step / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": profile_traffic(args.workload),
+                "frac": round(achieved / peak, 4),
+                "traffic": profile_traffic(args.workload) if not (args.grouped or args.sigma != "none" or
+                                                                   args.merge > 1) else None,
                 "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
                 else "fallback 6.65 TB/s",
                 "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),

@@ -292,15 +292,22 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     if (valid) {
         // CTA j reduces rows [16 j, 16 j + 16) over the 8 partials, in CTA order
         const uint32_t part_addr = smem_u32(part);
-        for (int e = tid; e < 16 * r; e += kThreadsPF) {
-            const int rr = crank * 16 + e / r, k = e % r;
-            float sum = 0.f;
-            float pv[kKSplit];
+        // (four columns per load: r is a multiple of 8 on this path; same order of additions)
+        const int q4 = r >> 2;
+        for (int e = tid; e < 16 * q4; e += kThreadsPF) {
+            const int rr = crank * 16 + e / q4, k = (e % q4) * 4;
+            float4 pv[kKSplit];
 #pragma unroll
-            for (int j = 0; j < kKSplit; ++j) pv[j] = ld_dsmem_f32(part_addr + 4u * (rr * PRS + k), j);
+            for (int j = 0; j < kKSplit; ++j) pv[j] = ld_dsmem_f32x4(part_addr + 4u * (rr * PRS + k), j);
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < kKSplit; ++j) sum += pv[j];
-            if (rr < rows) p.v[(int64_t)(row0 + rr) * p.ldv + k] = sum;
+            for (int j = 0; j < kKSplit; ++j) {
+                sum.x += pv[j].x;
+                sum.y += pv[j].y;
+                sum.z += pv[j].z;
+                sum.w += pv[j].w;
+            }
+            if (rr < rows) *reinterpret_cast<float4 *>(p.v + (int64_t)(row0 + rr) * p.ldv + k) = sum;
         }
     }
     cluster_sync_all();   // no peer reads this CTA's partial any more
