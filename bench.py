@@ -146,6 +146,30 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ----------------------------------------------------------------------------- ranks
+# One process per GPU, each an independent replica with its own token batch (the path
+# shards by tokens and exchanges nothing).  The job is as slow as its slowest rank.
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Seed of rank `rank`'s batch: every replica draws its own inputs."""
+    return workloads.SEED_BASE + workloads.WORKLOAD_NAMES.index(workload) + 1000 * rank
+
+
+def max_over_ranks(value: float, dist=None, device=None) -> float:
+    """The largest per-rank value (a time) over all ranks; the value itself without a group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank processed `steps` steps in at most `ms` milliseconds."""
+    return world * tokens_per_step * steps / (ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- our arm
 
 class Copy:
@@ -258,8 +282,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         import torch.distributed as dist
 
-    seed = workloads.SEED_BASE + workloads.WORKLOAD_NAMES.index(args.workload) + 1000 * rank
-    wl = workloads.generate(args.workload, seed=seed)
+    wl = workloads.generate(args.workload, seed=rank_seed(args.workload, rank))
     T = wl.T
     step, launches_per_step, kname = make_step(wl, L, args.grouped, args.merge)
     if args.jd_clusters and args.sigma == "none":
@@ -344,13 +367,9 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
     if dist:
         dist.barrier(device_ids=[local_rank])
-    ms = float(ev0.elapsed_time(ev1))
-    if dist:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(float(ev0.elapsed_time(ev1)), dist, "cuda")
     ms_step = ms / K
-    value = world * T * K / (ms / 1e3)
+    value = job_throughput(world, T, K, ms)
 
     # roofline of the dominant kernel: per launch (for one-launch steps the launch is the step)
     peak, peak_kind = measured_peaks()
@@ -409,12 +428,8 @@ def run_ours(args, rank, world, local_rank):
                 e2e_step()
             e1.record(stream)
         torch.cuda.synchronize()
-        ems = float(e0.elapsed_time(e1))
-        if dist:
-            tt = torch.tensor([ems], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
-        e2e = {"value": round(world * T * Ke / (ems / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        ems = max_over_ranks(float(e0.elapsed_time(e1)), dist, "cuda")
+        e2e = {"value": round(job_throughput(world, T, Ke, ems), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": Ke, "ms_per_step": round(ems / Ke, 6),
                "path": "pinned host -> cudaMemcpyAsync -> C-ABI call -> cudaMemcpyAsync -> pinned host"}
 
