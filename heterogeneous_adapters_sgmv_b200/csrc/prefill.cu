@@ -557,24 +557,39 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 }
             }
             tc_fence_before();
+            fence_proxy_async_smem();            // the updated tile is read by the TMA unit below
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ctl.accempty[ab]));
             named_bar_sync(2, kEpiWarps * 32);   // the whole tile is updated in shared memory
-            // coalesced stores: epilogue warp ew stores rows 16 ew .. 16 ew + 15, two per step
-            uint8_t *yg = static_cast<uint8_t *>(p.y);
-            const int chunk = lane & 15;
+            const bool full_tile = inf.rows == kTileM && inf.ncols == kTileN;
+            if (full_tile) {
+                // a full tile lies inside one segment: two TMA stores write it back
+                if (ew == 0 && lane == 0) {
+                    const uint32_t yt0 = smem_u32(ring + s * kExStageBytes + 16384);
+                    tma_store_2d(&p.tmap_io, yt0, inf.col0, inf.row0);
+                    tma_store_2d(&p.tmap_io, yt0 + 16384, inf.col0 + 64, inf.row0);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();     // the stage is reused only after this warp arrives
+                }
+            } else {
+                // coalesced stores masked to the segment's rows and to o: epilogue warp ew stores
+                // rows 16 ew .. 16 ew + 15, two per step
+                uint8_t *yg = static_cast<uint8_t *>(p.y);
+                const int chunk = lane & 15;
 #pragma unroll 1
-            for (int rr = ew * 16 + (lane >> 4); rr < ew * 16 + 16; rr += 2) {
-                if (rr < inf.rows && chunk * 8 < inf.ncols) {
-                    const uint8_t *box = ring + s * kExStageBytes + 16384 + (chunk >= 8 ? 16384 : 0);
-                    const uint4 w = *reinterpret_cast<const uint4 *>(box + sw128_off(rr, chunk & 7));
-                    *reinterpret_cast<uint4 *>(
-                        yg + ((int64_t)(inf.row0 + rr) * p.ldy + p.y_off + inf.col0 + chunk * 8) * 2) = w;
+                for (int rr = ew * 16 + (lane >> 4); rr < ew * 16 + 16; rr += 2) {
+                    if (rr < inf.rows && chunk * 8 < inf.ncols) {
+                        const uint8_t *box = ring + s * kExStageBytes + 16384 + (chunk >= 8 ? 16384 : 0);
+                        const uint4 w = *reinterpret_cast<const uint4 *>(box + sw128_off(rr, chunk & 7));
+                        *reinterpret_cast<uint4 *>(
+                            yg + ((int64_t)(inf.row0 + rr) * p.ldy + p.y_off + inf.col0 + chunk * 8) * 2) = w;
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
         }
+        if (ew == 0 && lane == 0) bulk_wait_group0();   // this CTA's tile stores are complete
     }
     tc_fence_before();
     __syncthreads();
