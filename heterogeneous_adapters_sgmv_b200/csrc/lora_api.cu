@@ -30,6 +30,7 @@ Options &options()
         o.decode_cluster = env_or("LORA_DECODE_CLUSTER", o.decode_cluster);
         o.decode_max_clusters = env_or("LORA_DECODE_MAX_CLUSTERS", o.decode_max_clusters);
         o.prefill_min_seg_len = env_or("LORA_PREFILL_MIN_SEG_LEN", o.prefill_min_seg_len);
+        o.prefill_ksplit = env_or("LORA_PREFILL_KSPLIT", o.prefill_ksplit);
         o.split = env_or("LORA_SPLIT", o.split);
     });
     return o;
@@ -566,6 +567,7 @@ int lora_set_option(const char *key, int64_t value)
     else if (!std::strcmp(key, "decode_cluster")) o.decode_cluster = value;
     else if (!std::strcmp(key, "decode_max_clusters")) o.decode_max_clusters = value;
     else if (!std::strcmp(key, "prefill_min_seg_len")) o.prefill_min_seg_len = value;
+    else if (!std::strcmp(key, "prefill_ksplit")) o.prefill_ksplit = value;
     else if (!std::strcmp(key, "split")) o.split = value;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
@@ -581,6 +583,7 @@ int lora_get_option(const char *key, int64_t *value)
     else if (!std::strcmp(key, "decode_cluster")) *value = o.decode_cluster;
     else if (!std::strcmp(key, "decode_max_clusters")) *value = o.decode_max_clusters;
     else if (!std::strcmp(key, "prefill_min_seg_len")) *value = o.prefill_min_seg_len;
+    else if (!std::strcmp(key, "prefill_ksplit")) *value = o.prefill_ksplit;
     else if (!std::strcmp(key, "split")) *value = o.split;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;

@@ -59,6 +59,7 @@ struct Options {
     int64_t decode_cluster = 0;      // 0: automatic; else 1, 2, 4 or 8 CTAs per cluster
     int64_t decode_max_clusters = 0; // 0: as many as are co-resident
     int64_t prefill_min_seg_len = 256;
+    int64_t prefill_ksplit = 4;      // CTAs splitting h in the tcgen05 shrink (4 or 8)
     int64_t split = 0;
 };
 Options &options();

@@ -3,8 +3,8 @@
 // y += s_i * v . B_i^T are dense contractions ("Compress then Serve" review thread,
 // add_lora_slice pseudocode; "TGI Multi-LoRA" page, "Technical Foundation: LoRA").
 //
-// Shrink kernel: one cluster of 8 CTAs per (segment, 128-token tile); CTA j takes the j-th
-// eighth of h.  A producer thread streams x and A_i tiles (64 columns of h, 128-byte swizzle)
+// Shrink kernel: one cluster of KS CTAs (8, or 4 with the "prefill_ksplit" option) per
+// (segment, 128-token tile); CTA j takes the j-th KS-th of h.  A producer thread streams x and A_i tiles (64 columns of h, 128-byte swizzle)
 // with 2-D tensor-map TMA loads into a 4-deep ring; one thread issues tcgen05.mma
 // (M = 128 tokens, N = rank rounded up to 16, K = 16) accumulating in tensor memory; the
 // partials are summed in fixed CTA order through distributed shared memory and written to
@@ -36,8 +36,9 @@ namespace {
 constexpr int kTileM = 128;          // tokens per tile
 constexpr int kTileN = 128;          // columns of o per expand tile
 constexpr int kBK = 64;              // columns of h per shrink k-block (128 bytes of bf16)
-constexpr int kKSplit = 8;           // CTAs per shrink cluster
-constexpr int kStages = 4;           // shrink pipeline depth
+constexpr int kStagesMax = 4;        // shrink pipeline depth
+// (eight stages with the split of 4 measured slower: 17.4 against 16.3 us)
+__host__ __device__ constexpr int shrink_stages(int) { return 4; }
 constexpr int kThreadsPF = 128;      // 4 warps: one TMEM lane quarter each
 constexpr int kMaxRankPF = 64;
 
@@ -173,21 +174,24 @@ __device__ bool find_tile(const PrefillParams &p, int g, int *seg, int *row0, in
 }
 
 struct __align__(8) ShrinkCtl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kStagesMax];
+    uint64_t empty[kStagesMax];
     uint64_t done;
     uint32_t tmem_base;
     int32_t info[5];   // valid, row0, rows, adapter, rank
 };
 
+template <int KS>
 __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __grid_constant__ PrefillParams p)
 {
+    constexpr int kRowsPerCta = kTileM / KS;   // rows of the tile each CTA reduces
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the swizzled tiles
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int kXBytes = kTileM * 128;              // 16 KiB
     constexpr int kABytes = kMaxRankPF * 128;          //  8 KiB (room for rank <= 64)
     constexpr int kStageBytes = kXBytes + kABytes;
+    constexpr int kStages = shrink_stages(KS);
     ShrinkCtl &ctl = *reinterpret_cast<ShrinkCtl *>(smem + kStages * kStageBytes);
     float *part = reinterpret_cast<float *>(smem);     // [128][PRS] fp32, reuses the ring after the MMAs
     constexpr int PRS = kMaxRankPF + 4;                // padded row stride of the partial
@@ -230,8 +234,8 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     const int npad = (r + 15) & ~15;
     const uint32_t tmem = ctl.tmem_base;
     const int nkb_all = (p.h + kBK - 1) / kBK;
-    const int kb0 = (int)((int64_t)crank * nkb_all / kKSplit);
-    const int kb1 = (int)((int64_t)(crank + 1) * nkb_all / kKSplit);
+    const int kb0 = (int)((int64_t)crank * nkb_all / KS);
+    const int kb1 = (int)((int64_t)(crank + 1) * nkb_all / KS);
     const int nkb = valid ? kb1 - kb0 : 0;
     bool ok = true;
 
@@ -294,14 +298,14 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
         const uint32_t part_addr = smem_u32(part);
         // (four columns per load: r is a multiple of 8 on this path; same order of additions)
         const int q4 = r >> 2;
-        for (int e = tid; e < 16 * q4; e += kThreadsPF) {
-            const int rr = crank * 16 + e / q4, k = (e % q4) * 4;
-            float4 pv[kKSplit];
+        for (int e = tid; e < kRowsPerCta * q4; e += kThreadsPF) {
+            const int rr = crank * kRowsPerCta + e / q4, k = (e % q4) * 4;
+            float4 pv[KS];
 #pragma unroll
-            for (int j = 0; j < kKSplit; ++j) pv[j] = ld_dsmem_f32x4(part_addr + 4u * (rr * PRS + k), j);
+            for (int j = 0; j < KS; ++j) pv[j] = ld_dsmem_f32x4(part_addr + 4u * (rr * PRS + k), j);
             float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < kKSplit; ++j) {
+            for (int j = 0; j < KS; ++j) {
                 sum.x += pv[j].x;
                 sum.y += pv[j].y;
                 sum.z += pv[j].z;
@@ -627,9 +631,10 @@ int encode_sw128(CUtensorMap *out, const void *base, uint64_t cols, uint64_t row
     return rc == CUDA_SUCCESS ? LORA_OK : LORA_ERR_UNSUPPORTED;
 }
 
-constexpr int kShrinkSmem = kStages * (kTileM * 128 + kMaxRankPF * 128) + 256 + 1024;
+constexpr int shrink_smem(int ks) { return shrink_stages(ks) * (kTileM * 128 + kMaxRankPF * 128) + 256 + 1024; }
 constexpr int kExpandSmem = 2 * kExVBytes + kExStages * kExStageBytes + (int)sizeof(ExpandCtl) + 1024;
-static_assert(kStages * (kTileM * 128 + kMaxRankPF * 128) >= kTileM * (kMaxRankPF + 4) * 4, "partial fits ring");
+static_assert(shrink_stages(8) * (kTileM * 128 + kMaxRankPF * 128) >= kTileM * (kMaxRankPF + 4) * 4, "partial fits ring");
+static_assert(shrink_smem(4) <= 227 * 1024, "shrink shared memory");
 
 }  // namespace
 
@@ -690,8 +695,10 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LORA_ERR_CUDA;
     if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(prefill_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kShrinkSmem) !=
-                cudaSuccess ||
+        if (cudaFuncSetAttribute(prefill_shrink_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 shrink_smem(8)) != cudaSuccess ||
+            cudaFuncSetAttribute(prefill_shrink_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 shrink_smem(4)) != cudaSuccess ||
             cudaFuncSetAttribute(prefill_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kExpandSmem) !=
                 cudaSuccess)
             return LORA_ERR_CUDA;
@@ -699,18 +706,19 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
     }
     const Options &opt = options();
 
-    // shrink: clusters of kKSplit CTAs, one cluster per 128-token tile
+    // shrink: clusters of KS CTAs (split of h), one cluster per 128-token tile
     int rc = encode_sw128(&p.tmap_io, x, (uint64_t)t->h, (uint64_t)seg->T, (uint64_t)ldx, kTileM);
     if (rc != LORA_OK) return rc;
     {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(kKSplit * mt_bound);
+        const int KS = opt.prefill_ksplit == 8 ? 8 : 4;
+        cfg.gridDim = dim3(KS * mt_bound);
         cfg.blockDim = dim3(kThreadsPF);
-        cfg.dynamicSmemBytes = kShrinkSmem;
+        cfg.dynamicSmemBytes = shrink_smem(KS);
         cfg.stream = s;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = kKSplit;
+        attr[0].val.clusterDim.x = KS;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         int na = 1;
@@ -721,7 +729,9 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
         }
         cfg.attrs = attr;
         cfg.numAttrs = na;
-        if (cudaLaunchKernelEx(&cfg, prefill_shrink_kernel, p) != cudaSuccess) return LORA_ERR_CUDA;
+        const cudaError_t e = KS == 4 ? cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<4>, p)
+                                      : cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<8>, p);
+        if (e != cudaSuccess) return LORA_ERR_CUDA;
     }
     // expand: persistent, one CTA per SM over all (128-token tile, 128-column tile) pairs
     rc = encode_sw128(&p.tmap_io, static_cast<uint8_t *>(y) + (int64_t)y_off * 2, (uint64_t)t->o, (uint64_t)seg->T,

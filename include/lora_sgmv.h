@@ -233,7 +233,8 @@ const char *lora_status_string(int code);
  * "decode_cluster" (0: automatic, else 1, 2, 4 or 8 CTAs sharing one decode work unit; the
  * width changes the fp32 summation order, so results can differ in the last bits between
  * widths), "decode_max_clusters" (0: every co-resident cluster; else an upper bound on
- * the persistent decode grid, for tuning), "prefill_min_seg_len" (segment-length hint at or above which lora_sgmv takes the tcgen05
+ * the persistent decode grid, for tuning), "prefill_ksplit" (4, the default, or 8 CTAs splitting
+ * h in the tcgen05 shrink), "prefill_min_seg_len" (segment-length hint at or above which lora_sgmv takes the tcgen05
  * path; 0 disables that path), "split" (1: lora_sgmv runs lora_shrink then lora_expand
  * through the workspace instead of the fused kernel).  Returns LORA_ERR_INVALID_ARG for an
  * unknown key. */
