@@ -4,30 +4,38 @@
 // "TGI Multi-LoRA" page, "Technical Foundation: LoRA").
 //
 // Design for sm_100a:
-//  * A cluster of CL CTAs (CL = 8, 4, 2 or 1, picked per launch from the number of work units)
-//    owns one work unit at a time: up to 16 tokens of one adapter (one SGMV segment chunk, or
-//    one group of equal ids in the per-token BGMV form).  CTA j of the cluster streams the j-th
-//    CL-th of h for the shrink and the j-th CL-th of o for the expand, so each adapter's A_i
-//    and B_i are read once per unit and every token of the unit reuses that read.  Few units
-//    (a small decode batch) take wide clusters so every SM streams; many units take narrow
-//    ones so units run side by side instead of one after another.
+//  * A cluster of CL CTAs (8 by default; 4, 2 or 1 through the "decode_cluster" option or when
+//    the exchange buffers of wider clusters do not fit) owns one work unit at a time: up to 16
+//    tokens of one adapter (a 16-token chunk of an SGMV segment, or of a group of equal ids in
+//    the per-token BGMV form).  CTA j of the cluster streams the j-th CL-th of h for the shrink
+//    and the j-th CL-th of o for the expand, so each adapter's A_i and B_i are read once per
+//    unit and every token of the unit reuses that read.  Segment chunks are dealt to clusters
+//    round-robin, so a long segment spreads over many clusters.
 //  * One producer warp per CTA runs ahead across units: it stages this CTA's slice of A_i with
 //    2-D tensor-map TMA loads (one or two instructions per unit) and its slice of B_i with one
 //    bulk copy, into a ring of shared-memory stages guarded by mbarriers, and hints the unit's
 //    x and y rows into L2.  No multicast anywhere.
-//  * Consumer warps stage x (and the unit's y) rows with coalesced 128-bit loads.  Shrink:
-//    warp-level split-K; a warp owns rank rows k = warp + 8 i, a lane 16 bytes at two places of
-//    each 1 KiB row; each dot product is folded across the warp with a 5-step butterfly.
+//  * Consumer warps load the next tile's x (or y) rows with coalesced 128-bit loads while the
+//    current tile computes.  Shrink: warp-level split-K; a warp owns rank rows k = warp + 8 i, a
+//    lane 16 bytes at two places of each 1 KiB row; two tokens x two rows are formed at once
+//    and folded across the warp by one transposed butterfly (the summation tree of a plain
+//    butterfly, so the blocking does not change results).
 //  * Each CTA pushes its partial intermediate into every peer's shared memory with st.async
 //    (completion counted in bytes on the peer's mbarrier); every CTA then sums the CL partials
 //    in fixed CTA order.  No atomics, no grid barrier: bit-identical run to run.  A cluster of
-//    one keeps its own sum and exchanges nothing.
-//  * Expand: a thread owns two output columns (bf16) and walks the unit's tokens; one rounding
-//    (nearest-even) per output, coalesced 32-bit stores.
-//  * Short kernels like this one are dominated by instruction fetch, so the per-unit code is
-//    kept to a few compact loops (no wide unrolling, no run-time integer division), and work
-//    that reads no input (barrier set-up, the adapter descriptor when a cluster owns a fixed
-//    adapter) happens before the wait on the previous grid.
+//    one keeps its own sum and exchanges nothing.  The three-stage form applies the adapter's
+//    Sigma_i (full or diagonal) to the summed intermediate here.
+//  * Expand: a thread owns two output columns (bf16) and takes the unit's tokens two at a time,
+//    sharing each B_i load; products are added in ascending k, one rounding (nearest-even) per
+//    output, coalesced 32-bit stores.  A per-token weight (merged ensembles) multiplies the
+//    scale.
+//  * A grouped launch carries up to four projections (tables, x, y slices); each unit then
+//    runs once per projection, back to back on the same cluster.
+//  * Short kernels like this one are dominated by instruction fetch and dependent latency, so
+//    the per-unit code is kept to a few compact loops (no run-time integer division), and
+//    work that reads no input (barrier set-up; in the direct BGMV mode the adapter descriptor
+//    and the copies of the first stages of the cluster's adapter) happens before the wait on
+//    the previous grid.
 //  * Persistent grid: as many clusters as fit, each walking the unit list with a stride.
 #include <cuda.h>
 #include <cudaTypedefs.h>
