@@ -4,6 +4,8 @@ import ctypes
 import os
 import re
 
+import pytest
+
 import heterogeneous_adapters_sgmv_b200 as L
 from heterogeneous_adapters_sgmv_b200 import build as B
 
@@ -78,3 +80,31 @@ def test_product_path_does_not_use_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, f)).read().lower()
                 assert "oracle" not in src, f
+
+
+def test_every_documented_option_round_trips():
+    """Each runtime option the header documents can be set and read back (host only), and an
+    unknown key is rejected."""
+    txt = open(os.path.join(ROOT, "include", "lora_sgmv.h")).read()
+    block = txt[txt.index("Runtime knobs"):txt.index("int lora_set_option")]
+    keys = re.findall(r'"([a-z_]+)"', block)
+    assert {"pdl", "decode_stages", "decode_ctas_per_sm", "decode_cluster", "decode_max_clusters",
+            "prefill_ksplit", "prefill_min_seg_len", "split"} <= set(keys)
+    for key in keys:
+        old = L.lora_get_option(key)
+        try:
+            L.lora_set_option(key, old + 3)
+            assert L.lora_get_option(key) == old + 3
+        finally:
+            L.lora_set_option(key, old)
+        assert L.lora_get_option(key) == old
+    with pytest.raises(L.LoraError):
+        L.lora_set_option("no_such_option", 1)
+
+
+def test_merged_and_sigma_host_checks():
+    """Argument checks of the next-row entry points that need no device."""
+    lib = L._load()
+    assert lib.lora_table_set_sigma(None, L.LORA_SIGMA_FULL, None, None) == L.LORA_ERR_INVALID_ARG
+    assert lib.lora_bgmv_merged(None, None, None, 4, 2, None, 0, None, 0, 0, None, 0, None) == \
+        L.LORA_ERR_INVALID_ARG
