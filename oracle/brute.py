@@ -32,3 +32,41 @@ def lora_delta(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray,
         s = float(np.float32(scales[i]))
         out[rows] += s * ((xd[rows] @ Ai.T) @ Bi.T)
     return out
+
+
+def lora_delta_sigma(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray,
+                     A: Sequence[np.ndarray], B: Sequence[np.ndarray], scales: Sequence[float],
+                     sigma_kind: int, sigma: Sequence[np.ndarray]) -> np.ndarray:
+    """Three-stage form per adapter group: y0 + s_i * ((x_g @ A_i^T) @ Sigma_i^T) @ B_i^T, with
+    Sigma_i full (sigma_kind 1) or diagonal (sigma_kind 2)."""
+    ids = np.asarray(ids)
+    if ((ids < -1) | (ids >= len(A))).any():
+        raise ValueError("adapter id out of range")
+    xd = to_float64(x, dtype)
+    out = to_float64(y0, dtype).copy()
+    for i in np.unique(ids[ids >= 0]):
+        rows = np.nonzero(ids == i)[0]
+        S = np.asarray(sigma[i], dtype=np.float64)
+        S = S if sigma_kind == 1 else np.diag(S)
+        u = xd[rows] @ to_float64(A[i], dtype).T
+        out[rows] += float(np.float32(scales[i])) * ((u @ S.T) @ to_float64(B[i], dtype).T)
+    return out
+
+
+def lora_delta_merged(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray, w: np.ndarray,
+                      A: Sequence[np.ndarray], B: Sequence[np.ndarray], scales: Sequence[float]) -> np.ndarray:
+    """Merged ensembles, grouped by (slot, adapter): for every slot j and adapter i, the tokens
+    whose slot j names i gain w[t, j] * s_i * (x_g @ A_i^T) @ B_i^T."""
+    ids = np.asarray(ids)
+    w = np.asarray(w, dtype=np.float64)
+    if ((ids < -1) | (ids >= len(A))).any():
+        raise ValueError("adapter id out of range")
+    xd = to_float64(x, dtype)
+    out = to_float64(y0, dtype).copy()
+    for j in range(ids.shape[1]):
+        col = ids[:, j]
+        for i in np.unique(col[col >= 0]):
+            rows = np.nonzero(col == i)[0]
+            d = (xd[rows] @ to_float64(A[i], dtype).T) @ to_float64(B[i], dtype).T
+            out[rows] += (w[rows, j] * float(np.float32(scales[i])))[:, None] * d
+    return out

@@ -74,6 +74,8 @@ PIN_TESTS = [
     pins.test_merged_single_slot_unit_weight_is_the_plain_delta,
     pins.test_merged_equals_merged_weight_closed_form,
     pins.test_merged_slot_order_and_duplicate_slots,
+    lambda: [pins.test_sigma_loop_matches_grouped_products(k, d) for k in ("full", "diag") for d in (False, True)],
+    lambda: [pins.test_merged_loop_matches_grouped_products(d) for d in (False, True)],
 ]
 
 

@@ -515,3 +515,30 @@ def test_merged_empty_slots_and_bad_ids():
     bad[3, 1] = wl.n
     with pytest.raises(oracle.OracleError):
         oracle.lora_delta_merged(wl.dtype, p.x, p.y0, bad, w, A, B, p.scales)
+
+
+@pytest.mark.parametrize("kind", ["full", "diag"])
+@pytest.mark.parametrize("delta_only", [False, True])
+def test_sigma_loop_matches_grouped_products(kind, delta_only):
+    """The C loop's three-stage form against numpy products per adapter group (a different
+    evaluation order and code)."""
+    wl = workloads.generate("multirank_decode", delta_only=delta_only, T=60, n=11, shapes=[("q", 200, 120, 0)])
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    sig = workloads.draw_sigma(p.ranks, kind, seed=13)
+    k = oracle.SIGMA_FULL if kind == "full" else oracle.SIGMA_DIAG
+    ref = oracle.lora_delta_sigma(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales, k, sig)
+    alt = brute.lora_delta_sigma(wl.dtype, p.x, p.y0, wl.ids, A, B, p.scales, k, sig)
+    assert np.abs(ref - alt).max() <= 1e-12 * max(np.abs(alt).max(), 1e-30)
+
+
+@pytest.mark.parametrize("delta_only", [False, True])
+def test_merged_loop_matches_grouped_products(delta_only):
+    wl = workloads.generate("many_adapter_qkvo", delta_only=delta_only, T=48, n=30,
+                            shapes=[("q", 128, 96, 0)])
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    ids, w = workloads.draw_merge(wl.ids, wl.n, 3, seed=6, empty=0.3)
+    ref = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids, w, A, B, p.scales)
+    alt = brute.lora_delta_merged(wl.dtype, p.x, p.y0, ids, w, A, B, p.scales)
+    assert np.abs(ref - alt).max() <= 1e-12 * max(np.abs(alt).max(), 1e-30)
