@@ -1,6 +1,7 @@
 // C ABI of liblora_sgmv.so: adapter tables, host-side validation, workspace carving and the
 // choice of device path.  Nothing here computes the delta; every step runs in the kernels of
 // decode.cu, segments.cu and prefill.cu.
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -39,7 +40,7 @@ Options &options()
 // prefill.cu
 bool prefill_supported(const lora_table *t);
 int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y,
-                   int64_t ldy, int32_t y_off, float *v, int32_t ldv, cudaStream_t s);
+                   int64_t ldy, int32_t y_off, void *v, cudaStream_t s);
 
 }  // namespace lora
 
@@ -66,7 +67,10 @@ WsLayout ws_layout(const lora_table *t, int32_t T)
     WsLayout w;
     size_t off = 0;
     w.v = off;
-    off += up256((size_t)T * ldv_of(t) * sizeof(float));
+    // the fp32 intermediate, or (tcgen05 path) its bf16 hi and lo parts of 64 columns each
+    size_t vbytes = (size_t)T * ldv_of(t) * sizeof(float);
+    if (t->d_tmaps_pfA) vbytes = std::max(vbytes, (size_t)T * 64 * 2 * sizeof(uint16_t));
+    off += up256(vbytes);
     w.perm = off;
     off += up256((size_t)T * sizeof(int32_t));
     w.seg_ptr = off;
@@ -347,7 +351,7 @@ int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int6
         if (!ws || ws_bytes < w.total) return LORA_ERR_WORKSPACE;
         if (!al16(ws)) return LORA_ERR_UNSUPPORTED;
         float *v = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + w.v);
-        if (prefill) return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, ldv_of(t), s);
+        if (prefill) return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, s);
         if ((rc = lora_shrink(t, seg, x, ldx, v, ldv_of(t), stream))) return rc;
         return lora_expand(t, seg, v, ldv_of(t), y, ldy, y_off, stream);
     }

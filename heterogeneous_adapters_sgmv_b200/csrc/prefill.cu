@@ -3,20 +3,21 @@
 // y += s_i * v . B_i^T are dense contractions ("Compress then Serve" review thread,
 // add_lora_slice pseudocode; "TGI Multi-LoRA" page, "Technical Foundation: LoRA").
 //
-// Shrink kernel: one cluster of KS CTAs (8, or 4 with the "prefill_ksplit" option) per
-// (segment, 128-token tile); CTA j takes the j-th KS-th of h.  A producer thread streams x and A_i tiles (64 columns of h, 128-byte swizzle)
-// with 2-D tensor-map TMA loads into a 4-deep ring; one thread issues tcgen05.mma
-// (M = 128 tokens, N = rank rounded up to 16, K = 16) accumulating in tensor memory; the
-// partials are summed in fixed CTA order through distributed shared memory and written to
-// v in fp32.
+// Shrink kernel: one cluster of KS CTAs (4, or 8 with the "prefill_ksplit" option) per
+// (segment, 128-token tile); CTA j takes the j-th KS-th of h.  A producer thread streams x
+// and A_i tiles (64 columns of h, 128-byte swizzle) with 2-D tensor-map TMA loads into a
+// 4-deep ring; one thread issues tcgen05.mma (M = 128 tokens, N = rank rounded up to 16,
+// K = 16) accumulating in tensor memory; the partials are summed in fixed CTA order through
+// distributed shared memory, and the fp32 sum is stored as bf16 hi + lo (v = hi + lo to about
+// 16 bits, zero past the rank).
 //
-// Expand kernel: one CTA per (segment, 128-token tile, 128-column tile of o).  The fp32
-// intermediate is split into bf16 hi + lo (v = hi + lo to about 16 bits), written into shared
-// memory in the 128-byte-swizzled K-major layout the tensor core reads, and multiplied with
-// the B_i tile (TMA) in 8 MMAs of K = 16.  The y tile arrives by TMA; the epilogue reads the
-// accumulator from tensor memory row by row, adds s_i * acc to y, rounds once to bf16 and
-// stores with coalesced 16-byte stores masked to the segment, so neighbouring segments are
-// never touched.
+// Expand kernel: persistent CTAs over the (128-token tile, 128-column tile of o) pairs.  Both
+// parts of the intermediate come in by TMA, already in the 128-byte-swizzled K-major layout
+// the tensor core reads, and are multiplied with the B_i tile (TMA) in 8 MMAs of K = 16.  The
+// y tile arrives by TMA; the epilogue reads the accumulator from tensor memory row by row,
+// adds s_i * acc to y in shared memory, rounds once to bf16, and writes a full tile back with
+// TMA stores, a partial one with coalesced 16-byte stores masked to the segment, so
+// neighbouring segments are never touched.
 //
 // No TMA multicast.  Every wait is bounded; on timeout a status bit is latched, in-flight
 // copies are drained and tensor memory is released before the CTA exits.
@@ -122,13 +123,13 @@ __device__ __forceinline__ uint32_t sw128_off(int m, int c) { return (uint32_t)(
 
 struct PrefillParams {
     CUtensorMap tmap_io;          // shrink: x [T, h]; expand: y slice [T, o]   (box 64 x 128)
+    CUtensorMap tmap_vhi, tmap_vlo;   // expand: intermediate hi / lo parts [T, 64] bf16 (box 64 x 128)
     const AdapterDesc *desc;
     const uint8_t *tm_A;          // per adapter: tensor map of A_i, box 64 x roundup(r, 16)
     const uint8_t *tm_B;          // per adapter: tensor map of B_i, box 64 x 128
     const int32_t *seg_ptr, *seg_adapter, *num_segs;
     int32_t max_segs, T, h, o, n;
-    float *v;
-    int32_t ldv;
+    uint16_t *v_hi, *v_lo;        // the fp32 intermediate as bf16 hi + lo, [T, 64] each, zero past the rank
     void *y;
     int64_t ldy;
     int32_t y_off;
@@ -296,22 +297,38 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     if (valid) {
         // CTA j reduces rows [16 j, 16 j + 16) over the 8 partials, in CTA order
         const uint32_t part_addr = smem_u32(part);
-        // (four columns per load: r is a multiple of 8 on this path; same order of additions)
+        // Four columns per load (r is a multiple of 8 on this path; same order of additions).
+        // The sum is stored as bf16 hi + lo (v = hi + lo to about 16 bits), the layout the
+        // expand's tensor-core operand takes by TMA; columns past r are zero.
+        constexpr int q4all = kMaxRankPF / 4;
         const int q4 = r >> 2;
-        for (int e = tid; e < kRowsPerCta * q4; e += kThreadsPF) {
-            const int rr = crank * kRowsPerCta + e / q4, k = (e % q4) * 4;
-            float4 pv[KS];
-#pragma unroll
-            for (int j = 0; j < KS; ++j) pv[j] = ld_dsmem_f32x4(part_addr + 4u * (rr * PRS + k), j);
+        for (int e = tid; e < kRowsPerCta * q4all; e += kThreadsPF) {
+            const int rr = crank * kRowsPerCta + e / q4all, kq = e % q4all, k = kq * 4;
             float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (kq < q4) {
+                float4 pv[KS];
 #pragma unroll
-            for (int j = 0; j < KS; ++j) {
-                sum.x += pv[j].x;
-                sum.y += pv[j].y;
-                sum.z += pv[j].z;
-                sum.w += pv[j].w;
+                for (int j = 0; j < KS; ++j) pv[j] = ld_dsmem_f32x4(part_addr + 4u * (rr * PRS + k), j);
+#pragma unroll
+                for (int j = 0; j < KS; ++j) {
+                    sum.x += pv[j].x;
+                    sum.y += pv[j].y;
+                    sum.z += pv[j].z;
+                    sum.w += pv[j].w;
+                }
             }
-            if (rr < rows) *reinterpret_cast<float4 *>(p.v + (int64_t)(row0 + rr) * p.ldv + k) = sum;
+            if (rr < rows) {
+                const __nv_bfloat162 h01 = __floats2bfloat162_rn(sum.x, sum.y);
+                const __nv_bfloat162 h23 = __floats2bfloat162_rn(sum.z, sum.w);
+                const float2 g01 = __bfloat1622float2(h01), g23 = __bfloat1622float2(h23);
+                const __nv_bfloat162 l01 = __floats2bfloat162_rn(sum.x - g01.x, sum.y - g01.y);
+                const __nv_bfloat162 l23 = __floats2bfloat162_rn(sum.z - g23.x, sum.w - g23.y);
+                const int64_t off = (int64_t)(row0 + rr) * kMaxRankPF + k;
+                *reinterpret_cast<uint2 *>(p.v_hi + off) =
+                    make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
+                *reinterpret_cast<uint2 *>(p.v_lo + off) =
+                    make_uint2(*reinterpret_cast<const uint32_t *>(&l01), *reinterpret_cast<const uint32_t *>(&l23));
+            }
         }
     }
     cluster_sync_all();   // no peer reads this CTA's partial any more
@@ -414,7 +431,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        int cur_g = -1, vcount = 0, row0 = 0, rows = 0, a = 0, r = 0, vb = 0;
+        int cur_g = -1, vcount = 0, row0 = 0, rows = 0, a = 0, vb = 0;
         float sc = 0.f;
         for (int t = t0; t < t1 && ok; ++t) {
             const int i = t - t0, s = i % kExStages;
@@ -428,7 +445,6 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                     rows = 0;
                     a = 0;
                 }
-                r = rows > 0 ? p.desc[a].rank : 0;
                 sc = p.desc[a].scale;
                 cur_g = g;
                 vb = vcount & 1;
@@ -436,37 +452,16 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                     ok = false;
                     break;
                 }
-                // intermediate tile: row m, 4 columns per lane-quarter, hi and lo bf16, swizzled
-                uint8_t *vhi = vbuf + vb * kExVBytes, *vlo = vhi + 16384;
-                const int k = (lane & 15) * 4;
-                for (int b0 = 0; b0 < kTileM / 2; b0 += 16) {
-                    // 16 independent loads in flight, then convert: one round trip per batch
-                    float4 fb[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int m = (b0 + j) * 2 + (lane >> 4);
-                        fb[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (m < rows && k < r) fb[j] = *reinterpret_cast<const float4 *>(p.v + (int64_t)(row0 + m) * p.ldv + k);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                    const int m = (b0 + j) * 2 + (lane >> 4);
-                    const float4 f = fb[j];
-                    const __nv_bfloat162 h01 = __floats2bfloat162_rn(f.x, f.y);
-                    const __nv_bfloat162 h23 = __floats2bfloat162_rn(f.z, f.w);
-                    const float2 g01 = __bfloat1622float2(h01), g23 = __bfloat1622float2(h23);
-                    const __nv_bfloat162 l01 = __floats2bfloat162_rn(f.x - g01.x, f.y - g01.y);
-                    const __nv_bfloat162 l23 = __floats2bfloat162_rn(f.z - g23.x, f.w - g23.y);
-                    const uint32_t off = sw128_off(m, k >> 3) + ((k & 4) ? 8 : 0);
-                    *reinterpret_cast<uint2 *>(vhi + off) =
-                        make_uint2(*reinterpret_cast<const uint32_t *>(&h01), *reinterpret_cast<const uint32_t *>(&h23));
-                    *reinterpret_cast<uint2 *>(vlo + off) =
-                        make_uint2(*reinterpret_cast<const uint32_t *>(&l01), *reinterpret_cast<const uint32_t *>(&l23));
-                    }
+                // intermediate tile: hi and lo parts (128 rows x 64 columns each) by TMA; rows
+                // past the segment belong to no output of this tile and are masked at the store
+                if (lane == 0) {
+                    uint8_t *vhi = vbuf + vb * kExVBytes;
+                    const uint32_t vf = smem_u32(&ctl.vfull[vb]);
+                    mbar_arrive_expect_tx(vf, (uint32_t)kExVBytes);
+                    tma_load_2d(smem_u32(vhi), &p.tmap_vhi, 0, row0, vf);
+                    tma_load_2d(smem_u32(vhi + 16384), &p.tmap_vlo, 0, row0, vf);
                 }
-                fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&ctl.vfull[vb]));
                 ++vcount;
             }
             if (i >= kExStages && !mbar_wait(smem_u32(&ctl.empty[s]), ((i / kExStages) - 1) & 1, p.status)) {
@@ -492,9 +487,12 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         }
         // drain: every TMA issued by this CTA has landed before shared memory is released
         const int n = t1 - t0;
-        if (lane == 0)
+        if (lane == 0) {
             for (int i = max(0, n - kExStages); i < n; ++i)
                 mbar_wait(smem_u32(&ctl.full[i % kExStages]), (i / kExStages) & 1, p.status);
+            for (int c = max(0, vcount - 2); c < vcount; ++c)
+                mbar_wait(smem_u32(&ctl.vfull[c & 1]), (c >> 1) & 1, p.status);
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -667,7 +665,7 @@ int prefill_build_maps(lora_table *t)
 }
 
 int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y, int64_t ldy,
-                   int32_t y_off, float *v, int32_t ldv, cudaStream_t s)
+                   int32_t y_off, void *v, cudaStream_t s)
 {
     if (!prefill_supported(t)) return LORA_ERR_UNSUPPORTED;
     PrefillParams p;
@@ -683,8 +681,8 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
     p.h = t->h;
     p.o = t->o;
     p.n = t->n;
-    p.v = v;
-    p.ldv = ldv;
+    p.v_hi = static_cast<uint16_t *>(v);
+    p.v_lo = p.v_hi + (int64_t)seg->T * kMaxRankPF;
     p.y = y;
     p.ldy = ldy;
     p.y_off = y_off;
@@ -734,6 +732,9 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
         if (e != cudaSuccess) return LORA_ERR_CUDA;
     }
     // expand: persistent, one CTA per SM over all (128-token tile, 128-column tile) pairs
+    if ((rc = encode_sw128(&p.tmap_vhi, p.v_hi, kMaxRankPF, (uint64_t)seg->T, kMaxRankPF, kTileM)) != LORA_OK ||
+        (rc = encode_sw128(&p.tmap_vlo, p.v_lo, kMaxRankPF, (uint64_t)seg->T, kMaxRankPF, kTileM)) != LORA_OK)
+        return rc;
     rc = encode_sw128(&p.tmap_io, static_cast<uint8_t *>(y) + (int64_t)y_off * 2, (uint64_t)t->o, (uint64_t)seg->T,
                       (uint64_t)ldy, kTileM);
     if (rc != LORA_OK) return rc;
