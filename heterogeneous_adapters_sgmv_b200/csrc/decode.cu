@@ -26,8 +26,9 @@
 //    one keeps its own sum and exchanges nothing.  The three-stage form applies the adapter's
 //    Sigma_i (full or diagonal) to the summed intermediate here.
 //  * Expand: a thread owns two output columns (bf16) and takes the unit's tokens two at a time,
-//    sharing each B_i load; products are added in ascending k, one rounding (nearest-even) per
-//    output, coalesced 32-bit stores.  A per-token weight (merged ensembles) multiplies the
+//    sharing each B_i load; it walks its B rows from a rotated 16-byte chunk so a quarter warp
+//    hits distinct shared-memory banks; one rounding (nearest-even) per output, coalesced
+//    32-bit stores.  A per-token weight (merged ensembles) multiplies the
 //    scale.
 //  * A grouped launch carries up to four projections (tables, x, y slices); each unit then
 //    runs once per projection, back to back on the same cluster.
@@ -783,9 +784,18 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             const float sc = hdr.scale;
             const ProjParams &pj = p.pj[hdr.proj];
             const int c = tid * CPT;   // first column of this thread within the tile
+            // starting chunk of this thread's B rows (bf16: rows of 2 r bytes, two per thread)
+            int krot = 0;
+            if (CPT == 2 && (r % EPC) == 0) {
+                const int nchk = r / EPC;
+                if ((nchk & (nchk - 1)) == 0) {
+                    const int sh = r >= 32 ? 0 : (r == 16 ? 1 : 2);
+                    krot = ((tid >> sh) & (nchk - 1)) * EPC;
+                }
+            }
             if (c < len) {
                 // Two tokens per pass share each load of this thread's B rows; per output the
-                // products are still added in ascending k.
+                // products are added in one fixed order (the thread's rotated chunk order).
                 const uint8_t *brow = data + (size_t)c * r * ESZ;   // CPT consecutive rows of B
                 for (int l = 0; l < L; l += 2) {
                     const bool l2 = l + 1 < L;   // row l + 1 of vsum exists even when unused
@@ -794,7 +804,12 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
 #pragma unroll
                     for (int j = 0; j < CPT; ++j) acc0[j] = acc1[j] = 0.f;
                     if ((r % EPC) == 0) {
-                        for (int k = 0; k < r; k += EPC) {
+                        // Each thread starts its walk over the 16-byte chunks of its B rows at
+                        // a rotated chunk, so the lanes of a quarter warp read different bank
+                        // groups (rows of 2 r bytes would otherwise put them on one group).
+                        for (int kk = 0; kk < r; kk += EPC) {
+                            int k = kk + krot;
+                            if (k >= r) k -= r;
                             float v0[EPC], v1[EPC];
 #pragma unroll
                             for (int e = 0; e < EPC; e += 4) {
