@@ -542,3 +542,25 @@ def test_merged_loop_matches_grouped_products(delta_only):
     ref = oracle.lora_delta_merged(wl.dtype, p.x, p.y0, ids, w, A, B, p.scales)
     alt = brute.lora_delta_merged(wl.dtype, p.x, p.y0, ids, w, A, B, p.scales)
     assert np.abs(ref - alt).max() <= 1e-12 * max(np.abs(alt).max(), 1e-30)
+
+
+def test_next_row_generators_are_seeded_and_shaped():
+    """Sigma, cluster and ensemble draws: deterministic per seed, the stated shapes and laws."""
+    ranks = np.array([4, 8, 16, 64], dtype=np.int32)
+    s1 = workloads.draw_sigma(ranks, "full", seed=3)
+    s2 = workloads.draw_sigma(ranks, "full", seed=3)
+    assert all(np.array_equal(a, b) for a, b in zip(s1, s2))
+    assert [a.shape for a in s1] == [(4, 4), (8, 8), (16, 16), (64, 64)]
+    assert all(a.dtype == np.float32 for a in s1)
+    assert 0.8 / 64 < float(np.var(s1[3])) < 1.2 / 64   # variance 1/r at r = 64
+    d = workloads.draw_sigma(ranks, "diag", seed=3)
+    assert [a.shape for a in d] == [(4,), (8,), (16,), (64,)]
+    assert np.array_equal(workloads.jd_clusters(7, 3), np.array([0, 1, 2, 0, 1, 2, 0]))
+    ids = np.arange(50, dtype=np.int32) % 9
+    m1, w1 = workloads.draw_merge(ids, 9, 3, seed=5, empty=0.4)
+    m2, w2 = workloads.draw_merge(ids, 9, 3, seed=5, empty=0.4)
+    assert np.array_equal(m1, m2) and np.array_equal(w1, w2)
+    assert m1.shape == w1.shape == (50, 3) and np.array_equal(m1[:, 0], ids)
+    assert ((m1 >= -1) & (m1 < 9)).all() and (m1[:, 1:] == -1).any()
+    assert (w1[m1 < 0] == 0).all() and (w1[m1 >= 0] > 0).all()
+    assert np.allclose(w1.sum(axis=1), 1.0, atol=1e-6)
