@@ -155,10 +155,12 @@ int lora_expand(const lora_table *table, const lora_segments *seg, const float *
                 int32_t ldv, void *y, int64_t ldy, int32_t y_offset, void *stream);
 
 /* SGMV: shrink and expand for sorted segments, in place on the y slice.  Picks the path:
- * the fused cluster kernel (decode), or the tcgen05 tensor-core path when the hint
- * max_seg_len is long, perm is NULL and the table is bf16 (prefill).  ws may be NULL when
- * ws_bytes is 0 and the chosen path needs none; otherwise ws_bytes >=
- * lora_workspace_bytes(table, seg->T). */
+ * the fused cluster kernel (decode), or the tcgen05 tensor-core path (prefill) when the hint
+ * max_seg_len reaches the "prefill_min_seg_len" option (256), perm is NULL, the table is
+ * bf16 with every rank a multiple of 8 and at most 64, and it carries no Sigma.  The
+ * tcgen05 path keeps its intermediate (bf16 hi + lo) in the workspace; the fused kernel
+ * needs none, so ws may be NULL when ws_bytes is 0 and the chosen path needs none;
+ * otherwise ws_bytes >= lora_workspace_bytes(table, seg->T). */
 int lora_sgmv(const lora_table *table, const lora_segments *seg, const void *x, int64_t ldx,
               void *y, int64_t ldy, int32_t y_offset, void *ws, size_t ws_bytes, void *stream);
 
