@@ -240,8 +240,8 @@ def make_step(wl, L, grouped=False, merge=1):
     if grouped:
         if name != "many_adapter_qkvo":
             raise SystemExit("--grouped applies to many_adapter_qkvo only")
-        grp = [g for (_n, _h, _o, g) in wl.spec.projections]
-        src = [grp.index(g) for g in grp]   # the first projection reading the same x
+        xs_host = [q.x for q in wl.projections]
+        src = [next(j for j, xa in enumerate(xs_host) if xa is xh) for xh in xs_host]   # first reader of each x
 
         def step(c, s):
             st = c.seg_t

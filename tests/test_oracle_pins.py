@@ -564,3 +564,30 @@ def test_next_row_generators_are_seeded_and_shaped():
     assert ((m1 >= -1) & (m1 < 9)).all() and (m1[:, 1:] == -1).any()
     assert (w1[m1 < 0] == 0).all() and (w1[m1 >= 0] > 0).all()
     assert np.allclose(w1.sum(axis=1), 1.0, atol=1e-6)
+
+
+def test_byte_accounting_of_the_bench_variants():
+    """The bench's algorithmic bytes for its option variants, against hand counts: a grouped
+    launch reads the shared x once; Sigma adds 4 r^2 (full) or 4 r (diagonal) bytes per touched
+    adapter; shared cluster weights count once per touched cluster; one merged slot is the
+    plain call."""
+    wl = workloads.generate("many_adapter_qkvo", T=40, n=30, shapes=[("q", 64, 64, 0), ("k", 64, 16, 0),
+                                                                      ("v", 64, 16, 0), ("o", 64, 64, 1)])
+    e = 2
+    T_valid = int((wl.ids >= 0).sum())
+    base = accounting.workload_bytes(wl)
+    assert accounting.workload_bytes(wl, shared_x=True) == base - 2 * T_valid * 64 * e
+    d = accounting.distinct_adapters(wl.ids)
+    r = wl.projections[0].ranks
+    assert accounting.workload_bytes(wl, sigma="full") == base + 4 * 4 * int(sum(int(r[i]) ** 2 for i in d))
+    assert accounting.workload_bytes(wl, sigma="diag") == base + 4 * 4 * int(sum(int(r[i]) for i in d))
+    C = 7
+    leaders = np.unique(d % C)
+    w_all = sum(int(r[i]) * (q.h + q.o) * e for i in d for q in wl.projections)
+    w_cl = sum(int(r[i]) * (q.h + q.o) * e for i in leaders for q in wl.projections)
+    assert accounting.workload_bytes(wl, sigma="diag", clusters=C) == \
+        base - w_all + w_cl + 4 * 4 * int(sum(int(r[i]) for i in d))
+    one = wl.ids.reshape(-1, 1)
+    p = wl.projections[0]
+    assert accounting.merged_bytes(wl, one) == accounting.projection_bytes(
+        T_valid, p.h, p.o, (p.ranks[i] for i in d), e)

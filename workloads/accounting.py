@@ -48,7 +48,8 @@ def workload_bytes(wl, shared_x: bool = False, sigma: str = "none", clusters: in
     leaders = np.unique(d % clusters) if clusters > 0 else d
     tot = 0
     seen = set()
-    groups = [g for (_n, _h, _o, g) in wl.spec.projections] if shared_x else range(len(wl.projections))
+    # projections of one x group hold the same activation array
+    groups = [id(p.x) for p in wl.projections] if shared_x else range(len(wl.projections))
     for p, g in zip(wl.projections, groups):
         tot += projection_bytes(T_valid, p.h, p.o, (p.ranks[i] for i in leaders), e)
         if g in seen:
