@@ -74,6 +74,9 @@ def bind(path: str):
     lib.oracle_lora_delta_merged.argtypes = [ctypes.c_int, i64, i64, i64, P, i64, P, i64, i64, i32, P, P, i32,
                                              P, P, P, P, P, ctypes.c_int]
     lib.oracle_lora_delta_merged.restype = ctypes.c_int
+    lib.oracle_lora_base_delta.argtypes = [ctypes.c_int, i64, i64, i64, P, i64, P, i64, P, i64, i64, ctypes.c_int,
+                                           P, i32, P, P, P, P, P, ctypes.c_int]
+    lib.oracle_lora_base_delta.restype = ctypes.c_int
     lib.oracle_build_segments.argtypes = [i64, P, i32, P, P, P, P]
     lib.oracle_build_segments.restype = ctypes.c_int64
     lib.oracle_max_threads.argtypes = []
@@ -285,6 +288,40 @@ def lora_delta_merged(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray
     return out
 
 
+def lora_base_delta(dtype: str, x: np.ndarray, W: np.ndarray, y0: np.ndarray, ids: np.ndarray,
+                    A: Sequence[np.ndarray], B: Sequence[np.ndarray], scales: Sequence[float],
+                    accumulate: bool = True, y_offset: int = 0, o: Optional[int] = None,
+                    threads: int = 0) -> np.ndarray:
+    """Layer output with the frozen base weight W [o, h]: fp64 y_ref = (y0 if accumulate)
+    + W x[t] + s_i B_i (A_i x[t]) for i = ids[t] (id -1: no adapter term)."""
+    x = _check_store(x, dtype)
+    W = _check_store(W, dtype)
+    y0 = _check_store(y0, dtype)
+    T, h = x.shape
+    if o is None:
+        o = y0.shape[1] - y_offset
+    if W.shape[0] != o or W.shape[1] < h:
+        raise ValueError("W shape %s does not match h=%d o=%d" % (W.shape, h, o))
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    n = len(A)
+    As = [_check_store(a, dtype) for a in A]
+    Bs = [_check_store(b, dtype) for b in B]
+    ranks = np.array([a.shape[0] for a in As], dtype=np.int32)
+    for a, b, r in zip(As, Bs, ranks):
+        if a.shape != (r, h) or b.shape != (o, r):
+            raise ValueError("adapter shapes %s / %s do not match h=%d o=%d" % (a.shape, b.shape, h, o))
+    Ap = (ctypes.c_void_p * max(n, 1))(*[_ptr(a) for a in As])
+    Bp = (ctypes.c_void_p * max(n, 1))(*[_ptr(b) for b in Bs])
+    sc = np.ascontiguousarray(np.asarray(scales, dtype=np.float32).astype(np.float64))
+    out = np.empty((T, o), dtype=np.float64)
+    rc = _load().oracle_lora_base_delta(_dtype_code(dtype), T, h, o, _ptr(x), x.shape[1], _ptr(W), W.shape[1],
+                                        _ptr(y0), y0.shape[1], y_offset, 1 if accumulate else 0, _ptr(ids), n,
+                                        Ap, Bp, _ptr(ranks), _ptr(sc), _ptr(out), threads)
+    if rc != 0:
+        raise OracleError("adapter id out of range")
+    return out
+
+
 def build_segments(ids: np.ndarray, n_adapters: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Stable counting sort by adapter id -> (perm[valid], seg_ptr[S+1], seg_adapter[S])."""
     ids = np.ascontiguousarray(ids, dtype=np.int32)
@@ -299,6 +336,16 @@ def build_segments(ids: np.ndarray, n_adapters: int) -> Tuple[np.ndarray, np.nda
         raise OracleError("adapter id out of range")
     S = int(ns[0])
     return perm[:valid].copy(), seg_ptr[:S + 1].copy(), seg_adapter[:S].copy()
+
+
+def base_reference(wl, W: np.ndarray, accumulate: bool = True, proj_index: int = 0,
+                   threads: int = 0) -> np.ndarray:
+    """Oracle layer output (fp64, unrounded) of one projection with the base weight W."""
+    p = wl.projections[proj_index]
+    A = [p.A(i) for i in range(wl.n)]
+    B = [p.B(i) for i in range(wl.n)]
+    return lora_base_delta(wl.dtype, p.x, W, p.y0, wl.ids, A, B, p.scales, accumulate=accumulate,
+                           threads=threads)
 
 
 def workload_reference(wl, proj_index: int = 0, threads: int = 0) -> np.ndarray:

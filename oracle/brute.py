@@ -70,3 +70,16 @@ def lora_delta_merged(dtype: str, x: np.ndarray, y0: np.ndarray, ids: np.ndarray
             d = (xd[rows] @ to_float64(A[i], dtype).T) @ to_float64(B[i], dtype).T
             out[rows] += (w[rows, j] * float(np.float32(scales[i])))[:, None] * d
     return out
+
+
+def lora_base_delta(dtype: str, x: np.ndarray, W: np.ndarray, y0: np.ndarray, ids: np.ndarray,
+                    A: Sequence[np.ndarray], B: Sequence[np.ndarray], scales: Sequence[float],
+                    accumulate: bool = True) -> np.ndarray:
+    """Layer output with the frozen base weight: one library product x @ W^T for all tokens,
+    then the adapter terms grouped by adapter."""
+    xd = to_float64(x, dtype)
+    base = xd @ to_float64(W, dtype)[:, :xd.shape[1]].T
+    y = to_float64(y0, dtype) if accumulate else np.zeros_like(base)
+    zero = np.zeros_like(y0)
+    delta = lora_delta(dtype, x, zero, ids, A, B, scales)
+    return y + base + delta

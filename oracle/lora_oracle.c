@@ -428,3 +428,79 @@ int64_t oracle_build_segments(int64_t T, const int32_t *ids, int32_t n_adapters,
     free(next);
     return pos;
 }
+
+/*
+ * Layer output with the frozen base weight: the "TGI Multi-LoRA" page ("Technical
+ * Foundation: LoRA") keeps the pretrained weight W frozen and adds the adapter's low-rank
+ * term, so one layer computes W x + s_i B_i A_i x; the "predibase/lorax" repository page
+ * describes the adapter update as part of a single forward pass of the layer.
+ *
+ *   y_ref[t, n] = (accumulate ? y0[t, y_offset + n] : 0)
+ *               + sum_j W[n, j] * x[t, j]                          (base product)
+ *               + s_i * sum_k B_i[n, k] * v[k],  v[k] = sum_j x[t, j] * A_i[k, j]
+ *
+ * for i = ids[t]; a token with id -1 gets the first two terms only.  W is [o, ldw] row-major
+ * (an output feature per row, the first h columns used), the orientation of a linear
+ * layer's weight.  Terms are added in the order written, in fp64, unrounded.
+ * Returns 0, or -1 if an id is out of range (nothing is written then).
+ */
+int oracle_lora_base_delta(int dtype, int64_t T, int64_t h, int64_t o,
+                           const void *x, int64_t ldx,
+                           const void *W, int64_t ldw,
+                           const void *y0, int64_t ldy, int64_t y_offset, int accumulate,
+                           const int32_t *ids, int32_t n_adapters,
+                           const void *const *A, const void *const *B,
+                           const int32_t *ranks, const double *scales,
+                           double *y_ref, int n_threads)
+{
+    if (!ids_valid(T, ids, n_adapters))
+        return -1;
+    set_threads(n_threads);
+#pragma omp parallel
+    {
+        double *xr = (double *)malloc((size_t)h * sizeof(double));
+        double *u = NULL;
+        int32_t ucap = 0;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < T; ++t) {
+            double *yr = y_ref + t * o;
+            for (int64_t j = 0; j < h; ++j)
+                xr[j] = widen(x, dtype, t * ldx + j);
+            for (int64_t n = 0; n < o; ++n)
+                yr[n] = accumulate ? widen(y0, dtype, t * ldy + y_offset + n) : 0.0;
+            /* base product: y += W x */
+            for (int64_t n = 0; n < o; ++n) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < h; ++j)
+                    acc += widen(W, dtype, n * ldw + j) * xr[j];
+                yr[n] += acc;
+            }
+            int32_t i = ids[t];
+            if (i < 0)
+                continue;
+            const int32_t ri = ranks[i];
+            if (ri > ucap) {
+                free(u);
+                u = (double *)malloc((size_t)ri * sizeof(double));
+                ucap = ri;
+            }
+            /* adapter shrink: u = A_i x  (scale 1) */
+            for (int32_t m = 0; m < ri; ++m) {
+                double su = 0.0;
+                for (int64_t j = 0; j < h; ++j)
+                    su += xr[j] * widen(A[i], dtype, (int64_t)m * h + j);
+                u[m] = su;
+            }
+            /* adapter expand: y += s_i * B_i u */
+            for (int64_t n = 0; n < o; ++n) {
+                double sd = 0.0;
+                for (int32_t m = 0; m < ri; ++m)
+                    sd += widen(B[i], dtype, n * ri + m) * u[m];
+                yr[n] += scales[i] * sd;
+            }
+        }
+        free(u);
+        free(xr);
+    }
+    return 0;
+}

@@ -53,6 +53,17 @@ MUTATIONS = {
     "sigma_diag_skipped": ("w[k] = (double)S[k] * u[k];", "w[k] = u[k];"),
     "sigma_scale_dropped": ("yr[n] += scales[i] * acc;\n            }\n        }\n        free(u);",
                             "yr[n] += acc;\n            }\n        }\n        free(u);"),
+    "base_W_transposed": ("acc += widen(W, dtype, n * ldw + j) * xr[j];",
+                          "acc += widen(W, dtype, j * o + n) * xr[j];"),
+    "base_A_transposed": ("su += xr[j] * widen(A[i], dtype, (int64_t)m * h + j);",
+                          "su += xr[j] * widen(A[i], dtype, (int64_t)j * ri + m);"),
+    "base_delta_scale_dropped": ("yr[n] += scales[i] * sd;", "yr[n] += sd;"),
+    "base_term_dropped": ("                yr[n] += acc;\n            }\n            int32_t i = ids[t];",
+                          "                (void)acc;\n            }\n            int32_t i = ids[t];"),
+    "base_accumulate_ignored": ("yr[n] = accumulate ? widen(y0, dtype, t * ldy + y_offset + n) : 0.0;",
+                                "yr[n] = widen(y0, dtype, t * ldy + y_offset + n);"),
+    "base_skipped_without_adapter": ("/* base product: y += W x */\n            for (int64_t n = 0; n < o; ++n) {",
+                                     "/* base product: y += W x */\n            for (int64_t n = 0; n < o && ids[t] >= 0; ++n) {"),
 }
 
 PIN_TESTS = [
@@ -76,6 +87,11 @@ PIN_TESTS = [
     pins.test_merged_slot_order_and_duplicate_slots,
     lambda: [pins.test_sigma_loop_matches_grouped_products(k, d) for k in ("full", "diag") for d in (False, True)],
     lambda: [pins.test_merged_loop_matches_grouped_products(d) for d in (False, True)],
+    pins.test_base_with_zero_weight_is_the_delta,
+    pins.test_base_single_adapter_equals_merged_weight,
+    pins.test_base_rows_without_adapter_and_accumulate_flag,
+    lambda: [pins.test_base_selection_matrix_closed_form(h, o) for h, o in ((24, 16), (16, 40))],
+    pins.test_base_linear_in_weight_and_matches_grouped_products,
 ]
 
 

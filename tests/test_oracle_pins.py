@@ -591,3 +591,97 @@ def test_byte_accounting_of_the_bench_variants():
     p = wl.projections[0]
     assert accounting.merged_bytes(wl, one) == accounting.projection_bytes(
         T_valid, p.h, p.o, (p.ranks[i] for i in d), e)
+
+
+# ------------------------------------------------------------------ fused base product (layer output)
+# "TGI Multi-LoRA" page, "Technical Foundation: LoRA": the frozen base weight's product plus
+# the adapter's low-rank term; "predibase/lorax" repository page: one forward pass.
+
+def _base_case(seed=3, T=12, h=96, o=80, n=3, ranks=(8, 16, 8), dtype="bf16", minus_one=True):
+    wl = workloads.generate("multirank_decode", T=T, n=n, shapes=[("q", h, o, 0)], ranks=ranks, seed=seed)
+    ids = wl.ids.copy()
+    if minus_one:
+        ids[::4] = -1
+    W = workloads.draw_base_weight(o, h, seed=seed + 1, dtype=dtype)
+    return wl, ids, W
+
+
+def test_base_with_zero_weight_is_the_delta():
+    """W = 0: the layer output is exactly the delta form y0 + s_i B_i A_i x."""
+    wl, ids, W = _base_case()
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    zero = np.zeros_like(W)
+    got = oracle.lora_base_delta(wl.dtype, p.x, zero, p.y0, ids, A, B, p.scales)
+    want = oracle.lora_delta(wl.dtype, p.x, p.y0, ids, A, B, p.scales)
+    assert np.array_equal(got, want)
+
+
+def test_base_single_adapter_equals_merged_weight():
+    """Every token on adapter 0: y = y0 + x (W + s B A)^T with the merged weight formed
+    first, the LoRA merge of the definition."""
+    wl, _ids, W = _base_case(minus_one=False)
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    ids = np.zeros(wl.T, np.int32)
+    got = oracle.lora_base_delta(wl.dtype, p.x, W, p.y0, ids, A, B, p.scales)
+    Wm = to_float64(W, wl.dtype) + float(p.scales[0]) * (to_float64(B[0], wl.dtype) @ to_float64(A[0], wl.dtype))
+    want = to_float64(p.y0, wl.dtype) + to_float64(p.x, wl.dtype) @ Wm.T
+    assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max()
+
+
+def test_base_rows_without_adapter_and_accumulate_flag():
+    """Id -1 rows get y0 + x W^T only; without accumulate the result ignores y0 and equals
+    the accumulated result minus y0."""
+    wl, ids, W = _base_case()
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    ids[:] = -1
+    got = oracle.lora_base_delta(wl.dtype, p.x, W, p.y0, ids, A, B, p.scales)
+    want = to_float64(p.y0, wl.dtype) + to_float64(p.x, wl.dtype) @ to_float64(W, wl.dtype).T
+    assert np.abs(got - want).max() <= 1e-12 * np.abs(want).max()
+    wl, ids, W = _base_case()
+    garbage = workloads.generate("multirank_decode", T=wl.T, n=wl.n, shapes=[("q", 96, 80, 0)],
+                                 ranks=(8, 16, 8), seed=99).projections[0].y0
+    fresh = oracle.lora_base_delta(wl.dtype, p.x, W, garbage, ids, A, B, p.scales, accumulate=False)
+    zero_y0 = oracle.lora_base_delta(wl.dtype, p.x, W, np.zeros_like(p.y0), ids, A, B, p.scales)
+    acc = oracle.lora_base_delta(wl.dtype, p.x, W, p.y0, ids, A, B, p.scales)
+    assert np.array_equal(fresh, zero_y0)
+    assert np.abs((acc - to_float64(p.y0, wl.dtype)) - fresh).max() <= 1e-12 * np.abs(fresh).max()
+
+
+@pytest.mark.parametrize("h,o", [(24, 16), (16, 40)])
+def test_base_selection_matrix_closed_form(h, o):
+    """W selects coordinate sel[n] of x (W[n, sel[n]] = 1) and the adapter terms vanish:
+    y = y0 + x[:, sel] exactly.  A transposed W (non-square) selects other coordinates."""
+    rng = np.random.default_rng(5)
+    T = 6
+    sel = rng.integers(0, h, size=o)
+    W = np.zeros((o, h), np.float32)
+    W[np.arange(o), sel] = 1
+    x = rng.integers(-8, 9, size=(T, h)).astype(np.float32)
+    y0 = rng.integers(-8, 9, size=(T, o)).astype(np.float32)
+    A = [np.ones((8, h), np.float32)]
+    B = [np.zeros((o, 8), np.float32)]
+    ids = np.zeros(T, np.int32)
+    got = oracle.lora_base_delta("bf16", _int_store(x, "bf16"), _int_store(W, "bf16"), _int_store(y0, "bf16"), ids,
+                                 [_int_store(a, "bf16") for a in A], [_int_store(b, "bf16") for b in B], [2.0])
+    assert np.array_equal(got, y0.astype(np.float64) + x[:, sel].astype(np.float64))
+
+
+def test_base_linear_in_weight_and_matches_grouped_products():
+    """Doubling W doubles the base term exactly (power of two); the loop agrees with numpy
+    (one library product for the base term, grouped products for the adapters)."""
+    wl, ids, W = _base_case(T=20, h=128, o=96, n=4, ranks=(8, 16, 32, 8))
+    p = wl.projections[0]
+    A, B = _adapters(p, wl.n)
+    y0z = np.zeros_like(p.y0)
+    Bz = [np.zeros_like(b) for b in B]
+    one = oracle.lora_base_delta(wl.dtype, p.x, W, y0z, ids, A, Bz, p.scales)
+    W2 = f32_to_bf16_bits(2 * bf16_bits_to_f32(W))
+    two = oracle.lora_base_delta(wl.dtype, p.x, W2, y0z, ids, A, Bz, p.scales)
+    assert np.array_equal(two, 2 * one)
+    for acc in (True, False):
+        got = oracle.lora_base_delta(wl.dtype, p.x, W, p.y0, ids, A, B, p.scales, accumulate=acc)
+        alt = brute.lora_base_delta(wl.dtype, p.x, W, p.y0, ids, A, B, p.scales, accumulate=acc)
+        assert np.abs(got - alt).max() <= 1e-12 * np.abs(alt).max()

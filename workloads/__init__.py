@@ -306,3 +306,25 @@ def draw_merge(ids: np.ndarray, n: int, K: int, seed: int, empty: float = 0.0):
     tot = w.sum(axis=1, keepdims=True)
     w = np.where(tot > 0, w / np.where(tot > 0, tot, 1.0), 0.0)
     return out, w.astype(np.float32)
+
+
+def sweep_ids(T: int, n: int, distinct: int, seed: int) -> np.ndarray:
+    """Ids of a batch of T tokens that touch exactly ``distinct`` adapters out of n (distinct
+    <= min(T, n)): a seeded random subset of adapters, each carrying floor(T/distinct) or
+    ceil(T/distinct) tokens, in a seeded random token order.  Used to vary the number of
+    distinct adapters at a fixed batch size."""
+    if not 1 <= distinct <= min(T, n):
+        raise ValueError("distinct must lie in [1, min(T, n)]")
+    rng = np.random.default_rng(seed)
+    chosen = rng.choice(n, size=distinct, replace=False)
+    ids = np.resize(chosen, T)          # every chosen adapter at least once
+    rng.shuffle(ids)
+    return np.ascontiguousarray(ids, dtype=np.int32)
+
+
+def draw_base_weight(o: int, h: int, seed: int, dtype: str = "bf16", reading: str = "variance") -> np.ndarray:
+    """Seeded frozen base weight W [o, h] (a linear layer's orientation) for the fused layer
+    output: entries N(0, 1/h), so x W^T keeps the unit scale of x, drawn in fp64 and rounded
+    to fp32, then to bf16."""
+    rng = np.random.default_rng(seed)
+    return _normal(rng, (o, h), 1.0 / h, reading, dtype)
