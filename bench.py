@@ -2,16 +2,22 @@
 """Throughput of the heterogeneous-batch LoRA delta on B200.
 
 One step = one pass of the hot path over one batch of synthetic, seeded inputs.  The default
-workload is the decode form: a q_proj-shaped layer (4096 -> 4096), 32 rank-16 bf16 adapters,
-64 tokens with uniform per-token adapter ids, scale 2, run through ``lora_bgmv`` (per-token
-ids grouped on the device, one fused launch).  Other workloads: ``--workload``.
+workload is the largest one-GPU configuration: an up_proj-shaped layer (4096 -> 14336), 8
+contiguous segments of 512 tokens each with its own rank-64 bf16 adapter, scale 0.5, run
+through ``lora_sgmv`` (the tcgen05 path).  Other workloads: ``--workload``.  The same JSON line
+carries, under ``secondary``, the decode-form workloads (per-token ids on 4096 -> 4096,
+multi-rank, many adapters over q/k/v/o), each timed the same way with its own roofline, and
+under ``adapter_sweep`` the throughput as the number of distinct adapters in a 256-token batch
+grows from 1 to 256.
 
 Timing: the input set (adapter weights, x, y, ids) is replicated into C copies whose total
 exceeds 4x the L2 size, and consecutive steps rotate through the copies, so every step reads
-its weights from HBM.  Steps are captured into a CUDA graph of C calls and replayed; the timed
-region is exactly K steps between a barrier + synchronize on both sides, timed with CUDA
-events on the launching stream, max over ranks.  With ``torchrun`` each rank runs its own
-independent batches (the path shards by tokens with no exchange): weak scaling.
+its weights from HBM.  Steps are captured into CUDA graphs (all C copies, and the first K % C),
+each replayed once before timing.  The timed region is exactly K steps, bracketed by CUDA
+events on the launching stream; it is repeated, with a 256 MB buffer written before each
+repetition, and the median repetition is reported (max over ranks; a barrier and a synchronize
+on both sides of the timed repetitions).  With ``torchrun`` each rank runs its own independent
+batches (the path shards by tokens with no exchange): weak scaling.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead.
 """
@@ -55,11 +61,13 @@ def parse():
     ap.add_argument("--steps", type=int, default=0, help="timed steps (0: about one second of work)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode_bgmv", choices=list(workloads.WORKLOAD_NAMES))
+    ap.add_argument("--workload", default="prefill_sgmv", choices=list(workloads.WORKLOAD_NAMES))
     ap.add_argument("--copies", type=int, default=0, help="input copies rotated across steps (0: auto)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--e2e-steps", type=int, default=-1, help="end-to-end steps (-1: about 1.5 s; 0: skip)")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the decode-form lines and the distinct-adapter sweep")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying a graph")
     ap.add_argument("--sigma", default="none", choices=["none", "full", "diag"],
                     help="three-stage (compressed) form: a per-adapter Sigma_i between the A and B steps")
@@ -115,7 +123,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "--id=%s" % gpu_id, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
@@ -274,6 +282,213 @@ def make_step(wl, L, grouped=False, merge=1):
     raise ValueError(name)
 
 
+class Timer:
+    """Times exactly K steps of a workload through CUDA graphs of its rotating input copies.
+
+    Graphs: one of all C copies (replayed K // C times) and one of the first K % C copies;
+    both are replayed once before any timing, so no first-replay upload lands in a timed
+    region.  The K-step region is repeated `reps` times; before each repetition a 256 MB
+    buffer is written (outside the timed region) so no repetition starts with its inputs in
+    L2.  Each repetition is bracketed by CUDA events on the launching stream; the median
+    repetition is reported."""
+
+    FLUSH_BYTES = 256 * 1024 * 1024
+
+    def __init__(self, torch, copies, step, K, no_graph=False):
+        self.torch, self.copies, self.step, self.K = torch, copies, step, K
+        self.no_graph = no_graph
+        self.stream = torch.cuda.Stream()
+        self.sh = int(self.stream.cuda_stream)
+        self.flush_buf = torch.empty(self.FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.g_full = self.g_rem = None
+
+    def warm(self, W):
+        torch, C = self.torch, len(self.copies)
+        with torch.cuda.stream(self.stream):
+            for i in range(W):
+                self.step(self.copies[i % C], self.sh)
+        torch.cuda.synchronize()
+        if self.no_graph:
+            return
+        K = self.K
+        if K >= C:
+            self.g_full = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g_full, stream=self.stream):
+                for i in range(C):
+                    self.step(self.copies[i], int(torch.cuda.current_stream().cuda_stream))
+        if K % C:
+            self.g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g_rem, stream=self.stream):
+                for i in range(K % C):
+                    self.step(self.copies[i], int(torch.cuda.current_stream().cuda_stream))
+        with torch.cuda.stream(self.stream):
+            for g in (self.g_full, self.g_rem):
+                if g is not None:
+                    g.replay()
+        torch.cuda.synchronize()
+
+    def _region(self):
+        C, K = len(self.copies), self.K
+        if self.no_graph:
+            for i in range(K):
+                self.step(self.copies[i % C], self.sh)
+            return
+        for _ in range(K // C):
+            self.g_full.replay()
+        if self.g_rem is not None:
+            self.g_rem.replay()
+
+    def run(self, reps):
+        """Returns the per-repetition region times (ms) of `reps` repetitions."""
+        torch = self.torch
+        evs = []
+        with torch.cuda.stream(self.stream):
+            for i in range(reps):
+                self.flush_buf.fill_(i & 0xFF)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(self.stream)
+                self._region()
+                e1.record(self.stream)
+                evs.append((e0, e1))
+        torch.cuda.synchronize()
+        return [float(a.elapsed_time(b)) for a, b in evs]
+
+    def reps_for(self, seconds):
+        """Repetitions that fill about `seconds` of GPU time (at least 5, at most 2000)."""
+        t = self.run(2)
+        per = max(1e-6, min(t) / 1e3 + 50e-6)
+        return int(max(5, min(2000, seconds / per)))
+
+    def release(self):
+        self.g_full = self.g_rem = None
+        self.flush_buf = None
+
+
+def roofline_of(bytes_step, ms_step, launches_per_step, kname, traffic):
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    one = launches_per_step == 1
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+            else "fallback 6.65 TB/s",
+            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+            "algorithmic_bytes_per_launch": bytes_step if one else None,
+            "algorithmic_bytes_per_step": bytes_step,
+            "kernel": kname,
+            "kernel_ms_per_launch": round(ms_step, 6) if one else None,
+            "basis": "step time (one launch per step)" if one else
+            "whole step (%d launches): a lower bound on the dominant kernel's own rate" % launches_per_step}
+
+
+def make_copies(wl, L, torch, args, plain=False):
+    """C replicas of the inputs, C chosen so that together they exceed 4x the L2 size (at
+    least 2).  `plain` ignores the three-stage / merged options (secondary lines)."""
+    kw = {} if plain else dict(sigma=args.sigma, clusters=args.jd_clusters, merge=args.merge)
+    first = Copy(wl, L, torch, **kw)
+    per = first.nbytes()
+    C = args.copies or max(2, min(256, -(-4 * L2_BYTES // per)))
+    return [first] + [Copy(wl, L, torch, **kw) for _ in range(C - 1)], per
+
+
+def free_copies(torch, copies):
+    for c in copies:
+        for t in c.tables:
+            t.close()
+    copies.clear()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def timed_workload(args, L, torch, wl, grouped, seconds, dist, K=None):
+    """Median per-step time of one workload over repeated K-step regions (secondary lines)."""
+    step, launches, kname = make_step(wl, L, grouped, 1)
+    copies, per = make_copies(wl, L, torch, args, plain=True)
+    C = len(copies)
+    K = K or C * max(1, -(-32 // C))
+    tm = Timer(torch, copies, step, K, args.no_graph)
+    tm.warm(max(args.warmup, 3))
+    reps = tm.reps_for(seconds)
+    if dist:
+        dist.barrier()
+    times = tm.run(reps)
+    ms = max_over_ranks(float(np.median(times)), dist, "cuda") / K
+    tm.release()
+    free_copies(torch, copies)
+    return ms, launches, kname, C, per, K, reps
+
+
+def secondary_lines(args, L, torch, dist, world):
+    """The decode-form workloads, each timed on its own with its own roofline."""
+    out = []
+    for name, grouped in (("decode_bgmv", False), ("multirank_decode", False), ("many_adapter_qkvo", True)):
+        if name == args.workload and grouped == args.grouped:
+            continue
+        wl = workloads.generate(name, seed=rank_seed(name, int(os.environ.get("RANK", "0"))))
+        ms, launches, kname, C, per, K, reps = timed_workload(args, L, torch, wl, grouped, 0.4, dist)
+        b = accounting.workload_bytes(wl, shared_x=grouped)
+        traffic = profile_traffic(name) if not grouped else None
+        out.append({"workload": "%s: %s" % (name, workload_description(name, grouped)),
+                    "tokens_per_step": wl.T, "value": round(job_throughput(world, wl.T, 1, ms), 1),
+                    "unit": UNIT, "ms_per_step": round(ms, 6), "steps": K, "repetitions": reps,
+                    "algorithmic_bytes_per_step": b,
+                    "l2": "rotating %d input copies, %.0f MB in total; 256 MB written between repetitions" % (
+                        C, C * per / 1e6),
+                    "roofline": roofline_of(b, ms, launches, kname, traffic)})
+    return out
+
+
+def adapter_sweep(args, L, torch, dist, world):
+    """Distinct adapters touched per batch (1 .. 256) at the decode layer shape: 4096 -> 4096,
+    rank 16, 256 tokens, a table of 256 adapters, one lora_bgmv per step."""
+    from workloads.device import upload_projection
+    T, n = 256, 256
+    wl = workloads.generate("decode_bgmv", T=T, n=n, seed=rank_seed("decode_bgmv", 0) + 5000)
+    p = wl.projections[0]
+    e = accounting.ELEM_BYTES[wl.dtype]
+    per = sum(a.nbytes for a in (p.A_flat, p.B_flat, p.x, p.y0))
+    C = max(2, -(-4 * L2_BYTES // per))
+    dev = []
+    for _ in range(C):
+        d = upload_projection(p, wl.dtype)
+        t = L.AdapterTable(d.A_ptrs, d.B_ptrs, d.ranks, d.scales, p.h, p.o, L.LORA_BF16, keep=d)
+        dev.append((d, t))
+    points = []
+    for D in (1, 4, 16, 64, 256):
+        ids_np = workloads.sweep_ids(T, n, D, seed=wl.seed + D)
+        ids = torch.from_numpy(ids_np).cuda()
+
+        def step(c, s, ids=ids):
+            d, t = c
+            L.lora_bgmv(t.handle, ids, T, d.x, d.h, d.y0, d.o, 0, None, 0, s)
+        K = C * max(1, -(-32 // C))
+        tm = Timer(torch, dev, step, K, args.no_graph)
+        tm.warm(max(args.warmup, 3))
+        reps = tm.reps_for(0.25)
+        if dist:
+            dist.barrier()
+        ms = max_over_ranks(float(np.median(tm.run(reps))), dist, "cuda") / K
+        tm.release()
+        b = accounting.projection_bytes(T, p.h, p.o, (p.ranks[i] for i in np.unique(ids_np)), e)
+        peak, _ = measured_peaks()
+        gbs = b / (ms / 1e3) / 1e9
+        points.append({"distinct_adapters": D, "value": round(job_throughput(world, T, 1, ms), 1),
+                       "ms_per_step": round(ms, 6), "algorithmic_bytes_per_step": b,
+                       "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)})
+    for d, t in dev:
+        t.close()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return {"shape": "4096 -> 4096, rank 16 bf16, 256 tokens, table of 256 adapters, lora_bgmv; "
+                     "rotating %d input copies" % C, "unit": UNIT, "points": points}
+
+
+def workload_description(name, grouped):
+    d = DESCRIPTIONS[name]
+    return d.replace("4 x lora_sgmv", "one lora_sgmv_grouped, q/k/v sharing x") if grouped else d
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import heterogeneous_adapters_sgmv_b200 as L
@@ -294,54 +509,21 @@ def run_ours(args, rank, world, local_rank):
     flops_step = accounting.workload_flops(wl)
     distinct = int(accounting.distinct_adapters(wl.ids).size)
 
-    first = Copy(wl, L, torch, args.sigma, args.jd_clusters, args.merge)
-    ws_bytes = first.nbytes()
-    C = args.copies or max(1, min(256, -(-4 * L2_BYTES // ws_bytes)))
-    copies = [first] + [Copy(wl, L, torch, args.sigma, args.jd_clusters, args.merge) for _ in range(C - 1)]
+    copies, ws_bytes = make_copies(wl, L, torch, args)
+    C = len(copies)
     torch.cuda.synchronize()
-
-    stream = torch.cuda.Stream()
-    sh = int(stream.cuda_stream)
     K = args.steps
-    if K <= 0:
-        # about one second of work, from a short eager probe
-        with torch.cuda.stream(stream):
-            for i in range(3 * C):
-                step(copies[i % C], sh)
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        with torch.cuda.stream(stream):
-            for i in range(2 * C):
-                step(copies[i % C], sh)
-        torch.cuda.synchronize()
-        per = (time.perf_counter() - t0) / (2 * C)
-        K = int(max(1000, min(2_000_000, 1.0 / max(per, 1e-7) * 3)))   # graph replay is faster than eager
-        K = max(C, K // C * C)
+    if K <= 0:   # about 20 ms of work per repetition, a whole number of copy rotations
+        tm0 = Timer(torch, copies, step, C, args.no_graph)
+        tm0.warm(3)
+        per = min(tm0.run(3)) / C
+        tm0.release()
+        K = max(C, int(20.0 / max(per, 1e-4)) // C * C)
     W = max(args.warmup, 3)
 
-    # warm-up (eager) then capture one graph of C steps (and one of K % C steps)
-    with torch.cuda.stream(stream):
-        for i in range(W):
-            step(copies[i % C], sh)
-    torch.cuda.synchronize()
-    graphs = []
-    if not args.no_graph:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(C):
-                step(copies[i], int(torch.cuda.current_stream().cuda_stream))
-        graphs.append(g)
-        rem = K % C
-        g2 = None
-        if rem:
-            g2 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g2, stream=stream):
-                for i in range(rem):
-                    step(copies[i], int(torch.cuda.current_stream().cuda_stream))
-        for _ in range(2):
-            with torch.cuda.stream(stream):
-                g.replay()
-        torch.cuda.synchronize()
+    tm = Timer(torch, copies, step, K, args.no_graph)
+    tm.warm(W)
+    reps = tm.reps_for(1.0)
 
     gpu_id = torch.cuda.get_device_properties(local_rank).uuid
     gpu_id = "GPU-%s" % gpu_id if not str(gpu_id).startswith("GPU-") else str(gpu_id)
@@ -350,50 +532,23 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     sampler = ClockSampler(gpu_id)
     time.sleep(0.3)   # let the sampler start before the timed region
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        if args.no_graph:
-            for i in range(K):
-                step(copies[i % C], sh)
-        else:
-            for _ in range(K // C):
-                graphs[0].replay()
-            if K % C:
-                g2.replay()
-        ev1.record(stream)
+    times = tm.run(reps)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if dist:
         dist.barrier(device_ids=[local_rank])
-    ms = max_over_ranks(float(ev0.elapsed_time(ev1)), dist, "cuda")
+    ms = max_over_ranks(float(np.median(times)), dist, "cuda")
     ms_step = ms / K
     value = job_throughput(world, T, K, ms)
+    tm.release()
 
-    # roofline of the dominant kernel: per launch (for one-launch steps the launch is the step)
-    peak, peak_kind = measured_peaks()
-    kernel_ms = ms_step if launches_per_step == 1 else None
-    achieved = bytes_step / (ms_step / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4),
-                "traffic": profile_traffic(args.workload) if not (args.grouped or args.sigma != "none" or
-                                                                   args.merge > 1) else None,
-                "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind if peak_kind == "measured"
-                else "fallback 6.65 TB/s",
-                "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                "algorithmic_bytes_per_launch": bytes_step if launches_per_step == 1 else None,
-                "algorithmic_bytes_per_step": bytes_step,
-                "kernel": kname,
-                "kernel_ms_per_launch": round(kernel_ms, 6) if kernel_ms else None,
-                "basis": "step time (one launch per step)" if launches_per_step == 1 else
-                "whole step (all launches)"}
+    traffic = profile_traffic(args.workload) if not (args.grouped or args.sigma != "none" or args.merge > 1) else None
+    roofline = roofline_of(bytes_step, ms_step, launches_per_step, kname, traffic)
 
     # end to end through the C ABI with host buffers: H2D inputs, the call, D2H of y
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps != 0:
         c = copies[0]
-        d = c.projs[0]
         hx = [torch.empty_like(p.x, device="cpu").pin_memory() for p in c.projs]
         hy = [torch.empty_like(p.y0, device="cpu").pin_memory() for p in c.projs]
         hout = [torch.empty_like(p.y0, device="cpu").pin_memory() for p in c.projs]
@@ -403,7 +558,8 @@ def run_ours(args, rank, world, local_rank):
             hy[i].copy_(p.y0)
         h2d = sum(t.numel() * t.element_size() for t in hx + hy) + hids.numel() * 4
         d2h = sum(t.numel() * t.element_size() for t in hout)
-        Ke = args.e2e_steps
+        stream = tm.stream
+        sh = tm.sh
 
         def e2e_step():
             c.ids.copy_(hids, non_blocking=True)
@@ -418,6 +574,11 @@ def run_ours(args, rank, world, local_rank):
             for _ in range(W):
                 e2e_step()
         torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            e2e_step()
+        torch.cuda.synchronize()
+        Ke = args.e2e_steps if args.e2e_steps > 0 else int(max(20, min(5000, 1.5 / max(time.perf_counter() - t0, 1e-5))))
         if dist:
             dist.barrier(device_ids=[local_rank])
         e0 = torch.cuda.Event(enable_timing=True)
@@ -432,6 +593,11 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": round(job_throughput(world, T, Ke, ems), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": Ke, "ms_per_step": round(ems / Ke, 6),
                "path": "pinned host -> cudaMemcpyAsync -> C-ABI call -> cudaMemcpyAsync -> pinned host"}
+    pdl = bool(L.lora_get_option("pdl"))
+    free_copies(torch, copies)
+
+    secondary = secondary_lines(args, L, torch, dist, world) if not args.no_secondary else None
+    sweep = adapter_sweep(args, L, torch, dist, world) if not args.no_secondary else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -444,14 +610,14 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_step, 6), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": codes[wl.dtype], "data": "synthetic (seeded; random adapter weights and activations)",
-        "config": {"workload": "%s: %s" % (args.workload, DESCRIPTIONS[args.workload] if not args.grouped else
-                                           DESCRIPTIONS[args.workload].replace(
-                                               "4 x lora_sgmv", "one lora_sgmv_grouped, q/k/v sharing x")),
+        "config": {"workload": "%s: %s" % (args.workload, workload_description(args.workload, args.grouped)),
                    "tokens_per_step": T, "distinct_adapters_per_step": distinct,
                    "algorithmic_bytes_per_step": bytes_step, "flops_per_step": flops_step,
-                   "l2": "rotating %d input copies, %.0f MB in total against a 126 MB L2%s" % (
-                       C, C * ws_bytes / 1e6, "" if C * ws_bytes >= 4 * L2_BYTES else " (copy count capped)"),
-                   "graph": not args.no_graph, "pdl": bool(L.lora_get_option("pdl")),
+                   "l2": "rotating %d input copies, %.0f MB in total against a 126 MB L2; a 256 MB buffer is "
+                         "written before each timed repetition" % (C, C * ws_bytes / 1e6),
+                   "timing": "median of %d repetitions of the %d-step region (graphs warmed before timing)" % (
+                       reps, K),
+                   "graph": not args.no_graph, "pdl": pdl,
                    "sigma": args.sigma, "jd_clusters": args.jd_clusters, "merge_slots": args.merge,
                    "parallelism": "replicas x%d (independent token batches, no collective)" % world},
         "roofline": roofline,
@@ -459,12 +625,11 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
         "clocks": clocks,
         "gpu_launches": int(K * launches_per_step),
+        "secondary": secondary,
+        "adapter_sweep": sweep,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
-    for c in copies:
-        for t in c.tables:
-            t.close()
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -501,18 +666,24 @@ def sample_workload(wl, T_sample: int):
 
 
 def cpu_baseline(wl, seconds: float):
+    """The oracle as it stands on the host cores: all threads (OpenMP over tokens) for about
+    two thirds of `seconds`, then one thread for the rest."""
     import oracle
     threads = oracle.max_threads()
-    # calibrate on a small sample, then size the sample so one pass is a fraction of the budget
-    per_tok_s = None
-    Ts = min(wl.T, 8)
-    v, reps, el = _oracle_tokens_per_s(wl, Ts, 0.2, threads)
-    per_tok_s = 1.0 / v
-    T_sample = int(max(1, min(wl.T, seconds / 4 / per_tok_s)))
-    v, reps, el = _oracle_tokens_per_s(wl, T_sample, seconds, threads)
+    out = {}
+    for nthr, budget in ((threads, seconds * 2 / 3), (1, seconds / 3)):
+        # calibrate on a small sample, then size the sample so one pass is a fraction of the budget
+        v, _reps, _el = _oracle_tokens_per_s(wl, min(wl.T, 8), 0.2, nthr)
+        T_sample = int(max(1, min(wl.T, budget / 4 * v)))
+        v, reps, el = _oracle_tokens_per_s(wl, T_sample, budget, nthr)
+        out[nthr if nthr == 1 else "all"] = (v, T_sample, reps, el)
+    v, T_sample, reps, el = out["all"]
+    v1, T1, reps1, el1 = out[1]
     return {"value": round(v, 2), "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": "first %d of %d tokens of one batch, all projections, repeated %d times (%.1f s), "
-                      "fp64 C loop with OpenMP over tokens" % (T_sample, wl.T, reps, el)}
+                      "fp64 C loop with OpenMP over tokens" % (T_sample, wl.T, reps, el),
+            "one_thread": {"value": round(v1, 2), "unit": UNIT, "cores": 1,
+                           "sample": "first %d tokens, repeated %d times (%.1f s)" % (T1, reps1, el1)}}
 
 
 def run_reference(args, rank, world):
