@@ -10,7 +10,9 @@
 //
 // The array lives in device global memory for as long as the library is loaded, on every
 // GPU that loads it.  Its device address is looked up once per device, with that device
-// current, on the first call made on that device.
+// current, on the first call made on that device, and kept for the life of the process: the
+// library must not be used on a device after cudaDeviceReset (or anything else that tears
+// down that device's primary context), because the kept address would then be stale.
 #include <mutex>
 
 #include "lora_common.cuh"
@@ -47,6 +49,10 @@ extern "C" int lora_sgmv_noalloc(const lora_table *table, const lora_segments *s
 {
     if (!table || !seg) return LORA_ERR_INVALID_ARG;
     if (seg->T < 0) return LORA_ERR_INVALID_ARG;
+    // The array used is the current device's; the table's descriptors live on table->device.
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LORA_ERR_CUDA;
+    if (dev != table->device) return LORA_ERR_INVALID_ARG;
     const int32_t ldv = (table->max_rank + 3) & ~3;
     if ((int64_t)seg->T * ldv > LORA_NOALLOC_SCRATCH_FLOATS) return LORA_ERR_WORKSPACE;
     float *v = nullptr;
