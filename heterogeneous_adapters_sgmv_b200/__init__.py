@@ -43,6 +43,7 @@ EXPORTS = (
     "lora_build_segments", "lora_shrink", "lora_expand", "lora_sgmv", "lora_bgmv",
     "lora_get_status", "lora_status_string", "lora_set_option", "lora_get_option",
     "lora_sgmv_noalloc", "lora_sgmv_grouped", "lora_table_set_sigma", "lora_bgmv_merged",
+    "lora_sgmv_base",
 )
 
 
@@ -91,6 +92,8 @@ def _load():
         "lora_bgmv": ([P, P, I32, P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
         "lora_bgmv_merged": ([P, P, P, I32, I32, P, I64, P, I64, I32, P, SZ, P], ctypes.c_int),
         "lora_sgmv_noalloc": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, I32, P], ctypes.c_int),
+        "lora_sgmv_base": ([P, ctypes.POINTER(lora_segments), P, I64, P, I64, P, I64, I32, I32, P, SZ, P],
+                           ctypes.c_int),
         "lora_sgmv_grouped": ([P, I32, ctypes.POINTER(lora_segments), P, P, P, P, P, P, SZ, P], ctypes.c_int),
         "lora_get_status": ([P, ctypes.POINTER(ctypes.c_uint32), I32, P], ctypes.c_int),
         "lora_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -184,6 +187,14 @@ def lora_sgmv(table: int, seg: lora_segments, x, ldx: int, y, ldy: int, y_offset
               ws_bytes: int = 0, stream=None) -> None:
     _check(_load().lora_sgmv(table, ctypes.byref(seg), _ptr(x), ldx, _ptr(y), ldy, y_offset, _ptr(ws), ws_bytes,
                              _stream(stream)), "lora_sgmv")
+
+
+def lora_sgmv_base(table: int, seg: lora_segments, x, ldx: int, W, ldw: int, y, ldy: int, y_offset: int,
+                   accumulate: bool = False, ws=None, ws_bytes: int = 0, stream=None) -> None:
+    """Layer output with the frozen base weight W [o, h]: y = (y if accumulate) + x W^T +
+    s_i B_i A_i x, on the tensor cores (contiguous segments, bf16)."""
+    _check(_load().lora_sgmv_base(table, ctypes.byref(seg), _ptr(x), ldx, _ptr(W), ldw, _ptr(y), ldy, y_offset,
+                                  1 if accumulate else 0, _ptr(ws), ws_bytes, _stream(stream)), "lora_sgmv_base")
 
 
 def lora_sgmv_grouped(tables, seg: lora_segments, xs, ldxs, ys, ldys, y_offsets, ws=None, ws_bytes: int = 0,

@@ -232,6 +232,10 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         const uint32_t data = smem_u32(stage_base + (size_t)s * p.stage_bytes + kHeaderBytes);
         const uint32_t fb = smem_u32(&ctl.full[s]);
         mbar_arrive_expect_tx(fb, bytes);
+        // Test-only stall (option "inject_stall"): the first tile of every unit is armed but its
+        // copies are never started, so its phase never completes and the consumers' bounded
+        // wait runs out.  No copy is in flight for it.
+        if (p.inject && j == 0) return;
         if (j < g.n_shrink) {
             const char *tmapA = reinterpret_cast<const char *>(p.pj[pi].tmA) + (size_t)a * 128;
             for (int b = 0; b < nbox; ++b) tma_load_2d(data + b * d.rank * kBoxBytes, tmapA, off + b * BOXW, 0, fb);
@@ -472,7 +476,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 }
                 for (int j = 0; j < ntiles; ++j) {
                     const int s = ps, m = pround;
-                    if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
+                    if (m >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status,
+                                                                      p.wait_ns))) {
                         alive = false;
                         break;
                     }
@@ -525,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         // end marker
         if (alive) {
             const int s = ps, m = pround;
-            if (m < 1 || mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) {
+            if (m < 1 || __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status, p.wait_ns))) {
                 if (lane == 0) {
                     reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes)->kind = kTileEnd;
                     mbar_arrive(smem_u32(&ctl.meta[s]));
@@ -536,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         }
         // drain: no copy may still be writing into this CTA's shared memory at exit
         for (int i = max(0, issued - S); i < issued; ++i)
-            mbar_wait(smem_u32(&ctl.full[i % S]), (i / S) & 1, p.status);
+            mbar_wait(smem_u32(&ctl.full[i % S]), (i / S) & 1, p.status, p.wait_ns);
         return;
     }
 
@@ -566,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             if (l < L && c < nch) ld[i] = *reinterpret_cast<const uint4 *>(src + h.tok[l] * ld_row + c * 16);
         }
     };
-    bool live = mbar_wait(smem_u32(&ctl.meta[0]), 0, p.status);
+    bool live = named_bar_and(1, kConsumers, mbar_wait(smem_u32(&ctl.meta[0]), 0, p.status, p.wait_ns));
     if (live && stage_header(0).kind != kTileEnd) load_rows(stage_header(0));
     int s = 0;          // stage of tile `it`
     uint32_t ph = 0;    // its phase parity
@@ -580,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         const int r = hdr.rank, L = hdr.L, flags = hdr.flags, len = hdr.len, off = hdr.off;
         const uint8_t *data = stage_base + (size_t)s * p.stage_bytes + kHeaderBytes;
         const int nch = len / EPC;   // 16-byte chunks per staged row
-        if (tid == 0 && u < 8 && kind == kTileShrink && (flags & kFlagFirst)) LORA_TRACE_MARK(32 + 4 * u);
+        if (tid == 0 && u < 6 && kind == kTileShrink && (flags & kFlagFirst)) LORA_TRACE_MARK(40 + 4 * u);
 
         named_bar_sync(1, kConsumers);   // every consumer is done with the previous tile's buffers
         if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(6 + 5 * (it - kTraceTile0));
@@ -593,11 +598,12 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         }
         // next tile's rows (its stage was released S - 1 tiles ago, so its header comes
         // without waiting on this tile)
-        if (!mbar_wait(smem_u32(&ctl.meta[s1]), ph1, p.status)) break;
-        if (stage_header(s1).kind != kTileEnd) load_rows(stage_header(s1));
-        if (!mbar_wait(smem_u32(&ctl.full[s]), ph, p.status)) break;
+        const bool okm = mbar_wait(smem_u32(&ctl.meta[s1]), ph1, p.status, p.wait_ns);
+        if (okm && stage_header(s1).kind != kTileEnd) load_rows(stage_header(s1));
+        const bool okf = mbar_wait(smem_u32(&ctl.full[s]), ph, p.status, p.wait_ns);
         if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(7 + 5 * (it - kTraceTile0));
-        named_bar_sync(1, kConsumers);
+        // every consumer stops together if any of them ran out of time
+        if (!named_bar_and(1, kConsumers, okm && okf)) break;
         if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(8 + 5 * (it - kTraceTile0));
 
         if (kind == kTileShrink) {
@@ -623,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     cvt16(l2 && okA ? *reinterpret_cast<const uint4 *>(xr1 + lane * 16) : z, xv1, (E *)nullptr);
                     cvt16(l2 && okB ? *reinterpret_cast<const uint4 *>(xr1 + 512 + lane * 16) : z, xv1 + EPC,
                           (E *)nullptr);
+                    if (tid == 0 && l == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(26 + 3 * (it - kTraceTile0));
                     for (int k = warp; k < r; k += 2 * kConsumerWarps) {
                         const bool k2 = k + kConsumerWarps < r;
                         float p[4];   // (token l, row k), (l, k + 8), (l + 1, k), (l + 1, k + 8)
@@ -646,6 +653,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                             p[2 + q] = t0 + t1;
                         }
                         // lane ends with value j = (lane >> 3) & 3, summed over all 32 lanes
+                        if (tid == 0 && l == 0 && k == warp && (unsigned)(it - kTraceTile0) < 2u)
+                            LORA_TRACE_MARK(27 + 3 * (it - kTraceTile0));
                         const bool hi16 = lane & 16, hi8 = lane & 8;
                         float k0 = hi16 ? p[2] : p[0], k1 = hi16 ? p[3] : p[1];
                         k0 += __shfl_xor_sync(0xffffffffu, hi16 ? p[0] : p[2], 16);
@@ -659,12 +668,14 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                             float *dst = vpart + (l + (hi16 ? 1 : 0)) * RP + k + (hi8 ? kConsumerWarps : 0);
                             *dst = first ? tot : *dst + tot;
                         }
+                        if (tid == 0 && l == 0 && k == warp && (unsigned)(it - kTraceTile0) < 2u)
+                            LORA_TRACE_MARK(28 + 3 * (it - kTraceTile0));
                     }
                 }
             }
             if (flags & kFlagLast) {
                 if (tid == 0) LORA_TRACE_MARK(15);
-                if (tid == 0 && u < 8) LORA_TRACE_MARK(33 + 4 * u);
+                if (tid == 0 && u < 6) LORA_TRACE_MARK(41 + 4 * u);
                 named_bar_sync(1, kConsumers);
                 if (tid == 0) LORA_TRACE_MARK(16);
                 if constexpr (CL > 1) {
@@ -673,7 +684,10 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         cluster_wait_acquire();   // every peer has initialised its barriers
                         cluster_waited = true;
                     }
-                    if (u >= 1 && !mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status)) break;
+                    // (a wait that ran out here is acted on, by all consumers together, at the
+                    // barrier after the sum)
+                    const bool okF =
+                        u < 1 || mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status, p.wait_ns);
                     if (tid == 0) LORA_TRACE_MARK(17);
                     const int nq = L * RP / 4;            // float4 quads of the partial
                     const int lgq = ceil_log2(nq);
@@ -688,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     }
                     if (tid == 0) mbar_arrive_expect_tx(rbar, (uint32_t)(CL * nq * 16));
                     if (tid == 0) LORA_TRACE_MARK(18);
-                    if (!mbar_wait_cluster(rbar, u & 1, p.status)) break;
+                    const bool okR = mbar_wait_cluster(rbar, u & 1, p.status, p.wait_ns);
                     if (tid == 0) LORA_TRACE_MARK(19);
                     // ---- sum the CL partials in CTA order (entries k >= r are never read)
                     for (int e = tid; e < (L << lgRP); e += kConsumers) {
@@ -701,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         }
                     }
                     if (tid == 0) LORA_TRACE_MARK(20);
-                    named_bar_sync(1, kConsumers);
+                    if (!named_bar_and(1, kConsumers, okF && okR)) break;
                     if (tid == 0) LORA_TRACE_MARK(21);
                     if (tid < CL) mbar_arrive_remote_relaxed(smem_u32(&ctl.freed), tid);
                     if (tid == 0) LORA_TRACE_MARK(22);
@@ -770,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         if (k < r) p.v[(int64_t)hdr.tok[l] * p.ldv + k] = vsum[l * RP + k];
                     }
                 }
-                if (tid == 0 && u < 8) LORA_TRACE_MARK(34 + 4 * u);
+                if (tid == 0 && u < 6) LORA_TRACE_MARK(42 + 4 * u);
                 ++u;
             }
         } else {  // kTileExpand
@@ -840,6 +854,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                             }
                         }
                     }
+                    if (tid == 0 && l == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(32 + 2 * (it - kTraceTile0));
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         if (q == 1 && !l2) break;
@@ -857,11 +872,12 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                             static_cast<float *>(pj.y)[gofs] = fmaf(sl, acc[0], w);
                         }
                     }
+                    if (tid == 0 && l == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(33 + 2 * (it - kTraceTile0));
                 }
             }
         }
         if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(9 + 5 * (it - kTraceTile0));
-        if (tid == 0 && kind == kTileExpand && (flags & kFlagLast) && u >= 1 && u <= 8) LORA_TRACE_MARK(35 + 4 * (u - 1));
+        if (tid == 0 && kind == kTileExpand && (flags & kFlagLast) && u >= 1 && u <= 6) LORA_TRACE_MARK(43 + 4 * (u - 1));
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
         s = s1;
@@ -870,7 +886,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     if (tid == 0) LORA_TRACE_MARK(24);
     // No CTA may leave while a peer can still arrive on its barriers: wait until every peer
     // has released the partials of the last unit.
-    if (CL > 1 && MODE != kModeExpand && u >= 1) mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status);
+    if (CL > 1 && MODE != kModeExpand && u >= 1) mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status, p.wait_ns);
     if (tid == 0) LORA_TRACE_MARK(25);
 }
 

@@ -37,6 +37,12 @@ Options &options()
     return o;
 }
 
+uint64_t wait_limit_ns()
+{
+    const int64_t v = options().wait_limit_ns;
+    return v > 0 ? (uint64_t)v : kWaitLimitNs;
+}
+
 // prefill.cu
 bool prefill_supported(const lora_table *t);
 int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y,
@@ -128,6 +134,8 @@ DecodeParams base_params(const lora_table *t)
     p.n = t->n;
     p.R = t->max_rank;
     p.status = t->d_status;
+    p.wait_ns = wait_limit_ns();
+    p.inject = (int32_t)(options().inject_stall & 1);
     return p;
 }
 
@@ -365,6 +373,29 @@ int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int6
     return launch_decode(kModeFused, kSrcSegments, p, t->dtype, s);
 }
 
+int lora_sgmv_base(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, const void *W,
+                   int64_t ldw, void *y, int64_t ldy, int32_t y_off, int32_t accumulate, void *ws, size_t ws_bytes,
+                   void *stream)
+{
+    int rc = check_table(t);
+    if (rc) return rc;
+    if ((rc = check_segments(seg))) return rc;
+    if ((rc = check_io(t, x, ldx, y, ldy, y_off, true, true))) return rc;
+    if (!W || ldw < t->h || (accumulate != 0 && accumulate != 1)) return LORA_ERR_INVALID_ARG;
+    if (!al16(W) || ldw % 8) return LORA_ERR_UNSUPPORTED;
+    // tensor-core tiles only: bf16 tables with ranks that are multiples of 8 up to 64, no
+    // Sigma, tokens contiguous per segment
+    if (!prefill_supported(t) || seg->perm != nullptr) return LORA_ERR_UNSUPPORTED;
+    if (seg->T == 0) return LORA_OK;
+    const WsLayout w = ws_layout(t, seg->T);
+    if (!ws || ws_bytes < w.total) return LORA_ERR_WORKSPACE;
+    if (!al16(ws)) return LORA_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void *v = static_cast<uint8_t *>(ws) + w.v;
+    if (seg->max_segs > 0 && (rc = launch_prefill_shrink(t, seg, x, ldx, v, true, s)) != LORA_OK) return rc;
+    return launch_base_gemm(t, seg, x, ldx, W, ldw, y, ldy, y_off, accumulate, v, s);
+}
+
 int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_segments *seg,
                       const void *const *x, const int64_t *ldx, void *const *y, const int64_t *ldy,
                       const int32_t *y_off, void *ws, size_t ws_bytes, void *stream)
@@ -573,6 +604,8 @@ int lora_set_option(const char *key, int64_t value)
     else if (!std::strcmp(key, "prefill_min_seg_len")) o.prefill_min_seg_len = value;
     else if (!std::strcmp(key, "prefill_ksplit")) o.prefill_ksplit = value;
     else if (!std::strcmp(key, "split")) o.split = value;
+    else if (!std::strcmp(key, "wait_limit_ns")) o.wait_limit_ns = value;
+    else if (!std::strcmp(key, "inject_stall")) o.inject_stall = value;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }
@@ -589,6 +622,8 @@ int lora_get_option(const char *key, int64_t *value)
     else if (!std::strcmp(key, "prefill_min_seg_len")) *value = o.prefill_min_seg_len;
     else if (!std::strcmp(key, "prefill_ksplit")) *value = o.prefill_ksplit;
     else if (!std::strcmp(key, "split")) *value = o.split;
+    else if (!std::strcmp(key, "wait_limit_ns")) *value = o.wait_limit_ns;
+    else if (!std::strcmp(key, "inject_stall")) *value = o.inject_stall;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }

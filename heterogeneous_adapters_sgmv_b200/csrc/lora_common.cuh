@@ -25,7 +25,8 @@ struct __align__(32) AdapterDesc {
 };
 static_assert(sizeof(AdapterDesc) == 32, "descriptor size");
 
-// Upper bound of a bounded wait: about two seconds of %globaltimer.
+// Default upper bound of a bounded wait: about two seconds of %globaltimer.  Kernels take the
+// bound from their parameters (option "wait_limit_ns"), so a test can shorten it.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
@@ -124,29 +125,31 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
-// Bounded waits: false after ~2 s, with LORA_STATUS_TIMEOUT latched into *status.  The fast
-// path (phase already complete) is inlined; the polling loop is a separate function so the hot
-// code stays small (instruction-cache misses dominate short kernels).
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint32_t *status, bool cluster)
+// Bounded waits: false after `limit_ns` of %globaltimer, with LORA_STATUS_TIMEOUT latched into
+// *status.  The fast path (phase already complete) is inlined; the polling loop is a separate
+// function so the hot code stays small (instruction-cache misses dominate short kernels).
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint32_t *status, bool cluster,
+                                                   uint64_t limit_ns)
 {
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             atomicOr(status, LORA_STATUS_TIMEOUT);
             return false;
         }
     }
 }
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *status, uint64_t limit_ns)
 {
-    return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, status, false);
+    return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, status, false, limit_ns);
 }
 
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint32_t *status)
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint32_t *status,
+                                                  uint64_t limit_ns)
 {
-    return mbar_try_wait_cluster(bar, parity) || mbar_wait_slow(bar, parity, status, true);
+    return mbar_try_wait_cluster(bar, parity) || mbar_wait_slow(bar, parity, status, true, limit_ns);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -285,6 +288,22 @@ __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_addr, uint32_t r
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier over `count` threads that also returns the AND of `pred` over them: used so a
+// bounded wait that ran out in any thread stops all of them at the same point.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n"
+        " setp.ne.u32 p, %1, 0;\n"
+        " bar.red.and.pred q, %2, %3, p;\n"
+        " selp.u32 %0, 1, 0, q;\n}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------------------------------

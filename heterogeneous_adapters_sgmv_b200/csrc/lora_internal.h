@@ -47,6 +47,8 @@ struct DecodeParams {
     int32_t w_stride;
     int32_t T;
     uint32_t *status;
+    uint64_t wait_ns;      // bound of every device-side wait (option "wait_limit_ns")
+    int32_t inject;        // test-only stall injection (option "inject_stall"), 0 in normal use
     int32_t stages;        // pipeline depth
     int32_t stage_bytes;   // bytes of one stage (header + data)
     int32_t ids_smem;      // kSrcIds: bytes of the id / leader scratch in shared memory
@@ -61,7 +63,11 @@ struct Options {
     int64_t prefill_min_seg_len = 256;
     int64_t prefill_ksplit = 4;      // CTAs splitting h in the tcgen05 shrink (4 or 8)
     int64_t split = 0;
+    int64_t wait_limit_ns = 0;       // 0: the default bound (about 2 s)
+    int64_t inject_stall = 0;        // test-only: bit 0 decode, bit 1 prefill shrink, bit 2 prefill expand
 };
+// Bound of the device-side waits for the next launch.
+uint64_t wait_limit_ns();
 Options &options();
 
 // Launchers (return a LORA_* code).
@@ -70,6 +76,14 @@ int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *per
                           int32_t *seg_adapter, int32_t *num_segs, uint32_t *status, cudaStream_t s);
 // Tensor maps of every adapter for the tcgen05 prefill path (no-op when the table does not qualify).
 int prefill_build_maps(lora_table *t);
+// tcgen05 shrink alone (contiguous segments, prefill-capable table): v receives the bf16 hi and
+// lo parts ([T, 64] each) of x . A_i^T, multiplied by s_i when fold_scale.
+int launch_prefill_shrink(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *v,
+                          bool fold_scale, cudaStream_t s);
+// Fused layer output (base_gemm.cu): y = (y if accumulate) + x W^T + the adapter term, from the
+// scale-folded intermediate v that launch_prefill_shrink wrote.
+int launch_base_gemm(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, const void *W,
+                     int64_t ldw, void *y, int64_t ldy, int32_t y_off, int accumulate, const void *v, cudaStream_t s);
 // Encode the TMA tensor map of A_i [rank, h] used by the decode shrink (host side).
 int encode_tmap_A(void *out128, const void *A, int dtype, int h, int rank);
 

@@ -30,6 +30,7 @@
 
 #include "lora_common.cuh"
 #include "lora_internal.h"
+#include "tcgen05.cuh"
 
 namespace lora {
 namespace {
@@ -42,84 +43,6 @@ constexpr int kStagesMax = 4;        // shrink pipeline depth
 __host__ __device__ constexpr int shrink_stages(int) { return 4; }
 constexpr int kThreadsPF = 128;      // 4 warps: one TMEM lane quarter each
 constexpr int kMaxRankPF = 64;
-
-// ------------------------------------------------------------------- tcgen05 helpers
-
-__device__ __forceinline__ void tmem_alloc(uint32_t smem_dst, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish()
-{
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-
-// D[tmem] (+)= A[smem desc] . B[smem desc]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate)
-{
-    asm volatile(
-        "{\n .reg .pred p;\n"
-        " setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Arrive (once) on `bar` when all previously issued MMAs of this thread have completed.
-__device__ __forceinline__ void umma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// Shared-memory descriptor of a K-major operand stored with the 128-byte swizzle: rows of
-// 128 bytes, 8-row atoms of 1024 bytes stacked along M/N (stride 1024), sm_100 descriptor
-// version 1.  Advancing K by 16 bf16 within the 128-byte row adds 32 bytes to the start.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
-{
-    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)1u << 16;              // leading byte offset (unused with this swizzle)
-    d |= (uint64_t)(1024u >> 4) << 32;    // stride byte offset: next 8-row atom
-    d |= (uint64_t)1u << 46;              // descriptor version
-    d |= (uint64_t)2u << 61;              // SWIZZLE_128B
-    return d;
-}
-
-// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N)
-{
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-// Byte offset of 16-byte chunk c of row m in a 128-byte-swizzled [rows][128 B] tile.
-__device__ __forceinline__ uint32_t sw128_off(int m, int c) { return (uint32_t)(m * 128 + ((c ^ (m & 7)) << 4)); }
 
 struct PrefillParams {
     CUtensorMap tmap_io;          // shrink: x [T, h]; expand: y slice [T, o]   (box 64 x 128)
@@ -134,6 +57,9 @@ struct PrefillParams {
     int64_t ldy;
     int32_t y_off;
     uint32_t *status;
+    uint64_t wait_ns;             // bound of every device-side wait
+    int32_t inject;               // test-only stall injection: bit 1 shrink, bit 2 expand
+    int32_t fold_scale;           // shrink: store s_i * v instead of v (fused base product)
 };
 
 // Map a global 128-token tile index to (segment, first row, rows).  One warp scans the
@@ -180,6 +106,7 @@ struct __align__(8) ShrinkCtl {
     uint64_t done;
     uint32_t tmem_base;
     int32_t info[5];   // valid, row0, rows, adapter, rank
+    float scale;       // multiplier of the stored intermediate (1, or s_i when folding)
 };
 
 template <int KS>
@@ -215,6 +142,7 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
             ctl.info[2] = rows;
             ctl.info[3] = a;
             ctl.info[4] = good ? p.desc[a].rank : 0;
+            ctl.scale = (good && p.fold_scale) ? p.desc[a].scale : 1.f;
             for (int i = 0; i < kStages; ++i) {
                 mbar_init(smem_u32(&ctl.full[i]), 1);
                 mbar_init(smem_u32(&ctl.empty[i]), 1);
@@ -232,6 +160,7 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     tc_fence_after();
     const bool valid = ctl.info[0] != 0;
     const int row0 = ctl.info[1], rows = ctl.info[2], a = ctl.info[3], r = ctl.info[4];
+    const float vscale = ctl.scale;
     const int npad = (r + 15) & ~15;
     const uint32_t tmem = ctl.tmem_base;
     const int nkb_all = (p.h + kBK - 1) / kBK;
@@ -245,22 +174,35 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
             // producer: x tile (128 tokens x 64 columns) and A_i tile (npad rows x 64 columns)
             const void *tA = p.tm_A + (size_t)a * 128;
             const uint32_t bytes = (uint32_t)(kXBytes + npad * 128);
+            int issued = 0;
+            bool stalled = false;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kStages, m = kb / kStages;
-                if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status)) break;
+                if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status, p.wait_ns)) {
+                    stalled = true;
+                    break;
+                }
                 uint8_t *st = smem + s * kStageBytes;
                 const uint32_t fb = smem_u32(&ctl.full[s]);
                 mbar_arrive_expect_tx(fb, bytes);
+                ++issued;
+                // test-only stall: the first k-block is armed but never loaded
+                if ((p.inject & 2) && kb == 0) continue;
                 const int k0 = (kb0 + kb) * kBK;
                 tma_load_2d(smem_u32(st), &p.tmap_io, k0, row0, fb);
                 tma_load_2d(smem_u32(st + kXBytes), tA, k0, 0, fb);
             }
+            // After a timeout the ring is given up early: wait (bounded) for the copies of the
+            // last stages issued, so none is still writing when the ring is reused below.
+            if (stalled || (p.inject & 2))
+                for (int kb = max(0, issued - kStages); kb < issued; ++kb)
+                    mbar_wait(smem_u32(&ctl.full[kb % kStages]), (kb / kStages) & 1, p.status, p.wait_ns);
         } else if (warp == 1 && lane == 0) {
             // MMA issuer
             const uint32_t idesc = idesc_bf16(kTileM, npad);
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kStages, m = kb / kStages;
-                if (!mbar_wait(smem_u32(&ctl.full[s]), m & 1, p.status)) break;
+                if (!mbar_wait(smem_u32(&ctl.full[s]), m & 1, p.status, p.wait_ns)) break;
                 tc_fence_after();
                 uint8_t *st = smem + s * kStageBytes;
                 const uint64_t ad = sw128_desc(smem_u32(st));
@@ -273,11 +215,13 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
             umma_commit(smem_u32(&ctl.done));
         }
         __syncwarp();
-        ok = mbar_wait(smem_u32(&ctl.done), 0, p.status);
+        ok = mbar_wait(smem_u32(&ctl.done), 0, p.status, p.wait_ns);
         tc_fence_after();
     }
     // ---- epilogue: partial [128][npad] from tensor memory (zeros when this CTA had no k-blocks)
-    __syncthreads();   // the ring is free: all MMAs and loads that fed them are complete
+    // The ring is free: all MMAs and loads that fed them are complete.  A wait that ran out in
+    // any thread makes every thread skip the (warp-collective) tensor-memory loads.
+    ok = __syncthreads_and(ok) != 0;
     const int m = warp * 32 + lane;   // row of the tile = TMEM lane
     if (valid) {
         for (int c0 = 0; c0 < npad; c0 += 32) {
@@ -318,6 +262,10 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
                 }
             }
             if (rr < rows) {
+                sum.x *= vscale;   // exact when the scale is 1
+                sum.y *= vscale;
+                sum.z *= vscale;
+                sum.w *= vscale;
                 const __nv_bfloat162 h01 = __floats2bfloat162_rn(sum.x, sum.y);
                 const __nv_bfloat162 h23 = __floats2bfloat162_rn(sum.z, sum.w);
                 const float2 g01 = __bfloat1622float2(h01), g23 = __bfloat1622float2(h23);
@@ -431,7 +379,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        int cur_g = -1, vcount = 0, row0 = 0, rows = 0, a = 0, vb = 0;
+        int cur_g = -1, vcount = 0, row0 = 0, rows = 0, a = 0, vb = 0, nissued = 0;
         float sc = 0.f;
         for (int t = t0; t < t1 && ok; ++t) {
             const int i = t - t0, s = i % kExStages;
@@ -448,7 +396,8 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 sc = p.desc[a].scale;
                 cur_g = g;
                 vb = vcount & 1;
-                if (vcount >= 2 && !mbar_wait(smem_u32(&ctl.vempty[vb]), ((vcount >> 1) - 1) & 1, p.status)) {
+                if (vcount >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.vempty[vb]),
+                                                                     ((vcount >> 1) - 1) & 1, p.status, p.wait_ns))) {
                     ok = false;
                     break;
                 }
@@ -464,7 +413,8 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 __syncwarp();
                 ++vcount;
             }
-            if (i >= kExStages && !mbar_wait(smem_u32(&ctl.empty[s]), ((i / kExStages) - 1) & 1, p.status)) {
+            if (i >= kExStages && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]),
+                                                                     ((i / kExStages) - 1) & 1, p.status, p.wait_ns))) {
                 ok = false;
                 break;
             }
@@ -479,19 +429,24 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 uint8_t *st = ring + s * kExStageBytes;
                 const uint32_t fb = smem_u32(&ctl.full[s]);
                 mbar_arrive_expect_tx(fb, kExStageBytes);
-                tma_load_2d(smem_u32(st), p.tm_B + (size_t)a * 128, 0, nt * kTileN, fb);
-                tma_load_2d(smem_u32(st + 16384), &p.tmap_io, nt * kTileN, row0, fb);
-                tma_load_2d(smem_u32(st + 32768), &p.tmap_io, nt * kTileN + 64, row0, fb);
+                // test-only stall: the first tile's stage is armed but never loaded
+                if (!((p.inject & 4) && i == 0)) {
+                    tma_load_2d(smem_u32(st), p.tm_B + (size_t)a * 128, 0, nt * kTileN, fb);
+                    tma_load_2d(smem_u32(st + 16384), &p.tmap_io, nt * kTileN, row0, fb);
+                    tma_load_2d(smem_u32(st + 32768), &p.tmap_io, nt * kTileN + 64, row0, fb);
+                }
             }
+            ++nissued;
             __syncwarp();
         }
-        // drain: every TMA issued by this CTA has landed before shared memory is released
-        const int n = t1 - t0;
+        // drain: every TMA issued by this CTA has landed before shared memory is released (the
+        // stages of the last kExStages tiles armed; earlier ones were consumed before reuse)
+        const int n = nissued;
         if (lane == 0) {
             for (int i = max(0, n - kExStages); i < n; ++i)
-                mbar_wait(smem_u32(&ctl.full[i % kExStages]), (i / kExStages) & 1, p.status);
+                mbar_wait(smem_u32(&ctl.full[i % kExStages]), (i / kExStages) & 1, p.status, p.wait_ns);
             for (int c = max(0, vcount - 2); c < vcount; ++c)
-                mbar_wait(smem_u32(&ctl.vfull[c & 1]), (c >> 1) & 1, p.status);
+                mbar_wait(smem_u32(&ctl.vfull[c & 1]), (c >> 1) & 1, p.status, p.wait_ns);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -500,15 +455,15 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             int vuse = 0, prev_vb = -1;
             for (int t = t0; t < t1; ++t) {
                 const int i = t - t0, s = i % kExStages, ab = i & 1;
-                if (!mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status)) break;
+                if (!mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status, p.wait_ns)) break;
                 const int vb = ctl.info[s].vb;
                 if (vb != prev_vb) {
                     if (prev_vb >= 0) umma_commit(smem_u32(&ctl.vempty[prev_vb]));   // old tile may be rebuilt
-                    if (!mbar_wait(smem_u32(&ctl.vfull[vb]), (vuse >> 1) & 1, p.status)) break;
+                    if (!mbar_wait(smem_u32(&ctl.vfull[vb]), (vuse >> 1) & 1, p.status, p.wait_ns)) break;
                     ++vuse;
                     prev_vb = vb;
                 }
-                if (i >= 2 && !mbar_wait(smem_u32(&ctl.accempty[ab]), ((i >> 1) - 1) & 1, p.status)) break;
+                if (i >= 2 && !mbar_wait(smem_u32(&ctl.accempty[ab]), ((i >> 1) - 1) & 1, p.status, p.wait_ns)) break;
                 tc_fence_after();
                 const uint8_t *st = ring + s * kExStageBytes;
                 const uint64_t dh = sw128_desc(smem_u32(vbuf + vb * kExVBytes));
@@ -524,7 +479,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             }
             // every MMA of this CTA has completed before tensor memory is released
             umma_commit(smem_u32(&ctl.mma_done));
-            mbar_wait(smem_u32(&ctl.mma_done), 0, p.status);
+            mbar_wait(smem_u32(&ctl.mma_done), 0, p.status, p.wait_ns);
         }
         __syncwarp();
     } else {
@@ -535,8 +490,11 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         const int ew = warp - 2;                // epilogue warp 0..7
         for (int t = t0; t < t1; ++t) {
             const int i = t - t0, s = i % kExStages, ab = i & 1;
-            if (!mbar_wait(smem_u32(&ctl.accfull[ab]), (i >> 1) & 1, p.status)) break;
-            if (!mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status)) break;
+            // every epilogue warp leaves together if any lane ran out of time (the tensor-memory
+            // loads below are warp-collective and the warps meet at a named barrier)
+            const bool oka = mbar_wait(smem_u32(&ctl.accfull[ab]), (i >> 1) & 1, p.status, p.wait_ns);
+            const bool okf = mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status, p.wait_ns);
+            if (!named_bar_and(3, kEpiWarps * 32, oka && okf)) break;
             tc_fence_after();
             const ExTileInfo inf = ctl.info[s];
             uint8_t *yt = ring + s * kExStageBytes + 16384 + half * 16384;   // this half's 64-column box
@@ -600,35 +558,6 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
 
 // ------------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaDriverEntryPointQueryResult q;
-        void *fn = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
-    return encode;
-}
-
-// bf16 2-D map [rows, cols] with row stride `ld` elements, box 64 columns x box_rows, 128B swizzle.
-int encode_sw128(CUtensorMap *out, const void *base, uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_rows)
-{
-    auto encode = get_encode();
-    if (!encode) return LORA_ERR_CUDA;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {ld * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult rc = encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return rc == CUDA_SUCCESS ? LORA_OK : LORA_ERR_UNSUPPORTED;
-}
-
 constexpr int shrink_smem(int ks) { return shrink_stages(ks) * (kTileM * 128 + kMaxRankPF * 128) + 256 + 1024; }
 constexpr int kExpandSmem = 2 * kExVBytes + kExStages * kExStageBytes + (int)sizeof(ExpandCtl) + 1024;
 static_assert(shrink_stages(8) * (kTileM * 128 + kMaxRankPF * 128) >= kTileM * (kMaxRankPF + 4) * 4, "partial fits ring");
@@ -664,10 +593,10 @@ int prefill_build_maps(lora_table *t)
     return LORA_OK;
 }
 
-int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y, int64_t ldy,
-                   int32_t y_off, void *v, cudaStream_t s)
+namespace {
+
+PrefillParams prefill_params(const lora_table *t, const lora_segments *seg, void *v)
 {
-    if (!prefill_supported(t)) return LORA_ERR_UNSUPPORTED;
     PrefillParams p;
     std::memset(&p, 0, sizeof p);
     p.desc = t->d_desc;
@@ -683,12 +612,14 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
     p.n = t->n;
     p.v_hi = static_cast<uint16_t *>(v);
     p.v_lo = p.v_hi + (int64_t)seg->T * kMaxRankPF;
-    p.y = y;
-    p.ldy = ldy;
-    p.y_off = y_off;
     p.status = t->d_status;
-    const int mt_bound = seg->max_segs + (seg->T + kTileM - 1) / kTileM;
+    p.wait_ns = wait_limit_ns();
+    p.inject = (int32_t)(options().inject_stall & 6);
+    return p;
+}
 
+int set_prefill_attributes()
+{
     static bool attr_done[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LORA_ERR_CUDA;
@@ -702,35 +633,70 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
             return LORA_ERR_CUDA;
         attr_done[dev] = true;
     }
-    const Options &opt = options();
+    return LORA_OK;
+}
 
-    // shrink: clusters of KS CTAs (split of h), one cluster per 128-token tile
+// The tcgen05 shrink: clusters of KS CTAs (split of h), one cluster per 128-token tile of a
+// segment; the intermediate (times s_i when fold_scale) goes to v as bf16 hi + lo [T, 64] each.
+int launch_shrink_kernel(PrefillParams &p, const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx,
+                         cudaStream_t s)
+{
+    const Options &opt = options();
+    const int mt_bound = seg->max_segs + (seg->T + kTileM - 1) / kTileM;
     int rc = encode_sw128(&p.tmap_io, x, (uint64_t)t->h, (uint64_t)seg->T, (uint64_t)ldx, kTileM);
     if (rc != LORA_OK) return rc;
-    {
-        cudaLaunchConfig_t cfg = {};
-        const int KS = opt.prefill_ksplit == 8 ? 8 : 4;
-        cfg.gridDim = dim3(KS * mt_bound);
-        cfg.blockDim = dim3(kThreadsPF);
-        cfg.dynamicSmemBytes = shrink_smem(KS);
-        cfg.stream = s;
-        cudaLaunchAttribute attr[2];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = KS;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        int na = 1;
-        if (opt.pdl) {
-            attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[na].val.programmaticStreamSerializationAllowed = 1;
-            ++na;
-        }
-        cfg.attrs = attr;
-        cfg.numAttrs = na;
-        const cudaError_t e = KS == 4 ? cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<4>, p)
-                                      : cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<8>, p);
-        if (e != cudaSuccess) return LORA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    const int KS = opt.prefill_ksplit == 8 ? 8 : 4;
+    cfg.gridDim = dim3(KS * mt_bound);
+    cfg.blockDim = dim3(kThreadsPF);
+    cfg.dynamicSmemBytes = shrink_smem(KS);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = KS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    int na = 1;
+    if (opt.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
     }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    const cudaError_t e = KS == 4 ? cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<4>, p)
+                                  : cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<8>, p);
+    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_prefill_shrink(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *v,
+                          bool fold_scale, cudaStream_t s)
+{
+    if (!prefill_supported(t)) return LORA_ERR_UNSUPPORTED;
+    int rc = set_prefill_attributes();
+    if (rc != LORA_OK) return rc;
+    PrefillParams p = prefill_params(t, seg, v);
+    p.fold_scale = fold_scale ? 1 : 0;
+    return launch_shrink_kernel(p, t, seg, x, ldx, s);
+}
+
+int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y, int64_t ldy,
+                   int32_t y_off, void *v, cudaStream_t s)
+{
+    if (!prefill_supported(t)) return LORA_ERR_UNSUPPORTED;
+    int rc = set_prefill_attributes();
+    if (rc != LORA_OK) return rc;
+    PrefillParams p = prefill_params(t, seg, v);
+    p.y = y;
+    p.ldy = ldy;
+    p.y_off = y_off;
+    const int mt_bound = seg->max_segs + (seg->T + kTileM - 1) / kTileM;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LORA_ERR_CUDA;
+    const Options &opt = options();
+    if ((rc = launch_shrink_kernel(p, t, seg, x, ldx, s)) != LORA_OK) return rc;
     // expand: persistent, one CTA per SM over all (128-token tile, 128-column tile) pairs
     if ((rc = encode_sw128(&p.tmap_vhi, p.v_hi, kMaxRankPF, (uint64_t)seg->T, kMaxRankPF, kTileM)) != LORA_OK ||
         (rc = encode_sw128(&p.tmap_vlo, p.v_lo, kMaxRankPF, (uint64_t)seg->T, kMaxRankPF, kTileM)) != LORA_OK)

@@ -79,7 +79,8 @@ extern "C" {
 
 typedef struct lora_table lora_table; /* opaque */
 
-/* Segments: tokens grouped by adapter ("grouping requests that use the same LoRA model").
+/* Segments: tokens grouped by adapter, so that all requests of one LoRA model are served
+ * together ("Compress then Serve" review thread, authors' rebuttal on Punica, SGMV).
  * Segment s covers sorted positions [seg_ptr[s], seg_ptr[s+1]); the token at sorted position
  * p is perm[p], or p itself when perm is NULL (tokens already contiguous per adapter, as in
  * prefill).  All arrays are device memory and may be produced by lora_build_segments. */
@@ -183,6 +184,24 @@ int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_seg
                       const void *const *x, const int64_t *ldx, void *const *y, const int64_t *ldy,
                       const int32_t *y_offset, void *ws, size_t ws_bytes, void *stream);
 
+/* Layer output with the frozen base weight, fused with the adapter term ("TGI Multi-LoRA"
+ * page, "Technical Foundation: LoRA": the pretrained W stays frozen and the adapter adds
+ * B A x; "predibase/lorax" repository page: one forward pass of the layer):
+ *   y[t, y_offset + n] = (accumulate ? y[t, y_offset + n] : 0) + sum_j x[t, j] W[n, j]
+ *                        + s_i * sum_k B_i[n, k] (x[t] . A_i[k])       (n < o)
+ * for every token t < seg->T; tokens outside all segments get the first two terms only.
+ * W is [o, ldw] row-major bf16 (a linear layer's weight; the first h columns are used),
+ * 16-byte aligned, ldw a multiple of 8.  Runs on the tcgen05 tensor cores: the shrink stores
+ * s_i * (x . A_i^T) as bf16 hi + lo in the workspace, then one persistent kernel accumulates
+ * x W^T and that intermediate times B_i in the same tensor-memory tile and writes y once.
+ * Requires a bf16 table whose ranks are multiples of 8 and at most 64 without Sigma, and
+ * seg->perm == NULL (tokens contiguous per segment, segments in position order); otherwise
+ * LORA_ERR_UNSUPPORTED.  accumulate is 0 or 1.  ws_bytes >= lora_workspace_bytes(table, T).
+ * The products are rounded once, to bf16, per output (fp32 accumulation). */
+int lora_sgmv_base(const lora_table *table, const lora_segments *seg, const void *x, int64_t ldx,
+                   const void *W, int64_t ldw, void *y, int64_t ldy, int32_t y_offset,
+                   int32_t accumulate, void *ws, size_t ws_bytes, void *stream);
+
 /* BGMV: the same update driven by per-token ids (d_ids[T], device) without a caller-built
  * segment table, as the per-token "indices" of the pseudocode.  Tokens sharing an adapter
  * are grouped on the device so each adapter's weights are read once per group.  For
@@ -222,7 +241,10 @@ int lora_get_status(const lora_table *table, uint32_t *h_status, int32_t reset, 
  * The first call on a device looks up the array's address on that device (make that first
  * call outside any stream capture).  All calls share the one array: calls that can overlap on
  * the GPU (different streams, or different host threads) race on it and must be serialised by
- * the caller.  The array keeps the last call's contents; nothing relies on it starting at 0. */
+ * the caller.  The array keeps the last call's contents; nothing relies on it starting at 0.
+ * The current device must be the table's device (else LORA_ERR_INVALID_ARG).  The looked-up
+ * address is kept for the life of the process, so the library must not be used on a device
+ * after cudaDeviceReset (or any other teardown of that device's primary context). */
 #define LORA_NOALLOC_SCRATCH_FLOATS 262144
 int lora_sgmv_noalloc(const lora_table *table, const lora_segments *seg, const void *x, int64_t ldx,
                       void *y, int64_t ldy, int32_t y_offset, void *stream);
@@ -238,7 +260,12 @@ const char *lora_status_string(int code);
  * the persistent decode grid, for tuning), "prefill_ksplit" (4, the default, or 8 CTAs splitting
  * h in the tcgen05 shrink), "prefill_min_seg_len" (segment-length hint at or above which lora_sgmv takes the tcgen05
  * path; 0 disables that path), "split" (1: lora_sgmv runs lora_shrink then lora_expand
- * through the workspace instead of the fused kernel).  Returns LORA_ERR_INVALID_ARG for an
+ * through the workspace instead of the fused kernel), "wait_limit_ns" (bound of every
+ * device-side wait of the following launches; 0: the default of about 2 s), "inject_stall"
+ * (tests only: a bit mask, 1 decode kernels, 2 tcgen05 shrink, 4 tcgen05 expand, that arms one
+ * pipeline stage per unit or tile without ever loading it, so the bounded wait on it runs
+ * out, LORA_STATUS_TIMEOUT is latched and the kernel drains its copies, releases tensor
+ * memory and returns; results are then invalid).  Returns LORA_ERR_INVALID_ARG for an
  * unknown key. */
 int lora_set_option(const char *key, int64_t value);
 int lora_get_option(const char *key, int64_t *value);
