@@ -41,6 +41,7 @@ from workloads import accounting  # noqa: E402
 METRIC = "tokens/s of batched multi-LoRA delta; fraction of HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 NOMINAL_HBM_GBS = 8000.0
 L2_BYTES = 126 * 1024 * 1024
 
@@ -75,6 +76,9 @@ def parse():
                     help="with --sigma: adapters share the A and B of adapter (i mod K), as compressed clusters do")
     ap.add_argument("--merge", type=int, default=1,
                     help="decode_bgmv: K adapters merged per token (weighted ensembles, lora_bgmv_merged)")
+    ap.add_argument("--base", action="store_true",
+                    help="prefill_sgmv: the layer output with a synthetic frozen base weight, x W^T plus the adapter "
+                         "term, through lora_sgmv_base (tensor-core bound)")
     ap.add_argument("--grouped", action="store_true",
                     help="many_adapter_qkvo: one lora_sgmv_grouped launch for q, k, v, o (q, k, v reading one x) "
                          "instead of four lora_sgmv calls")
@@ -90,6 +94,29 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s sustained under the power cap (the kernels are timed over about a
+    second of back-to-back steps): the measured sustained figure, else this machine's fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        for key in ("bf16_tflops_sustained", "bf16_tflops"):
+            if key in d:
+                return float(d[key]), "measured (%s)" % key
+    return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
+
+
+def tensor_roofline(flops_step, ms_step, launches_per_step, kname):
+    peak, kind = measured_tensor_peak()
+    achieved = flops_step / (ms_step / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": "%s, MEASURED_PEAKS.json" % kind if kind != "fallback"
+            else "fallback 1.4 PFLOP/s sustained", "flops_per_step": flops_step, "kernel": kname,
+            "basis": "whole step (%d launches): a lower bound on the dominant kernel's own rate" % launches_per_step}
 
 
 def profile_traffic(workload: str):
@@ -183,8 +210,9 @@ def job_throughput(world: int, tokens_per_step: int, steps: int, ms: float) -> f
 class Copy:
     """One replica of the workload's inputs on the device plus its adapter tables."""
 
-    def __init__(self, wl, L, torch, sigma="none", clusters=0, merge=1):
-        from workloads.device import upload_projection
+    def __init__(self, wl, L, torch, sigma="none", clusters=0, merge=1, base_w=None):
+        from workloads.device import np_to_torch, upload_projection
+        self.W = np_to_torch(base_w, wl.dtype).cuda() if base_w is not None else None
         self.projs = []
         self.tables = []
         self.sigma = []
@@ -227,16 +255,26 @@ class Copy:
 
     def nbytes(self):
         tot = self.ids.numel() * 4 + self.ws.numel()
+        if self.W is not None:
+            tot += self.W.numel() * self.W.element_size()
         for d in self.projs:
             tot += d.A_flat.numel() * d.A_flat.element_size() + d.B_flat.numel() * d.B_flat.element_size()
             tot += d.x.numel() * d.x.element_size() + d.y0.numel() * d.y0.element_size()
         return tot
 
 
-def make_step(wl, L, grouped=False, merge=1):
+def make_step(wl, L, grouped=False, merge=1, base=False):
     """Returns (step(copy, stream_handle), launches per step, name of the dominant kernel)."""
     name = wl.name
     T = wl.T
+    if base:
+        if name != "prefill_sgmv":
+            raise SystemExit("--base applies to prefill_sgmv only")
+
+        def step(c, s):
+            d, t = c.projs[0], c.tables[0]
+            L.lora_sgmv_base(t.handle, c.seg, d.x, d.h, c.W, d.h, d.y0, d.o, 0, False, c.ws, c.ws.numel(), s)
+        return step, 2, "base_gemm_kernel (tcgen05, x W^T plus the adapter term in one accumulator)"
     if merge > 1:
         if name != "decode_bgmv":
             raise SystemExit("--merge applies to decode_bgmv only")
@@ -386,6 +424,8 @@ def make_copies(wl, L, torch, args, plain=False):
     """C replicas of the inputs, C chosen so that together they exceed 4x the L2 size (at
     least 2).  `plain` ignores the three-stage / merged options (secondary lines)."""
     kw = {} if plain else dict(sigma=args.sigma, clusters=args.jd_clusters, merge=args.merge)
+    if getattr(args, "base_w", None) is not None and not plain:
+        kw["base_w"] = args.base_w
     first = Copy(wl, L, torch, **kw)
     per = first.nbytes()
     C = args.copies or max(2, min(256, -(-4 * L2_BYTES // per)))
@@ -436,7 +476,51 @@ def secondary_lines(args, L, torch, dist, world):
                     "l2": "rotating %d input copies, %.0f MB in total; 256 MB written between repetitions" % (
                         C, C * per / 1e6),
                     "roofline": roofline_of(b, ms, launches, kname, traffic)})
+    if not args.base:
+        out.append(base_layer_line(args, L, torch, dist, world))
     return out
+
+
+def base_layer_line(args, L, torch, dist, world):
+    """The prefill shape's layer output with a synthetic frozen base weight through
+    lora_sgmv_base (tensor-core bound), and, for comparison only, the same result computed as
+    a library GEMM (torch.matmul) followed by lora_sgmv."""
+    wl = workloads.generate("prefill_sgmv", seed=rank_seed("prefill_sgmv", int(os.environ.get("RANK", "0"))))
+    p0 = wl.projections[0]
+    W = workloads.draw_base_weight(p0.o, p0.h, seed=wl.seed + 500)
+    C = max(2, -(-4 * L2_BYTES // (2 * p0.o * p0.h + 2 * wl.T * (p0.h + p0.o))))
+    copies = [Copy(wl, L, torch, base_w=W) for _ in range(C)]
+    fused, launches, kname = make_step(wl, L, base=True)
+
+    def unfused(c, s):   # comparison only: library GEMM, then the delta
+        d, t = c.projs[0], c.tables[0]
+        with torch.cuda.stream(torch.cuda.ExternalStream(s)):
+            torch.matmul(d.x, c.W.t(), out=d.y0)
+        L.lora_sgmv(t.handle, c.seg, d.x, d.h, d.y0, d.o, 0, c.ws, c.ws.numel(), s)
+
+    res = {}
+    for name, step in (("fused", fused), ("unfused", unfused)):
+        K = C * max(1, -(-8 // C))
+        tm = Timer(torch, copies, step, K, args.no_graph)
+        tm.warm(max(args.warmup, 3))
+        reps = tm.reps_for(0.5)
+        if dist:
+            dist.barrier()
+        res[name] = (max_over_ranks(float(np.median(tm.run(reps))), dist, "cuda") / K, K, reps)
+        tm.release()
+    free_copies(torch, copies)
+    ms, K, reps = res["fused"]
+    flops = accounting.base_layer_flops(wl)
+    return {"workload": "prefill_base: up_proj 4096->14336 layer output x W^T + s B A x with a synthetic frozen W, "
+                        "8 segments x 512 tokens, r64 bf16 (lora_sgmv_base)",
+            "tokens_per_step": wl.T, "value": round(job_throughput(world, wl.T, 1, ms), 1), "unit": UNIT,
+            "ms_per_step": round(ms, 6), "steps": K, "repetitions": reps,
+            "algorithmic_bytes_per_step": accounting.base_layer_bytes(wl),
+            "l2": "rotating %d input copies; 256 MB written between repetitions" % C,
+            "roofline": tensor_roofline(flops, ms, launches, kname),
+            "comparison": {"what": "torch.matmul (cuBLAS) then lora_sgmv, same inputs, same timing",
+                           "ms_per_step": round(res["unfused"][0], 6),
+                           "fused_speedup": round(res["unfused"][0] / ms, 4)}}
 
 
 def adapter_sweep(args, L, torch, dist, world):
@@ -499,7 +583,7 @@ def run_ours(args, rank, world, local_rank):
 
     wl = workloads.generate(args.workload, seed=rank_seed(args.workload, rank))
     T = wl.T
-    step, launches_per_step, kname = make_step(wl, L, args.grouped, args.merge)
+    step, launches_per_step, kname = make_step(wl, L, args.grouped, args.merge, args.base)
     if args.jd_clusters and args.sigma == "none":
         raise SystemExit("--jd-clusters needs --sigma")
     bytes_step = accounting.workload_bytes(wl, shared_x=args.grouped, sigma=args.sigma, clusters=args.jd_clusters)
@@ -507,6 +591,12 @@ def run_ours(args, rank, world, local_rank):
         m_ids, _m_w = workloads.draw_merge(wl.ids, wl.n, args.merge, seed=wl.seed + 99)
         bytes_step = accounting.merged_bytes(wl, m_ids)
     flops_step = accounting.workload_flops(wl)
+    args.base_w = None
+    if args.base:
+        p0 = wl.projections[0]
+        args.base_w = workloads.draw_base_weight(p0.o, p0.h, seed=wl.seed + 500)
+        bytes_step = accounting.base_layer_bytes(wl)
+        flops_step = accounting.base_layer_flops(wl)
     distinct = int(accounting.distinct_adapters(wl.ids).size)
 
     copies, ws_bytes = make_copies(wl, L, torch, args)
@@ -542,8 +632,11 @@ def run_ours(args, rank, world, local_rank):
     value = job_throughput(world, T, K, ms)
     tm.release()
 
-    traffic = profile_traffic(args.workload) if not (args.grouped or args.sigma != "none" or args.merge > 1) else None
+    traffic = profile_traffic(args.workload) if not (args.grouped or args.sigma != "none" or args.merge > 1
+                                                     or args.base) else None
     roofline = roofline_of(bytes_step, ms_step, launches_per_step, kname, traffic)
+    if args.base:
+        roofline = tensor_roofline(flops_step, ms_step, launches_per_step, kname)
 
     # end to end through the C ABI with host buffers: H2D inputs, the call, D2H of y
     e2e = None

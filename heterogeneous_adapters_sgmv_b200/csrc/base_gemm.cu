@@ -60,6 +60,7 @@ struct BaseParams {
     int32_t accumulate;
     uint32_t *status;
     uint64_t wait_ns;
+    int32_t early;                // 1: the shrink was launched just before (see the kernel)
 };
 
 struct __align__(8) BaseCtl {
@@ -153,7 +154,12 @@ __global__ void __launch_bounds__(kBThreads, 1) base_gemm_kernel(const __grid_co
         tmem_alloc(smem_u32(&ctl.tmem_base), 512);   // two 256-column accumulators
         tmem_relinquish();
     }
-    pdl_wait();
+    // Programmatic launch: the shrink that precedes this kernel signals its dependents only
+    // after its own wait on the grid before it, so x, W, y and the segment table are final when
+    // this kernel starts; only the intermediate the shrink writes needs the wait, which the
+    // producer performs before its first adapter k-block.  Without that shrink every thread
+    // waits here.
+    if (!p.early) pdl_wait();
     pdl_launch_dependents();
     if (warp == 0) {
         int r0, rw, ad;
@@ -176,7 +182,7 @@ __global__ void __launch_bounds__(kBThreads, 1) base_gemm_kernel(const __grid_co
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         int cur_g = -1, row0 = 0, rows = 0, a = -1, kbi = 0;
-        bool ok = true, bad = false;
+        bool ok = true, bad = false, waited = !p.early;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const int g = t % MT, nt = t / MT;
             if (g != cur_g) {
@@ -184,6 +190,10 @@ __global__ void __launch_bounds__(kBThreads, 1) base_gemm_kernel(const __grid_co
                 cur_g = g;
             }
             const int nk = nkb + (a >= 0 ? 2 : 0);
+            if (a >= 0 && !waited) {   // the intermediate is the shrink's output
+                pdl_wait();
+                waited = true;
+            }
             for (int kb = 0; kb < nk; ++kb, ++kbi) {
                 const int s = kbi % kBStages, m = kbi / kBStages;
                 if (m >= 1 &&
@@ -326,7 +336,8 @@ static_assert(kBaseSmem <= 227 * 1024, "base GEMM shared memory");
 }  // namespace
 
 int launch_base_gemm(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, const void *W,
-                     int64_t ldw, void *y, int64_t ldy, int32_t y_off, int accumulate, const void *v, cudaStream_t s)
+                     int64_t ldw, void *y, int64_t ldy, int32_t y_off, int accumulate, const void *v, bool after_shrink,
+                     cudaStream_t s)
 {
     BaseParams p;
     std::memset(&p, 0, sizeof p);
@@ -353,6 +364,7 @@ int launch_base_gemm(const lora_table *t, const lora_segments *seg, const void *
     p.accumulate = accumulate;
     p.status = t->d_status;
     p.wait_ns = wait_limit_ns();
+    p.early = (after_shrink && options().pdl) ? 1 : 0;
 
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LORA_ERR_CUDA;

@@ -18,8 +18,8 @@
 //  * Consumer warps load the next tile's x (or y) rows with coalesced 128-bit loads while the
 //    current tile computes.  Shrink: warp-level split-K; a warp owns rank rows k = warp + 8 i, a
 //    lane 16 bytes at two places of each 1 KiB row; two tokens x two rows are formed at once
-//    and folded across the warp by one transposed butterfly (the summation tree of a plain
-//    butterfly, so the blocking does not change results).
+//    (bf16 x bf16 -> fp32 fused multiply-adds straight from the packed words, even and odd
+//    elements in two chains) and folded across the warp by one transposed butterfly.
 //  * Each CTA pushes its partial intermediate into every peer's shared memory with st.async
 //    (completion counted in bytes on the peer's mbarrier); every CTA then sums the CL partials
 //    in fixed CTA order.  No atomics, no grid barrier: bit-identical run to run.  A cluster of
@@ -117,7 +117,8 @@ __host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int 
     const int rowb = row_bytes_for(R);
     l.RP = round_up(R, 8);
     l.ids_off = kCtlBytes;
-    const int ids_bytes = (src == kSrcIds) ? round_up(4 * (3 * T + n), 128) : 0;   // ids, first, leaders, weights
+    // ids, first member and count per adapter, leaders, weights, chunk offsets per group
+    const int ids_bytes = (src == kSrcIds) ? round_up(4 * (4 * T + n + 1), 128) : 0;
     l.xs_off = l.ids_off + ids_bytes;
     l.ys_off = l.xs_off + kTokChunk * rowb;
     l.vpart_off = l.ys_off + kTokChunk * rowb;
@@ -145,6 +146,20 @@ __device__ __forceinline__ void cvt16(const uint4 w, float *o, float *)
 }
 
 __device__ __forceinline__ int ceil_log2(int v) { return v <= 1 ? 0 : 32 - __clz(v - 1); }
+
+// lo += a.lo * b.lo and hi += a.hi * b.hi for packed bf16 pairs, each product taken exactly and
+// added with one rounding (a bf16 x bf16 fused multiply-add into fp32, no unpacking).
+__device__ __forceinline__ void fma_bf16x2(uint32_t a, uint32_t b, float &lo, float &hi)
+{
+    asm("{\n .reg .b16 al, ah, bl, bh;\n"
+        " mov.b32 {al, ah}, %2;\n"
+        " mov.b32 {bl, bh}, %3;\n"
+        " fma.rn.f32.bf16 %0, al, bl, %0;\n"
+        " fma.rn.f32.bf16 %1, ah, bh, %1;\n}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(a), "r"(b));
+}
+
 
 template <typename E, int MODE, int SRC, int CL>
 __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_constant__ DecodeParams p)
@@ -245,13 +260,16 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     };
 
     // Per-token ids: tokens with equal ids form one group.  With no more adapters than
-    // clusters, cluster c owns adapter c and its producer scans the ids itself; otherwise a
-    // group is led by the first token carrying its id and groups are listed in leader order.
+    // clusters and at most two tokens per adapter on average, cluster c owns adapter c and its
+    // producer scans the ids itself.  Otherwise a group is led by the first token carrying its
+    // id, groups are listed in leader order, and their 16-token chunks are numbered group by
+    // group and dealt to the clusters round-robin (so a heavy group spreads over many).
     int32_t *ids_s = reinterpret_cast<int32_t *>(smem + lay.ids_off);
-    int32_t *first = ids_s + p.T;
+    int32_t *first = ids_s + p.T;       // per adapter: first member (low 16 bits), count (high)
     int32_t *leaders = first + p.n;
     float *w_s = reinterpret_cast<float *>(leaders + p.T);   // per-token merge weights (ids form)
-    const bool direct_ids = (SRC == kSrcIds) && p.n <= G;
+    int32_t *chunk0 = reinterpret_cast<int32_t *>(w_s + p.T);   // [groups + 1] first chunk of each group
+    const bool direct_ids = (SRC == kSrcIds) && p.n <= G && p.T <= 2 * p.n;
     // The adapter table is immutable after creation: in direct mode this cluster's descriptor
     // and tensor map are fetched before waiting for the previous grid.
     // The weights are immutable too, so the copies of the first stages of this cluster's
@@ -297,24 +315,45 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                 }
             }
         }
-        for (int i = tid; i < p.n; i += kThreads) first[i] = INT_MAX;
+        for (int i = tid; i < p.n; i += kThreads) first[i] = 0xffff;
         if (__syncthreads_or(bad) && tid == 0 && crank == 0 && cid == 0) atomicOr(p.status, LORA_STATUS_BAD_ID);
         for (int t = tid; t < p.T; t += kThreads) {
             const int32_t a = ids_s[t];
             if (a >= 0 && a < p.n) atomicMin(&first[a], t);
         }
         __syncthreads();
+        for (int t = tid; t < p.T; t += kThreads) {   // member counts in the high half (T <= 1024)
+            const int32_t a = ids_s[t];
+            if (a >= 0 && a < p.n) atomicAdd(&first[a], 1 << 16);
+        }
+        __syncthreads();
         if (warp == 0) {
-            int cnt = 0;
+            int cnt = 0, chunks = 0;
             for (int base = 0; base < p.T; base += 32) {
                 const int t = base + lane;
                 const int32_t a = t < p.T ? ids_s[t] : -1;
-                const bool lead = a >= 0 && a < p.n && first[a] == t;
+                const int32_t f = (a >= 0 && a < p.n) ? first[a] : 0;
+                const bool lead = a >= 0 && a < p.n && (f & 0xffff) == t;
                 const uint32_t m = __ballot_sync(0xffffffffu, lead);
-                if (lead) leaders[cnt + __popc(m & ((1u << lane) - 1u))] = t;
+                const int nch = lead ? ((f >> 16) + kTokChunk - 1) / kTokChunk : 0;
+                int incl = nch;
+#pragma unroll
+                for (int dl = 1; dl < 32; dl <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, dl);
+                    if (lane >= dl) incl += v;
+                }
+                if (lead) {
+                    const int gi = cnt + __popc(m & ((1u << lane) - 1u));
+                    leaders[gi] = t;
+                    chunk0[gi] = chunks + incl - nch;
+                }
                 cnt += __popc(m);
+                chunks += __shfl_sync(0xffffffffu, incl, 31);
             }
-            if (lane == 0) ctl.n_groups = cnt;
+            if (lane == 0) {
+                ctl.n_groups = cnt;
+                chunk0[cnt] = chunks;
+            }
         }
         __syncthreads();
     }
@@ -359,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         const int nseg = (SRC == kSrcSegments) ? min(*p.num_segs, p.max_segs) : 0;
         int sb = -32, ubase = 0, w_p0 = 0, w_p1 = 0, w_sa = -1, w_nu = 0, w_incl = 0, w_total = 0;
         int un = cid;
-        int g = cid, base = -1, cnt = 0;
+        int g = cid, base = -1, cnt = 0, gi = 0;
         for (;;) {
             int a = -1, my_tok = 0, L = 0;
             AdapterDesc d = {};
@@ -376,8 +415,11 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                             w_sa = p.seg_adapter[sg];
                             w_p0 = p.seg_ptr[sg];
                             w_p1 = p.seg_ptr[sg + 1];
-                            if (w_sa >= 0 && w_sa < p.n && w_p0 >= 0 && w_p1 >= w_p0 && w_p1 <= p.T)
-                                w_nu = (w_p1 - w_p0 + kTokChunk - 1) / kTokChunk;
+                            if (w_sa >= 0 && w_sa < p.n && w_p0 >= 0 && w_p1 >= w_p0 && w_p1 <= p.T) {
+                                // a long segment served by the tensor-core kernels has no units here
+                                if (p.long_len == 0 || w_p1 - w_p0 < p.long_len)
+                                    w_nu = (w_p1 - w_p0 + kTokChunk - 1) / kTokChunk;
+                            }
                             else if (cid == 0 && crank == 0)   // every cluster scans every segment
                                 atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
                         }
@@ -413,11 +455,43 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     L = __popc(m);
                     a = sa;
                 }
+            } else if (!direct_ids) {
+                // chunk `un` of the numbering: members 16 k .. 16 k + 15 of group gi, in batch
+                // order, found by scanning the ids from the group's first member
+                const int ng = ctl.n_groups;
+                if (un < chunk0[ng]) {
+                    while (chunk0[gi + 1] <= un) ++gi;
+                    const int t0 = leaders[gi];
+                    const int ga = ids_s[t0];
+                    int skip = (un - chunk0[gi]) * kTokChunk;
+                    int c = 0;
+                    for (int bs = t0; bs < p.T && c < kTokChunk; bs += 32) {
+                        const int t = bs + lane;
+                        const uint32_t m = __ballot_sync(0xffffffffu, t < p.T && ids_s[t] == ga);
+                        const int pc = __popc(m);
+                        if (skip >= pc) {
+                            skip -= pc;
+                            continue;
+                        }
+                        const int take = min(pc - skip, kTokChunk - c);
+                        const int rk = __popc(m & ((1u << lane) - 1u)) - skip;
+                        if (((m >> lane) & 1u) && rk >= 0 && rk < take) ctl.pending[c + rk] = t;
+                        c += take;
+                        skip = 0;
+                    }
+                    __syncwarp();
+                    my_tok = ctl.pending[lane & (kTokChunk - 1)];
+                    __syncwarp();
+                    L = c;
+                    a = ga;
+                    d = p.pj[0].desc[ga];
+                    un += G;
+                }
             } else {
-                const int ng = direct_ids ? min(p.n, cid + 1) : ctl.n_groups;
+                const int ng = min(p.n, cid + 1);
                 while (g < ng && L == 0) {
-                    const int t0 = direct_ids ? 0 : leaders[g];
-                    const int ga = direct_ids ? g : ids_s[t0];
+                    const int t0 = 0;
+                    const int ga = g;
                     if (base < 0) base = t0;
                     // gather up to kTokChunk members of group g, resuming at `base`
                     while (base < p.T && cnt < kTokChunk) {
@@ -441,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         my_tok = ctl.pending[lane & (kTokChunk - 1)];
                         L = cnt;
                         a = ga;
-                        d = direct_ids ? pre_desc : p.pj[0].desc[ga];
+                        d = pre_desc;
                     }
                     __syncwarp();
                     cnt = 0;
@@ -619,7 +693,51 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             // its 16 elements, and one transposed butterfly folds all four across the warp.
             const bool okA = lane < nch, okB = lane + 32 < nch;
             const uint4 z = make_uint4(0, 0, 0, 0);
-            if (warp < r) {
+            if (ESZ == 2 && warp < r) {
+                for (int l = 0; l < L; l += 2) {
+                    const bool l2 = l + 1 < L;
+                    const uint8_t *xr0 = xs + l * rowb, *xr1 = xr0 + rowb;
+                    const uint4 x00 = okA ? *reinterpret_cast<const uint4 *>(xr0 + lane * 16) : z;
+                    const uint4 x01 = okB ? *reinterpret_cast<const uint4 *>(xr0 + 512 + lane * 16) : z;
+                    const uint4 x10 = l2 && okA ? *reinterpret_cast<const uint4 *>(xr1 + lane * 16) : z;
+                    const uint4 x11 = l2 && okB ? *reinterpret_cast<const uint4 *>(xr1 + 512 + lane * 16) : z;
+                    const uint32_t xw0[8] = {x00.x, x00.y, x00.z, x00.w, x01.x, x01.y, x01.z, x01.w};
+                    const uint32_t xw1[8] = {x10.x, x10.y, x10.z, x10.w, x11.x, x11.y, x11.z, x11.w};
+                    for (int k = warp; k < r; k += 2 * kConsumerWarps) {
+                        const bool k2 = k + kConsumerWarps < r;
+                        float p[4];
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const uint8_t *row = data + (k + q * kConsumerWarps) * kBoxBytes;
+                            const bool ok = q == 0 || k2;
+                            const uint4 a0 = ok && okA ? *reinterpret_cast<const uint4 *>(row + lane * 16) : z;
+                            const uint4 a1 = ok && okB ? *reinterpret_cast<const uint4 *>(row + r * kBoxBytes + lane * 16) : z;
+                            const uint32_t aw[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                            float s0 = 0.f, s1 = 0.f, t0 = 0.f, t1 = 0.f;
+#pragma unroll
+                            for (int w = 0; w < 8; ++w) {
+                                fma_bf16x2(xw0[w], aw[w], s0, s1);
+                                fma_bf16x2(xw1[w], aw[w], t0, t1);
+                            }
+                            p[q] = s0 + s1;
+                            p[2 + q] = t0 + t1;
+                        }
+                        const bool hi16 = lane & 16, hi8 = lane & 8;
+                        float k0 = hi16 ? p[2] : p[0], k1 = hi16 ? p[3] : p[1];
+                        k0 += __shfl_xor_sync(0xffffffffu, hi16 ? p[0] : p[2], 16);
+                        k1 += __shfl_xor_sync(0xffffffffu, hi16 ? p[1] : p[3], 16);
+                        float tot = hi8 ? k1 : k0;
+                        tot += __shfl_xor_sync(0xffffffffu, hi8 ? k0 : k1, 8);
+                        tot += __shfl_xor_sync(0xffffffffu, tot, 4);
+                        tot += __shfl_xor_sync(0xffffffffu, tot, 2);
+                        tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+                        if ((lane & 7) == 0 && (!hi16 || l2) && (!hi8 || k2)) {
+                            float *dst = vpart + (l + (hi16 ? 1 : 0)) * RP + k + (hi8 ? kConsumerWarps : 0);
+                            *dst = first ? tot : *dst + tot;
+                        }
+                    }
+                }
+            } else if (warp < r) {
                 for (int l = 0; l < L; l += 2) {
                     const bool l2 = l + 1 < L;
                     const uint8_t *xr0 = xs + l * rowb, *xr1 = xr0 + rowb;
@@ -999,8 +1117,7 @@ template <typename E, int MODE, int SRC>
 int launch_mode(const DecodeParams &p, cudaStream_t s)
 {
     // units: an upper bound on the work units (16-token chunks of one adapter's tokens)
-    const int units = max(1, (SRC == kSrcSegments) ? min(p.T, p.max_segs + (p.T + kTokChunk - 1) / kTokChunk)
-                                                   : min(p.T, p.n));
+    const int units = max(1, min(p.T, ((SRC == kSrcSegments) ? p.max_segs : p.n) + (p.T + kTokChunk - 1) / kTokChunk));
     const int64_t forced = options().decode_cluster;
     int CL = (forced == 1 || forced == 2 || forced == 4) ? (int)forced : kMaxCluster;
     // The widest width whose pipeline fits in shared memory (the partial-exchange buffers grow

@@ -33,6 +33,8 @@ Options &options()
         o.prefill_min_seg_len = env_or("LORA_PREFILL_MIN_SEG_LEN", o.prefill_min_seg_len);
         o.prefill_ksplit = env_or("LORA_PREFILL_KSPLIT", o.prefill_ksplit);
         o.split = env_or("LORA_SPLIT", o.split);
+        o.tc_min_seg_len = env_or("LORA_TC_MIN_SEG_LEN", o.tc_min_seg_len);
+        o.tc_min_tokens = env_or("LORA_TC_MIN_TOKENS", o.tc_min_tokens);
     });
     return o;
 }
@@ -46,7 +48,7 @@ uint64_t wait_limit_ns()
 // prefill.cu
 bool prefill_supported(const lora_table *t);
 int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y,
-                   int64_t ldy, int32_t y_off, void *v, cudaStream_t s);
+                   int64_t ldy, int32_t y_off, void *v, int32_t min_len, cudaStream_t s);
 
 }  // namespace lora
 
@@ -359,7 +361,7 @@ int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int6
         if (!ws || ws_bytes < w.total) return LORA_ERR_WORKSPACE;
         if (!al16(ws)) return LORA_ERR_UNSUPPORTED;
         float *v = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + w.v);
-        if (prefill) return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, s);
+        if (prefill) return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, 0, s);
         if ((rc = lora_shrink(t, seg, x, ldx, v, ldv_of(t), stream))) return rc;
         return lora_expand(t, seg, v, ldv_of(t), y, ldy, y_off, stream);
     }
@@ -370,7 +372,16 @@ int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int6
     p.pj[0].y = y;
     p.pj[0].ldy = ldy;
     p.pj[0].y_off = y_off;
-    return launch_decode(kModeFused, kSrcSegments, p, t->dtype, s);
+    // Mixed batches (segments of any length, in any token order, e.g. from lora_build_segments):
+    // in a batch of at least "tc_min_tokens" tokens the segments of at least "tc_min_seg_len"
+    // tokens go to the tcgen05 kernels (rows gathered through perm), the shorter ones to the
+    // decode kernel.  Both read the same segment table and split it by length on the device.
+    const bool mixed = opt.tc_min_seg_len > 0 && seg->T >= opt.tc_min_tokens && prefill_supported(t) && ws &&
+                       ws_bytes >= ws_layout(t, seg->T).total && al16(ws);
+    if (mixed) p.long_len = (int32_t)opt.tc_min_seg_len;
+    if ((rc = launch_decode(kModeFused, kSrcSegments, p, t->dtype, s)) != LORA_OK || !mixed) return rc;
+    float *v = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_layout(t, seg->T).v);
+    return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, (int32_t)opt.tc_min_seg_len, s);
 }
 
 int lora_sgmv_base(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, const void *W,
@@ -392,8 +403,9 @@ int lora_sgmv_base(const lora_table *t, const lora_segments *seg, const void *x,
     if (!al16(ws)) return LORA_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void *v = static_cast<uint8_t *>(ws) + w.v;
-    if (seg->max_segs > 0 && (rc = launch_prefill_shrink(t, seg, x, ldx, v, true, s)) != LORA_OK) return rc;
-    return launch_base_gemm(t, seg, x, ldx, W, ldw, y, ldy, y_off, accumulate, v, s);
+    const bool shrink = seg->max_segs > 0;
+    if (shrink && (rc = launch_prefill_shrink(t, seg, x, ldx, v, true, s)) != LORA_OK) return rc;
+    return launch_base_gemm(t, seg, x, ldx, W, ldw, y, ldy, y_off, accumulate, v, shrink, s);
 }
 
 int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_segments *seg,
@@ -606,6 +618,8 @@ int lora_set_option(const char *key, int64_t value)
     else if (!std::strcmp(key, "split")) o.split = value;
     else if (!std::strcmp(key, "wait_limit_ns")) o.wait_limit_ns = value;
     else if (!std::strcmp(key, "inject_stall")) o.inject_stall = value;
+    else if (!std::strcmp(key, "tc_min_seg_len")) o.tc_min_seg_len = value;
+    else if (!std::strcmp(key, "tc_min_tokens")) o.tc_min_tokens = value;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }
@@ -624,6 +638,8 @@ int lora_get_option(const char *key, int64_t *value)
     else if (!std::strcmp(key, "split")) *value = o.split;
     else if (!std::strcmp(key, "wait_limit_ns")) *value = o.wait_limit_ns;
     else if (!std::strcmp(key, "inject_stall")) *value = o.inject_stall;
+    else if (!std::strcmp(key, "tc_min_seg_len")) *value = o.tc_min_seg_len;
+    else if (!std::strcmp(key, "tc_min_tokens")) *value = o.tc_min_tokens;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }

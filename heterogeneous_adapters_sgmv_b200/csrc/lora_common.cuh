@@ -128,12 +128,17 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // Bounded waits: false after `limit_ns` of %globaltimer, with LORA_STATUS_TIMEOUT latched into
 // *status.  The fast path (phase already complete) is inlined; the polling loop is a separate
 // function so the hot code stays small (instruction-cache misses dominate short kernels).
+// Between probes the warp sleeps (32 ns doubling to 512 ns), so waiting warps do not take issue
+// slots from the warps that are working, and the clock is read only once per probe.
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint32_t *status, bool cluster,
                                                    uint64_t limit_ns)
 {
     const uint64_t t0 = globaltimer_ns();
+    uint32_t pause = 32;
     for (;;) {
         if (cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        __nanosleep(pause);
+        pause = pause < 512 ? 2 * pause : 512;
         if (globaltimer_ns() - t0 > limit_ns) {
             atomicOr(status, LORA_STATUS_TIMEOUT);
             return false;

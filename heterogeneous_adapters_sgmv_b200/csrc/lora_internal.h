@@ -49,6 +49,7 @@ struct DecodeParams {
     uint32_t *status;
     uint64_t wait_ns;      // bound of every device-side wait (option "wait_limit_ns")
     int32_t inject;        // test-only stall injection (option "inject_stall"), 0 in normal use
+    int32_t long_len;      // segments of at least this many tokens are served elsewhere (0: none)
     int32_t stages;        // pipeline depth
     int32_t stage_bytes;   // bytes of one stage (header + data)
     int32_t ids_smem;      // kSrcIds: bytes of the id / leader scratch in shared memory
@@ -65,6 +66,8 @@ struct Options {
     int64_t split = 0;
     int64_t wait_limit_ns = 0;       // 0: the default bound (about 2 s)
     int64_t inject_stall = 0;        // test-only: bit 0 decode, bit 1 prefill shrink, bit 2 prefill expand
+    int64_t tc_min_seg_len = 64;     // mixed batches: segments this long take the tcgen05 kernels (0: never)
+    int64_t tc_min_tokens = 1024;    // ... in batches of at least this many tokens
 };
 // Bound of the device-side waits for the next launch.
 uint64_t wait_limit_ns();
@@ -82,8 +85,11 @@ int launch_prefill_shrink(const lora_table *t, const lora_segments *seg, const v
                           bool fold_scale, cudaStream_t s);
 // Fused layer output (base_gemm.cu): y = (y if accumulate) + x W^T + the adapter term, from the
 // scale-folded intermediate v that launch_prefill_shrink wrote.
+// after_shrink: launch_prefill_shrink was the launch just before on `s` (lets the kernel start
+// its base-product tiles before the shrink has finished).
 int launch_base_gemm(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, const void *W,
-                     int64_t ldw, void *y, int64_t ldy, int32_t y_off, int accumulate, const void *v, cudaStream_t s);
+                     int64_t ldw, void *y, int64_t ldy, int32_t y_off, int accumulate, const void *v, bool after_shrink,
+                     cudaStream_t s);
 // Encode the TMA tensor map of A_i [rank, h] used by the decode shrink (host side).
 int encode_tmap_A(void *out128, const void *A, int dtype, int h, int rank);
 

@@ -24,6 +24,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -60,7 +61,43 @@ struct PrefillParams {
     uint64_t wait_ns;             // bound of every device-side wait
     int32_t inject;               // test-only stall injection: bit 1 shrink, bit 2 expand
     int32_t fold_scale;           // shrink: store s_i * v instead of v (fused base product)
+    const int32_t *perm;          // token of each sorted position, or null (tokens contiguous)
+    int32_t min_len;              // only segments of at least this many tokens (0: all)
+    CUtensorMap tmap_g;           // perm: x [T, h] (shrink) or the y slice (expand), box 64 x 1
 };
+
+// 4-row gather (TMA tile::gather4, one-row box, 128-byte swizzle) of columns [c0, c0 + 64) of
+// rows r0..r3 into 512 bytes of shared memory, counted on `bar`.  The rows land exactly as
+// rows 4k .. 4k + 3 of a tiled box would at the same shared-memory offset.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, int32_t c0, int32_t r0, int32_t r1,
+                                            int32_t r2, int32_t r3, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(tmap), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+        : "memory");
+}
+
+// Tokens of rows 4 lane .. 4 lane + 3 of a tile at sorted positions [row0, row0 + rows): rows
+// past the tile repeat its last row (their results are never stored); an entry outside [0, T)
+// latches LORA_STATUS_BAD_SEGMENT and reads row 0 instead.
+__device__ __forceinline__ void tile_tokens(const PrefillParams &p, int row0, int rows, int tk[4])
+{
+    const int lane = threadIdx.x & 31;
+    bool bad = false;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int r = min(4 * lane + q, rows - 1);
+        int t = p.perm[row0 + r];
+        if (t < 0 || t >= p.T) {
+            bad = true;
+            t = 0;
+        }
+        tk[q] = t;
+    }
+    if (bad) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+}
 
 // Map a global 128-token tile index to (segment, first row, rows).  One warp scans the
 // segment table; returns false when the index is past the last tile.
@@ -73,6 +110,7 @@ __device__ bool find_tile(const PrefillParams &p, int g, int *seg, int *row0, in
         const int s = s0 + lane;
         int len = 0;
         if (s < nseg) len = max(0, min(p.seg_ptr[s + 1], p.T) - max(p.seg_ptr[s], 0));   // bad bounds: empty
+        if (len < p.min_len) len = 0;   // a short segment is served by the decode kernel
         const int tiles = (len + kTileM - 1) / kTileM;
         int incl = tiles;
 #pragma unroll
@@ -170,31 +208,41 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     bool ok = true;
 
     if (valid && nkb > 0) {
-        if (warp == 0 && lane == 0) {
-            // producer: x tile (128 tokens x 64 columns) and A_i tile (npad rows x 64 columns)
+        if (warp == 0) {
+            // producer: x tile (128 tokens x 64 columns) and A_i tile (npad rows x 64 columns);
+            // with a permutation each lane gathers four of the tile's token rows
             const void *tA = p.tm_A + (size_t)a * 128;
             const uint32_t bytes = (uint32_t)(kXBytes + npad * 128);
+            int tk[4] = {0, 0, 0, 0};
+            if (p.perm) tile_tokens(p, row0, rows, tk);
             int issued = 0;
             bool stalled = false;
             for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kStages, m = kb / kStages;
-                if (m >= 1 && !mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status, p.wait_ns)) {
+                if (m >= 1 &&
+                    !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status, p.wait_ns))) {
                     stalled = true;
                     break;
                 }
                 uint8_t *st = smem + s * kStageBytes;
                 const uint32_t fb = smem_u32(&ctl.full[s]);
-                mbar_arrive_expect_tx(fb, bytes);
                 ++issued;
-                // test-only stall: the first k-block is armed but never loaded
-                if ((p.inject & 2) && kb == 0) continue;
                 const int k0 = (kb0 + kb) * kBK;
-                tma_load_2d(smem_u32(st), &p.tmap_io, k0, row0, fb);
-                tma_load_2d(smem_u32(st + kXBytes), tA, k0, 0, fb);
+                // test-only stall: the first k-block is armed but never loaded
+                const bool load = !((p.inject & 2) && kb == 0);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(fb, bytes);
+                    if (load) {
+                        if (!p.perm) tma_load_2d(smem_u32(st), &p.tmap_io, k0, row0, fb);
+                        tma_load_2d(smem_u32(st + kXBytes), tA, k0, 0, fb);
+                    }
+                }
+                __syncwarp();
+                if (p.perm && load) tma_gather4(smem_u32(st + lane * 512), &p.tmap_g, k0, tk[0], tk[1], tk[2], tk[3], fb);
             }
             // After a timeout the ring is given up early: wait (bounded) for the copies of the
             // last stages issued, so none is still writing when the ring is reused below.
-            if (stalled || (p.inject & 2))
+            if (lane == 0 && (stalled || (p.inject & 2)))
                 for (int kb = max(0, issued - kStages); kb < issued; ++kb)
                     mbar_wait(smem_u32(&ctl.full[kb % kStages]), (kb / kStages) & 1, p.status, p.wait_ns);
         } else if (warp == 1 && lane == 0) {
@@ -325,6 +373,7 @@ __device__ int count_m_tiles(const PrefillParams &p)
         const int s = s0 + lane;
         int len = 0;
         if (s < nseg) len = max(0, min(p.seg_ptr[s + 1], p.T) - max(p.seg_ptr[s], 0));
+        if (len < p.min_len) len = 0;
         int tiles = (len + kTileM - 1) / kTileM;
 #pragma unroll
         for (int d = 16; d >= 1; d >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, d);
@@ -380,6 +429,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         int cur_g = -1, vcount = 0, row0 = 0, rows = 0, a = 0, vb = 0, nissued = 0;
+        int tk[4] = {0, 0, 0, 0};   // with a permutation: tokens of rows 4 lane .. 4 lane + 3
         float sc = 0.f;
         for (int t = t0; t < t1 && ok; ++t) {
             const int i = t - t0, s = i % kExStages;
@@ -395,6 +445,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 }
                 sc = p.desc[a].scale;
                 cur_g = g;
+                if (p.perm && rows > 0) tile_tokens(p, row0, rows, tk);
                 vb = vcount & 1;
                 if (vcount >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.vempty[vb]),
                                                                      ((vcount >> 1) - 1) & 1, p.status, p.wait_ns))) {
@@ -432,9 +483,18 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 // test-only stall: the first tile's stage is armed but never loaded
                 if (!((p.inject & 4) && i == 0)) {
                     tma_load_2d(smem_u32(st), p.tm_B + (size_t)a * 128, 0, nt * kTileN, fb);
-                    tma_load_2d(smem_u32(st + 16384), &p.tmap_io, nt * kTileN, row0, fb);
-                    tma_load_2d(smem_u32(st + 32768), &p.tmap_io, nt * kTileN + 64, row0, fb);
+                    if (!p.perm) {
+                        tma_load_2d(smem_u32(st + 16384), &p.tmap_io, nt * kTileN, row0, fb);
+                        tma_load_2d(smem_u32(st + 32768), &p.tmap_io, nt * kTileN + 64, row0, fb);
+                    }
                 }
+            }
+            __syncwarp();
+            if (p.perm && !((p.inject & 4) && i == 0)) {   // the y tile's rows, four per lane
+                const uint32_t st = smem_u32(ring + s * kExStageBytes);
+                const uint32_t fb = smem_u32(&ctl.full[s]);
+                tma_gather4(st + 16384 + lane * 512, &p.tmap_g, nt * kTileN, tk[0], tk[1], tk[2], tk[3], fb);
+                tma_gather4(st + 32768 + lane * 512, &p.tmap_g, nt * kTileN + 64, tk[0], tk[1], tk[2], tk[3], fb);
             }
             ++nissued;
             __syncwarp();
@@ -521,7 +581,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&ctl.accempty[ab]));
             named_bar_sync(2, kEpiWarps * 32);   // the whole tile is updated in shared memory
-            const bool full_tile = inf.rows == kTileM && inf.ncols == kTileN;
+            const bool full_tile = !p.perm && inf.rows == kTileM && inf.ncols == kTileN;
             if (full_tile) {
                 // a full tile lies inside one segment: two TMA stores write it back
                 if (ew == 0 && lane == 0) {
@@ -534,15 +594,18 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             } else {
                 // coalesced stores masked to the segment's rows and to o: epilogue warp ew stores
                 // rows 16 ew .. 16 ew + 15, two per step
+                // (with a permutation, row rr of the tile is token perm[row0 + rr])
                 uint8_t *yg = static_cast<uint8_t *>(p.y);
                 const int chunk = lane & 15;
 #pragma unroll 1
                 for (int rr = ew * 16 + (lane >> 4); rr < ew * 16 + 16; rr += 2) {
                     if (rr < inf.rows && chunk * 8 < inf.ncols) {
+                        const int tok = p.perm ? p.perm[inf.row0 + rr] : inf.row0 + rr;
+                        if (tok < 0 || tok >= p.T) continue;   // latched when the rows were gathered
                         const uint8_t *box = ring + s * kExStageBytes + 16384 + (chunk >= 8 ? 16384 : 0);
                         const uint4 w = *reinterpret_cast<const uint4 *>(box + sw128_off(rr, chunk & 7));
                         *reinterpret_cast<uint4 *>(
-                            yg + ((int64_t)(inf.row0 + rr) * p.ldy + p.y_off + inf.col0 + chunk * 8) * 2) = w;
+                            yg + ((int64_t)tok * p.ldy + p.y_off + inf.col0 + chunk * 8) * 2) = w;
                     }
                 }
             }
@@ -595,6 +658,14 @@ int prefill_build_maps(lora_table *t)
 
 namespace {
 
+// Upper bound of the 128-token tiles of the segments with at least min_len tokens: one partial
+// tile per segment at most, and no more such segments than T / min_len.
+int tile_bound(const lora_segments *seg, int min_len)
+{
+    const int segs = min_len > 0 ? std::min(seg->max_segs, seg->T / min_len) : seg->max_segs;
+    return segs + (seg->T + kTileM - 1) / kTileM;
+}
+
 PrefillParams prefill_params(const lora_table *t, const lora_segments *seg, void *v)
 {
     PrefillParams p;
@@ -615,6 +686,7 @@ PrefillParams prefill_params(const lora_table *t, const lora_segments *seg, void
     p.status = t->d_status;
     p.wait_ns = wait_limit_ns();
     p.inject = (int32_t)(options().inject_stall & 6);
+    p.perm = seg->perm;
     return p;
 }
 
@@ -642,9 +714,12 @@ int launch_shrink_kernel(PrefillParams &p, const lora_table *t, const lora_segme
                          cudaStream_t s)
 {
     const Options &opt = options();
-    const int mt_bound = seg->max_segs + (seg->T + kTileM - 1) / kTileM;
+    const int mt_bound = tile_bound(seg, p.min_len);
     int rc = encode_sw128(&p.tmap_io, x, (uint64_t)t->h, (uint64_t)seg->T, (uint64_t)ldx, kTileM);
     if (rc != LORA_OK) return rc;
+    // with a permutation the x rows are gathered four at a time (one-row boxes)
+    if (p.perm && (rc = encode_sw128(&p.tmap_g, x, (uint64_t)t->h, (uint64_t)seg->T, (uint64_t)ldx, 1)) != LORA_OK)
+        return rc;
     cudaLaunchConfig_t cfg = {};
     const int KS = opt.prefill_ksplit == 8 ? 8 : 4;
     cfg.gridDim = dim3(KS * mt_bound);
@@ -683,7 +758,7 @@ int launch_prefill_shrink(const lora_table *t, const lora_segments *seg, const v
 }
 
 int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y, int64_t ldy,
-                   int32_t y_off, void *v, cudaStream_t s)
+                   int32_t y_off, void *v, int32_t min_len, cudaStream_t s)
 {
     if (!prefill_supported(t)) return LORA_ERR_UNSUPPORTED;
     int rc = set_prefill_attributes();
@@ -692,7 +767,8 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
     p.y = y;
     p.ldy = ldy;
     p.y_off = y_off;
-    const int mt_bound = seg->max_segs + (seg->T + kTileM - 1) / kTileM;
+    p.min_len = min_len;
+    const int mt_bound = tile_bound(seg, min_len);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LORA_ERR_CUDA;
     const Options &opt = options();
@@ -704,6 +780,9 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
     rc = encode_sw128(&p.tmap_io, static_cast<uint8_t *>(y) + (int64_t)y_off * 2, (uint64_t)t->o, (uint64_t)seg->T,
                       (uint64_t)ldy, kTileM);
     if (rc != LORA_OK) return rc;
+    if (p.perm && (rc = encode_sw128(&p.tmap_g, static_cast<uint8_t *>(y) + (int64_t)y_off * 2, (uint64_t)t->o,
+                                     (uint64_t)seg->T, (uint64_t)ldy, 1)) != LORA_OK)
+        return rc;
     {
         cudaLaunchConfig_t cfg = {};
         static int n_sms[64];

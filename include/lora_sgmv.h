@@ -156,12 +156,19 @@ int lora_expand(const lora_table *table, const lora_segments *seg, const float *
                 int32_t ldv, void *y, int64_t ldy, int32_t y_offset, void *stream);
 
 /* SGMV: shrink and expand for sorted segments, in place on the y slice.  Picks the path:
- * the fused cluster kernel (decode), or the tcgen05 tensor-core path (prefill) when the hint
- * max_seg_len reaches the "prefill_min_seg_len" option (256), perm is NULL, the table is
- * bf16 with every rank a multiple of 8 and at most 64, and it carries no Sigma.  The
- * tcgen05 path keeps its intermediate (bf16 hi + lo) in the workspace; the fused kernel
- * needs none, so ws may be NULL when ws_bytes is 0 and the chosen path needs none;
- * otherwise ws_bytes >= lora_workspace_bytes(table, seg->T). */
+ *  - the tcgen05 tensor-core path (prefill) for every segment when the hint max_seg_len
+ *    reaches the "prefill_min_seg_len" option (256), perm is NULL, and the table is
+ *    tensor-core capable (bf16, every rank a multiple of 8 and at most 64, no Sigma);
+ *  - otherwise, in a batch of at least "tc_min_tokens" (1024) tokens on a tensor-core capable
+ *    table with the workspace given, a split decided on the device from the segment lengths:
+ *    segments of at least "tc_min_seg_len" (64) tokens run on the tcgen05 kernels, which
+ *    gather their token rows through perm (TMA four-row gathers), and the shorter ones on the
+ *    fused cluster kernel; both launches read the same segment table;
+ *  - otherwise every segment runs on the fused cluster kernel (decode).
+ * The tcgen05 kernels keep their intermediate (bf16 hi + lo) in the workspace; the fused
+ * kernel needs none, so ws may be NULL when ws_bytes is 0 (every segment then runs on the
+ * fused kernel); a path that needs the workspace requires ws_bytes >=
+ * lora_workspace_bytes(table, seg->T). */
 int lora_sgmv(const lora_table *table, const lora_segments *seg, const void *x, int64_t ldx,
               void *y, int64_t ldy, int32_t y_offset, void *ws, size_t ws_bytes, void *stream);
 
@@ -265,8 +272,10 @@ const char *lora_status_string(int code);
  * (tests only: a bit mask, 1 decode kernels, 2 tcgen05 shrink, 4 tcgen05 expand, that arms one
  * pipeline stage per unit or tile without ever loading it, so the bounded wait on it runs
  * out, LORA_STATUS_TIMEOUT is latched and the kernel drains its copies, releases tensor
- * memory and returns; results are then invalid).  Returns LORA_ERR_INVALID_ARG for an
- * unknown key. */
+ * memory and returns; results are then invalid), "tc_min_seg_len" (segments at least this
+ * long take the tcgen05 kernels in mixed batches; 0 disables that split), "tc_min_tokens"
+ * (smallest batch that considers the split).  Returns LORA_ERR_INVALID_ARG for an unknown
+ * key. */
 int lora_set_option(const char *key, int64_t value);
 int lora_get_option(const char *key, int64_t *value);
 

@@ -110,3 +110,24 @@ class DeviceProj:
     def to_np(self, y):
         torch.cuda.synchronize()
         return torch_to_np(y, self.dtype)
+
+
+def kernels_launched(fn, tries: int = 3) -> set:
+    """Names of the CUDA kernels that ran during fn() (torch profiler, device events).  A
+    profiler session late in a long process can come back with no device events at all; the
+    session is then repeated (fn must tolerate being called again)."""
+    from torch.profiler import ProfilerActivity, profile
+    names = set()
+    for _ in range(tries):
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA], acc_events=True) as prof:
+            fn()
+            torch.cuda.synchronize()
+        names = {e.name for e in prof.events() if e.device_type.name == "CUDA"}
+        if names:
+            break
+    return names
+
+
+def ran(names: set, kernel: str) -> bool:
+    return any(kernel in k for k in names)

@@ -12,7 +12,7 @@ import torch
 import heterogeneous_adapters_sgmv_b200 as L
 import oracle
 import workloads
-from tests.gpu_util import DeviceProj, assert_close
+from tests.gpu_util import DeviceProj, assert_close, kernels_launched, ran
 from workloads.device import np_to_torch
 
 pytestmark = pytest.mark.gpu
@@ -90,11 +90,9 @@ def test_base_accumulate_into_zero_is_bit_identical_and_kernels_run():
     dp = DeviceProj(wl)
     seg, _keep = _contiguous(seg_ptr, seg_ad, wl.T, wl.n)
     W = np_to_torch(workloads.draw_base_weight(512, 512, seed=6), "bf16").cuda()
-    with torch.profiler.profile(activities=[torch.profiler.ProfilerActivity.CUDA]) as prof:
-        a = _run(dp, seg, W, False)
-        torch.cuda.synchronize()
-    names = {e.key for e in prof.key_averages()}
-    assert any("base_gemm_kernel" in k for k in names) and any("prefill_shrink_kernel" in k for k in names)
+    names = kernels_launched(lambda: _run(dp, seg, W, False))
+    assert ran(names, "base_gemm_kernel") and ran(names, "prefill_shrink_kernel")
+    a = _run(dp, seg, W, False)
     b = _run(dp, seg, W, True, y=torch.zeros_like(dp.d.y0))
     assert torch.equal(a, b)
     # run to run bit-identical

@@ -8,7 +8,7 @@ import torch
 import heterogeneous_adapters_sgmv_b200 as L
 import oracle
 import workloads
-from tests.gpu_util import DeviceProj, assert_close, option, reference, workload
+from tests.gpu_util import DeviceProj, assert_close, kernels_launched, option, reference, workload
 from workloads import to_float64
 
 pytestmark = pytest.mark.gpu
@@ -441,14 +441,6 @@ def _prefill_case(seg_lens, h, o, ranks, seed=5, delta_only=False):
     return wl, dp, seg, (ptr, ad, num)
 
 
-def _kernels_launched(fn):
-    from torch.profiler import ProfilerActivity, profile
-    with profile(activities=[ProfilerActivity.CUDA]) as prof:
-        fn()
-        torch.cuda.synchronize()
-    return {e.name for e in prof.events() if e.device_type.name == "CUDA"}
-
-
 @pytest.mark.parametrize("seg_lens,h,o,ranks", [
     ([300], 512, 256, (16,)),
     ([130, 100, 700, 1, 256], 1024, 384, (64, 8, 32, 16, 64)),
@@ -460,9 +452,9 @@ def test_prefill_tcgen05_ragged_segments_and_ranks(seg_lens, h, o, ranks):
     path within tolerance, and it is the path that ran."""
     wl, dp, seg, _keep = _prefill_case(seg_lens, h, o, ranks)
     ref = oracle.workload_reference(wl)
-    y = dp.y()
-    names = _kernels_launched(lambda: dp.sgmv(y, seg))
+    names = kernels_launched(lambda: dp.sgmv(dp.y(), seg))
     assert any("prefill_expand_kernel" in k for k in names) and any("prefill_shrink_kernel" in k for k in names)
+    y = dp.sgmv(dp.y(), seg)
     assert_close(dp.to_np(y), ref, wl.dtype, "tcgen05 prefill")
     L.lora_set_option("prefill_min_seg_len", 0)
     try:

@@ -8,7 +8,7 @@ import torch
 import heterogeneous_adapters_sgmv_b200 as L
 import oracle
 import workloads
-from tests.gpu_util import DeviceProj, assert_close, option, workload
+from tests.gpu_util import DeviceProj, assert_close, kernels_launched, option, workload
 from workloads.device import torch_to_np, upload_projection
 
 pytestmark = pytest.mark.gpu
@@ -144,11 +144,9 @@ def test_sigma_long_segments_take_the_decode_kernels():
     seg_ptr = torch.arange(0, T + 1, 300, dtype=torch.int32, device="cuda")
     seg = L.make_segments(None, seg_ptr, torch.arange(n, dtype=torch.int32, device="cuda"),
                           torch.tensor([n], dtype=torch.int32, device="cuda"), T, n, 300)
-    with torch.profiler.profile(activities=[torch.profiler.ProfilerActivity.CUDA]) as prof:
-        y = dp.sgmv(dp.y(), seg)
-        torch.cuda.synchronize()
-    names = " ".join(e.name for e in prof.events())
+    names = " ".join(kernels_launched(lambda: dp.sgmv(dp.y(), seg)))
     assert "prefill" not in names and "lora_decode_kernel" in names
+    y = dp.sgmv(dp.y(), seg)
     assert_close(dp.to_np(y), ref, wl.dtype, "sigma long segments")
 
 

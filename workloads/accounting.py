@@ -81,3 +81,19 @@ def adapter_bytes(shapes: Sequence[Tuple[int, int]], rank: int, layers: int, e: 
     """Storage of one adapter: for every adapted (h -> o) projection of every layer,
     A is r x h and B is o x r."""
     return layers * sum(rank * (h + o) * e for (h, o) in shapes)
+
+
+def base_layer_bytes(wl) -> int:
+    """Algorithmic bytes of the layer output with a frozen base weight (projection 0, y written
+    and not read): x once, W [o, h] once, y written once, every distinct touched adapter once."""
+    e = ELEM_BYTES[wl.dtype]
+    p = wl.projections[0]
+    d = distinct_adapters(wl.ids)
+    return wl.T * p.h * e + p.o * p.h * e + wl.T * p.o * e + sum(int(p.ranks[i]) * (p.h + p.o) * e for i in d)
+
+
+def base_layer_flops(wl) -> int:
+    """Multiply-adds (2 flops each) of the layer output: the base product for every token plus
+    the adapter shrink and expand of every token with an adapter."""
+    p = wl.projections[0]
+    return 2 * wl.T * p.o * p.h + projection_flops(wl.ids, p.ranks, p.h, p.o)
