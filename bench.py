@@ -602,6 +602,14 @@ def run_ours(args, rank, world, local_rank):
     copies, ws_bytes = make_copies(wl, L, torch, args)
     C = len(copies)
     torch.cuda.synchronize()
+    # the library's own launch counters on one eager step confirm the launches a step makes
+    before = L.kernel_launches()
+    step(copies[0], int(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    after = L.kernel_launches()
+    counted = sum(after[k] - before[k] for k in after)
+    if counted != launches_per_step:
+        raise SystemExit("a step launched %d kernels, expected %d" % (counted, launches_per_step))
     K = args.steps
     if K <= 0:   # about 20 ms of work per repetition, a whole number of copy rotations
         tm0 = Timer(torch, copies, step, C, args.no_graph)

@@ -37,13 +37,14 @@ LORA_SIGMA_NONE = 0
 LORA_SIGMA_FULL = 1
 LORA_SIGMA_DIAG = 2
 LORA_MAX_MERGE = 8
+LORA_KERNEL_KINDS = 6
 
 EXPORTS = (
     "lora_table_create", "lora_table_destroy", "lora_table_info", "lora_workspace_bytes",
     "lora_build_segments", "lora_shrink", "lora_expand", "lora_sgmv", "lora_bgmv",
     "lora_get_status", "lora_status_string", "lora_set_option", "lora_get_option",
     "lora_sgmv_noalloc", "lora_sgmv_grouped", "lora_table_set_sigma", "lora_bgmv_merged",
-    "lora_sgmv_base",
+    "lora_sgmv_base", "lora_kernel_name", "lora_kernel_launches",
 )
 
 
@@ -99,6 +100,8 @@ def _load():
         "lora_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "lora_set_option": ([ctypes.c_char_p, I64], ctypes.c_int),
         "lora_get_option": ([ctypes.c_char_p, ctypes.POINTER(I64)], ctypes.c_int),
+        "lora_kernel_name": ([I32], ctypes.c_char_p),
+        "lora_kernel_launches": ([I32], I64),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -251,6 +254,12 @@ def lora_get_option(key: str) -> int:
     v = ctypes.c_int64()
     _check(_load().lora_get_option(key.encode(), ctypes.byref(v)), "lora_get_option")
     return int(v.value)
+
+
+def kernel_launches() -> dict:
+    """{kernel name: launches the CUDA runtime accepted so far in this process}."""
+    lib = _load()
+    return {lib.lora_kernel_name(k).decode(): int(lib.lora_kernel_launches(k)) for k in range(LORA_KERNEL_KINDS)}
 
 
 def lora_table_set_sigma(table: int, kind: int, sigma: Optional[Sequence] = None, stream=None) -> None:

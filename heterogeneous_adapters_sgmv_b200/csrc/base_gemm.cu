@@ -393,7 +393,9 @@ int launch_base_gemm(const lora_table *t, const lora_segments *seg, const void *
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, base_gemm_kernel, p) == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, base_gemm_kernel, p) != cudaSuccess) return LORA_ERR_CUDA;
+    note_launch(kKernBaseGemm);
+    return LORA_OK;
 }
 
 }  // namespace lora

@@ -1107,6 +1107,7 @@ int launch_one(const DecodeParams &p0, int units, cudaStream_t s)
     if (options().decode_max_clusters > 0) G = min(G, (int)options().decode_max_clusters);
     cfg.gridDim = dim3(G * CL);
     if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return LORA_ERR_CUDA;
+    note_launch(kKernDecode);
     return LORA_OK;
 }
 

@@ -2,6 +2,7 @@
 // choice of device path.  Nothing here computes the delta; every step runs in the kernels of
 // decode.cu, segments.cu and prefill.cu.
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -19,6 +20,14 @@ static int64_t env_or(const char *name, int64_t dflt)
     if (!v || !*v) return dflt;
     return std::strtoll(v, nullptr, 10);
 }
+
+static std::atomic<int64_t> g_launches[kKernKinds];
+static const char *const kKernelNames[kKernKinds] = {
+    "lora_decode_kernel", "count_segments_kernel", "build_segments_kernel", "prefill_shrink_kernel",
+    "prefill_expand_kernel", "base_gemm_kernel",
+};
+
+void note_launch(KernelKind k) { g_launches[k].fetch_add(1, std::memory_order_relaxed); }
 
 Options &options()
 {
@@ -57,6 +66,7 @@ using namespace lora;
 namespace {
 
 static_assert(kMaxProj == LORA_MAX_GROUP, "grouped-call limit");
+static_assert(kKernKinds == LORA_KERNEL_KINDS, "kernel kinds");
 constexpr int kBgmvMaxT = 1024;
 constexpr int kBgmvMaxN = 4096;
 
@@ -642,6 +652,16 @@ int lora_get_option(const char *key, int64_t *value)
     else if (!std::strcmp(key, "tc_min_tokens")) *value = o.tc_min_tokens;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
+}
+
+const char *lora_kernel_name(int32_t kind)
+{
+    return kind >= 0 && kind < kKernKinds ? kKernelNames[kind] : nullptr;
+}
+
+int64_t lora_kernel_launches(int32_t kind)
+{
+    return kind >= 0 && kind < kKernKinds ? g_launches[kind].load(std::memory_order_relaxed) : -1;
 }
 
 }  // extern "C"

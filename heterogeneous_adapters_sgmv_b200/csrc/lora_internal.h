@@ -73,6 +73,13 @@ struct Options {
 uint64_t wait_limit_ns();
 Options &options();
 
+// Host-side count of accepted launches per kernel (lora_kernel_launches).
+enum KernelKind {
+    kKernDecode = 0, kKernCountSegments, kKernBuildSegments, kKernPrefillShrink, kKernPrefillExpand,
+    kKernBaseGemm, kKernKinds
+};
+void note_launch(KernelKind k);
+
 // Launchers (return a LORA_* code).
 int launch_decode(int mode, int src, const DecodeParams &p, int dtype, cudaStream_t s);
 int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *perm, int32_t *seg_ptr,

@@ -34,6 +34,27 @@
 #include "tcgen05.cuh"
 
 namespace lora {
+#ifdef LORA_TRACE
+// instrumented builds only: per-CTA clock64 phase marks of the tcgen05 shrink
+__device__ unsigned long long lora_trace_shrink[4096 * 16];
+#define SHRINK_MARK(slot)                                                              \
+    do {                                                                               \
+        if (blockIdx.x < 4096u) ::lora::lora_trace_shrink[blockIdx.x * 16 + (slot)] = clock64(); \
+    } while (0)
+// and per-tile marks of the persistent expand: [CTA][tile 0..63, 64 = start][event 0..3]
+__device__ unsigned long long lora_trace_expand[160 * 65 * 4];
+#define EXPAND_MARK(i, e)                                                                          \
+    do {                                                                                           \
+        if (blockIdx.x < 160u && (i) <= 64) ::lora::lora_trace_expand[(blockIdx.x * 65 + (i)) * 4 + (e)] = clock64(); \
+    } while (0)
+#else
+#define SHRINK_MARK(slot) \
+    do {                  \
+    } while (0)
+#define EXPAND_MARK(i, e) \
+    do {                  \
+    } while (0)
+#endif
 namespace {
 
 constexpr int kTileM = 128;          // tokens per tile
@@ -100,16 +121,25 @@ __device__ __forceinline__ void tile_tokens(const PrefillParams &p, int row0, in
 }
 
 // Map a global 128-token tile index to (segment, first row, rows).  One warp scans the
-// segment table; returns false when the index is past the last tile.
+// segment table 32 entries at a time; each lane loads its entry's bounds and adapter together
+// with the segment count (one round trip per window rather than one per dependent value).
+// Returns false when the index is past the last tile.
 __device__ bool find_tile(const PrefillParams &p, int g, int *seg, int *row0, int *rows, int *adapter)
 {
     const int lane = threadIdx.x & 31;
-    const int nseg = min(*p.num_segs, p.max_segs);
+    const int ns_raw = *p.num_segs;
     int base_tiles = 0;
-    for (int s0 = 0; s0 < nseg; s0 += 32) {
+    for (int s0 = 0; s0 < p.max_segs; s0 += 32) {
         const int s = s0 + lane;
-        int len = 0;
-        if (s < nseg) len = max(0, min(p.seg_ptr[s + 1], p.T) - max(p.seg_ptr[s], 0));   // bad bounds: empty
+        int p0 = 0, p1 = 0, a = -1;
+        if (s < p.max_segs) {
+            p0 = p.seg_ptr[s];
+            p1 = p.seg_ptr[s + 1];
+            a = p.seg_adapter[s];
+        }
+        const int nseg = min(ns_raw, p.max_segs);
+        if (s0 >= nseg) break;
+        int len = (s < nseg) ? max(0, min(p1, p.T) - max(p0, 0)) : 0;   // bad bounds: empty
         if (len < p.min_len) len = 0;   // a short segment is served by the decode kernel
         const int tiles = (len + kTileM - 1) / kTileM;
         int incl = tiles;
@@ -123,14 +153,12 @@ __device__ bool find_tile(const PrefillParams &p, int g, int *seg, int *row0, in
         const uint32_t m = __ballot_sync(0xffffffffu, hit);
         if (m) {
             const int src = __ffs(m) - 1;
-            const int s_hit = __shfl_sync(0xffffffffu, s, src);
-            const int e_hit = __shfl_sync(0xffffffffu, excl, src);
-            const int start = max(p.seg_ptr[s_hit], 0);
-            const int end = min(p.seg_ptr[s_hit + 1], p.T);
-            *seg = s_hit;
-            *row0 = start + (g - e_hit) * kTileM;
+            const int start = max(__shfl_sync(0xffffffffu, p0, src), 0);
+            const int end = min(__shfl_sync(0xffffffffu, p1, src), p.T);
+            *seg = s0 + src;
+            *row0 = start + (g - __shfl_sync(0xffffffffu, excl, src)) * kTileM;
             *rows = min(kTileM, end - *row0);
-            *adapter = p.seg_adapter[s_hit];
+            *adapter = __shfl_sync(0xffffffffu, a, src);
             return true;
         }
         base_tiles += __shfl_sync(0xffffffffu, incl, 31);
@@ -166,8 +194,10 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     const uint32_t crank = cluster_ctarank();
     const int g = (int)cluster_id_x();
 
+    if (tid == 0) SHRINK_MARK(0);
     pdl_wait();
     pdl_launch_dependents();
+    if (tid == 0) SHRINK_MARK(1);
 
     if (warp == 0) {
         int s, row0 = 0, rows = 0, a = 0;
@@ -199,6 +229,7 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     const bool valid = ctl.info[0] != 0;
     const int row0 = ctl.info[1], rows = ctl.info[2], a = ctl.info[3], r = ctl.info[4];
     const float vscale = ctl.scale;
+    if (tid == 0) SHRINK_MARK(2);
     const int npad = (r + 15) & ~15;
     const uint32_t tmem = ctl.tmem_base;
     const int nkb_all = (p.h + kBK - 1) / kBK;
@@ -239,6 +270,7 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
                 }
                 __syncwarp();
                 if (p.perm && load) tma_gather4(smem_u32(st + lane * 512), &p.tmap_g, k0, tk[0], tk[1], tk[2], tk[3], fb);
+                if (lane == 0 && kb == 0) SHRINK_MARK(3);
             }
             // After a timeout the ring is given up early: wait (bounded) for the copies of the
             // last stages issued, so none is still writing when the ring is reused below.
@@ -252,6 +284,8 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
                 const int s = kb % kStages, m = kb / kStages;
                 if (!mbar_wait(smem_u32(&ctl.full[s]), m & 1, p.status, p.wait_ns)) break;
                 tc_fence_after();
+                if (kb == 0) SHRINK_MARK(4);
+                if (kb == nkb - 1) SHRINK_MARK(5);
                 uint8_t *st = smem + s * kStageBytes;
                 const uint64_t ad = sw128_desc(smem_u32(st));
                 const uint64_t bd = sw128_desc(smem_u32(st + kXBytes));
@@ -265,6 +299,7 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
         __syncwarp();
         ok = mbar_wait(smem_u32(&ctl.done), 0, p.status, p.wait_ns);
         tc_fence_after();
+        if (tid == 0) SHRINK_MARK(6);
     }
     // ---- epilogue: partial [128][npad] from tensor memory (zeros when this CTA had no k-blocks)
     // The ring is free: all MMAs and loads that fed them are complete.  A wait that ran out in
@@ -285,7 +320,9 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
                 if (c0 + i < npad) part[m * PRS + c0 + i] = acc[i];
         }
     }
+    if (tid == 0) SHRINK_MARK(7);
     cluster_sync_all();   // every CTA's partial is visible to its peers
+    if (tid == 0) SHRINK_MARK(8);
     if (valid) {
         // CTA j reduces rows [16 j, 16 j + 16) over the 8 partials, in CTA order
         const uint32_t part_addr = smem_u32(part);
@@ -327,10 +364,12 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
             }
         }
     }
+    if (tid == 0) SHRINK_MARK(9);
     cluster_sync_all();   // no peer reads this CTA's partial any more
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 64);
+    if (tid == 0) SHRINK_MARK(10);
 }
 
 // ----------------------------------------------------------------------------------------
@@ -367,12 +406,18 @@ struct __align__(8) ExpandCtl {
 __device__ int count_m_tiles(const PrefillParams &p)
 {
     const int lane = threadIdx.x & 31;
-    const int nseg = min(*p.num_segs, p.max_segs);
+    const int ns_raw = *p.num_segs;
     int tot = 0;
-    for (int s0 = 0; s0 < nseg; s0 += 32) {
+    for (int s0 = 0; s0 < p.max_segs; s0 += 32) {
         const int s = s0 + lane;
-        int len = 0;
-        if (s < nseg) len = max(0, min(p.seg_ptr[s + 1], p.T) - max(p.seg_ptr[s], 0));
+        int p0 = 0, p1 = 0;
+        if (s < p.max_segs) {
+            p0 = p.seg_ptr[s];
+            p1 = p.seg_ptr[s + 1];
+        }
+        const int nseg = min(ns_raw, p.max_segs);
+        if (s0 >= nseg) break;
+        int len = (s < nseg) ? max(0, min(p1, p.T) - max(p0, 0)) : 0;
         if (len < p.min_len) len = 0;
         int tiles = (len + kTileM - 1) / kTileM;
 #pragma unroll
@@ -392,6 +437,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = (p.o + kTileN - 1) / kTileN;
+    if (tid == 0) EXPAND_MARK(64, 0);
 
     if (tid == 0) {
         for (int i = 0; i < kExStages; ++i) {
@@ -420,6 +466,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (tid == 0) EXPAND_MARK(64, 1);
     const uint32_t tmem = ctl.tmem_base;
     const int total = ctl.total_m * NT;
     const int t0 = (int)((int64_t)blockIdx.x * total / gridDim.x);
@@ -470,6 +517,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 break;
             }
             if (lane == 0) {
+                EXPAND_MARK(i, 0);
                 ExTileInfo &inf = ctl.info[s];
                 inf.row0 = row0;
                 inf.rows = rows;
@@ -523,6 +571,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                     ++vuse;
                     prev_vb = vb;
                 }
+                EXPAND_MARK(i, 1);
                 if (i >= 2 && !mbar_wait(smem_u32(&ctl.accempty[ab]), ((i >> 1) - 1) & 1, p.status, p.wait_ns)) break;
                 tc_fence_after();
                 const uint8_t *st = ring + s * kExStageBytes;
@@ -556,6 +605,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             const bool okf = mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status, p.wait_ns);
             if (!named_bar_and(3, kEpiWarps * 32, oka && okf)) break;
             tc_fence_after();
+            if (ew == 0 && lane == 0) EXPAND_MARK(i, 2);
             const ExTileInfo inf = ctl.info[s];
             uint8_t *yt = ring + s * kExStageBytes + 16384 + half * 16384;   // this half's 64-column box
 #pragma unroll 1
@@ -610,6 +660,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 }
             }
             __syncwarp();
+            if (ew == 0 && lane == 0) EXPAND_MARK(i, 3);
             if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
         }
         if (ew == 0 && lane == 0) bulk_wait_group0();   // this CTA's tile stores are complete
@@ -741,7 +792,9 @@ int launch_shrink_kernel(PrefillParams &p, const lora_table *t, const lora_segme
     cfg.numAttrs = na;
     const cudaError_t e = KS == 4 ? cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<4>, p)
                                   : cudaLaunchKernelEx(&cfg, prefill_shrink_kernel<8>, p);
-    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    if (e != cudaSuccess) return LORA_ERR_CUDA;
+    note_launch(kKernPrefillShrink);
+    return LORA_OK;
 }
 
 }  // namespace
@@ -802,8 +855,24 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
         cfg.attrs = attr;
         cfg.numAttrs = na;
         if (cudaLaunchKernelEx(&cfg, prefill_expand_kernel, p) != cudaSuccess) return LORA_ERR_CUDA;
+        note_launch(kKernPrefillExpand);
     }
     return LORA_OK;
 }
 
 }  // namespace lora
+
+#ifdef LORA_TRACE
+// Instrumented builds only: copy the shrink's per-CTA phase marks to the host.
+extern "C" int lora_trace_read_shrink(unsigned long long *host, int n)
+{
+    if (n > 4096 * 16) n = 4096 * 16;
+    return cudaMemcpyFromSymbol(host, lora::lora_trace_shrink, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : -4;
+}
+
+extern "C" int lora_trace_read_expand(unsigned long long *host, int n)
+{
+    if (n > 160 * 65 * 4) n = 160 * 65 * 4;
+    return cudaMemcpyFromSymbol(host, lora::lora_trace_expand, sizeof(unsigned long long) * n) == cudaSuccess ? 0 : -4;
+}
+#endif

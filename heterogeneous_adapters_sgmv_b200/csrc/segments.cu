@@ -273,6 +273,7 @@ int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *per
     if (cudaLaunchKernelEx(&cfg, counting ? count_segments_kernel : build_segments_kernel, ids, T, n, perm,
                            seg_ptr, seg_adapter, num_segs, status) != cudaSuccess)
         return LORA_ERR_CUDA;
+    note_launch(counting ? kKernCountSegments : kKernBuildSegments);
     return LORA_OK;
 }
 

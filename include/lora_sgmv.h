@@ -279,6 +279,18 @@ const char *lora_status_string(int code);
 int lora_set_option(const char *key, int64_t value);
 int lora_get_option(const char *key, int64_t *value);
 
+/* Launch counters (diagnostics, process-wide): the number of launches of each of the library's
+ * kernels that the CUDA runtime has accepted since the library was loaded.  kind runs from 0 to
+ * LORA_KERNEL_KINDS - 1 (0 the decode kernel, 1 and 2 the two segment-building kernels, 3 and
+ * 4 the tcgen05 shrink and expand, 5 the fused base GEMM).  lora_kernel_name returns the
+ * kernel's name (static text; NULL outside that range) and lora_kernel_launches its count (-1
+ * outside that range).  A count says that a launch was enqueued, not that it has finished;
+ * lora_get_status reports what the device found.  Tests read them to see which path a call
+ * took. */
+#define LORA_KERNEL_KINDS 6
+const char *lora_kernel_name(int32_t kind);
+int64_t lora_kernel_launches(int32_t kind);
+
 #ifdef __cplusplus
 }
 #endif

@@ -112,21 +112,17 @@ class DeviceProj:
         return torch_to_np(y, self.dtype)
 
 
-def kernels_launched(fn, tries: int = 3) -> set:
-    """Names of the CUDA kernels that ran during fn() (torch profiler, device events).  A
-    profiler session late in a long process can come back with no device events at all; the
-    session is then repeated (fn must tolerate being called again)."""
-    from torch.profiler import ProfilerActivity, profile
-    names = set()
-    for _ in range(tries):
-        torch.cuda.synchronize()
-        with profile(activities=[ProfilerActivity.CUDA], acc_events=True) as prof:
-            fn()
-            torch.cuda.synchronize()
-        names = {e.name for e in prof.events() if e.device_type.name == "CUDA"}
-        if names:
-            break
-    return names
+def kernels_launched(fn) -> set:
+    """Names of the library's kernels that fn() launched, from the library's own launch
+    counters (lora_kernel_launches: launches the CUDA runtime accepted).  The call's results are
+    checked against the oracle separately; this says which path the dispatcher took.  (The torch
+    profiler was tried first: late in a long process it recorded only the last of several
+    launches, or none.)"""
+    before = L.kernel_launches()
+    fn()
+    torch.cuda.synchronize()
+    after = L.kernel_launches()
+    return {k for k in after if after[k] > before[k]}
 
 
 def ran(names: set, kernel: str) -> bool:

@@ -66,7 +66,8 @@ def test_header_constants_match_binding():
                  "LORA_ERR_WORKSPACE", "LORA_ERR_CUDA", "LORA_ERR_TIMEOUT", "LORA_ERR_DEVICE_STATUS",
                  "LORA_STATUS_BAD_ID", "LORA_STATUS_TIMEOUT", "LORA_STATUS_BAD_SEGMENT", "LORA_MAX_RANK",
                  "LORA_MAX_SEGMENT_TOKENS", "LORA_NOALLOC_SCRATCH_FLOATS", "LORA_MAX_GROUP",
-                 "LORA_SIGMA_NONE", "LORA_SIGMA_FULL", "LORA_SIGMA_DIAG", "LORA_MAX_MERGE"):
+                 "LORA_SIGMA_NONE", "LORA_SIGMA_FULL", "LORA_SIGMA_DIAG", "LORA_MAX_MERGE",
+                 "LORA_KERNEL_KINDS"):
         m = re.search(r"#define %s \(?(-?\d+)u?\)?" % name, txt)
         assert m, name
         assert int(m.group(1)) == getattr(L, name), name
@@ -100,6 +101,24 @@ def test_every_documented_option_round_trips():
         assert L.lora_get_option(key) == old
     with pytest.raises(L.LoraError):
         L.lora_set_option("no_such_option", 1)
+
+
+def test_launch_counters_name_every_kernel():
+    """The launch counters cover each __global__ kernel of the library by name, start at a
+    count of zero or more, and reject kinds outside the range (host only)."""
+    lib = L._load()
+    names = [lib.lora_kernel_name(k).decode() for k in range(L.LORA_KERNEL_KINDS)]
+    assert lib.lora_kernel_name(-1) is None and lib.lora_kernel_name(L.LORA_KERNEL_KINDS) is None
+    assert lib.lora_kernel_launches(-1) == -1 and lib.lora_kernel_launches(L.LORA_KERNEL_KINDS) == -1
+    src = ""
+    csrc = os.path.join(ROOT, "heterogeneous_adapters_sgmv_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith(".cu"):
+            src += open(os.path.join(csrc, f)).read()
+    kernels = set(re.findall(r"__global__ void(?: __launch_bounds__\([^)]*\))?\s+(\w+)\(", src))
+    assert kernels == set(names), (kernels, names)
+    counts = L.kernel_launches()
+    assert set(counts) == set(names) and all(v >= 0 for v in counts.values())
 
 
 def test_merged_and_sigma_host_checks():
