@@ -47,7 +47,14 @@ __device__ unsigned long long lora_trace_expand[160 * 65 * 4];
     do {                                                                                           \
         if (blockIdx.x < 160u && (i) <= 64) ::lora::lora_trace_expand[(blockIdx.x * 65 + (i)) * 4 + (e)] = clock64(); \
     } while (0)
+#define EXPAND_GMARK(e)                                                                            \
+    do {                                                                                           \
+        if (blockIdx.x < 160u) ::lora::lora_trace_expand[(blockIdx.x * 65 + 64) * 4 + (e)] = globaltimer_ns(); \
+    } while (0)
 #else
+#define EXPAND_GMARK(e) \
+    do {                \
+    } while (0)
 #define SHRINK_MARK(slot) \
     do {                  \
     } while (0)
@@ -376,16 +383,22 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
 // Persistent expand: CTA b walks tiles [b * total / G, (b + 1) * total / G) of the
 // (128-token tile, 128-column tile) grid, columns fastest, so consecutive tiles share the
 // intermediate tile.  Warp roles:
-//   warp 0      producer: builds the bf16 hi + lo intermediate tile (double-buffered) when the
-//               token tile changes, and streams B_i and y tiles by TMA into a 3-stage ring;
+//   warp 0      producer: loads the bf16 hi + lo intermediate tile (double-buffered) when the
+//               token tile changes, and streams y tiles (4-stage ring) and B_i tiles (2-stage
+//               ring: the MMA releases a B tile as soon as it has read it, while a y tile is
+//               held through the epilogue and its store) by TMA;
 //   warp 1      MMA issuer (one thread) into two TMEM accumulators used alternately;
 //   warps 2..9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 and columns
-//               64 ((w - 2) / 4) .. +63, adds s * acc to y in place in shared memory, then the
-//               eight warps store the tile's valid rows with coalesced 16-byte stores.
+//               64 ((w - 2) / 4) .. +63, adds s * acc to y in place in shared memory; a full
+//               tile goes back by two TMA stores, whose shared-memory reads are awaited only at
+//               the next tile (the y stage is released one tile late, the epilogue moves on at
+//               once); a partial tile by coalesced 16-byte stores masked to the segment.
 constexpr int kEpiWarps = 8;
 constexpr int kThreadsEX = (2 + kEpiWarps) * 32;
-constexpr int kExStages = 3;
-constexpr int kExStageBytes = 16384 + 32768;           // B tile + y tile (two 64-column boxes)
+constexpr int kExYStages = 4;
+constexpr int kExBStages = 2;
+constexpr int kExYBytes = 32768;                       // y tile: two 64-column boxes of 128 rows
+constexpr int kExBBytes = 16384;                       // B_i tile: 128 rows of o x 64 ranks
 constexpr int kExVBytes = 32768;                       // hi + lo intermediate tile
 
 struct ExTileInfo {
@@ -394,13 +407,14 @@ struct ExTileInfo {
 };
 
 struct __align__(8) ExpandCtl {
-    uint64_t full[kExStages], empty[kExStages];
+    uint64_t yfull[kExYStages], yempty[kExYStages];
+    uint64_t bfull[kExBStages], bempty[kExBStages];
     uint64_t vfull[2], vempty[2];
     uint64_t accfull[2], accempty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
     int32_t total_m;
-    ExTileInfo info[kExStages];
+    ExTileInfo info[kExYStages];   // per y stage; written before the tile's B and y loads are armed
 };
 
 __device__ int count_m_tiles(const PrefillParams &p)
@@ -432,17 +446,23 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *vbuf = smem;                                    // [2][hi 16 KiB | lo 16 KiB]
-    uint8_t *ring = smem + 2 * kExVBytes;                    // [kExStages][B 16 KiB | y 32 KiB]
-    ExpandCtl &ctl = *reinterpret_cast<ExpandCtl *>(ring + kExStages * kExStageBytes);
+    uint8_t *yring = smem + 2 * kExVBytes;                   // [kExYStages][y 32 KiB]
+    uint8_t *bring = yring + kExYStages * kExYBytes;         // [kExBStages][B 16 KiB]
+    ExpandCtl &ctl = *reinterpret_cast<ExpandCtl *>(bring + kExBStages * kExBBytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = (p.o + kTileN - 1) / kTileN;
     if (tid == 0) EXPAND_MARK(64, 0);
+    if (tid == 0) EXPAND_GMARK(2);
 
     if (tid == 0) {
-        for (int i = 0; i < kExStages; ++i) {
-            mbar_init(smem_u32(&ctl.full[i]), 1);
-            mbar_init(smem_u32(&ctl.empty[i]), 1 + kEpiWarps);
+        for (int i = 0; i < kExYStages; ++i) {
+            mbar_init(smem_u32(&ctl.yfull[i]), 1);
+            mbar_init(smem_u32(&ctl.yempty[i]), kEpiWarps);
+        }
+        for (int i = 0; i < kExBStages; ++i) {
+            mbar_init(smem_u32(&ctl.bfull[i]), 1);
+            mbar_init(smem_u32(&ctl.bempty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_u32(&ctl.vfull[i]), 1);
@@ -479,7 +499,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         int tk[4] = {0, 0, 0, 0};   // with a permutation: tokens of rows 4 lane .. 4 lane + 3
         float sc = 0.f;
         for (int t = t0; t < t1 && ok; ++t) {
-            const int i = t - t0, s = i % kExStages;
+            const int i = t - t0, sy = i % kExYStages, sb = i % kExBStages;
             const int g = t / NT, nt = t - g * NT;
             if (g != cur_g) {
                 int sg;
@@ -511,48 +531,57 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 __syncwarp();
                 ++vcount;
             }
-            if (i >= kExStages && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]),
-                                                                     ((i / kExStages) - 1) & 1, p.status, p.wait_ns))) {
+            if (i >= kExYStages && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.yempty[sy]),
+                                                                      ((i / kExYStages) - 1) & 1, p.status, p.wait_ns))) {
                 ok = false;
                 break;
             }
+            if (i >= kExBStages && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.bempty[sb]),
+                                                                      ((i / kExBStages) - 1) & 1, p.status, p.wait_ns))) {
+                ok = false;
+                break;
+            }
+            // test-only stall: the first tile's stages are armed but never loaded
+            const bool load = !((p.inject & 4) && i == 0);
             if (lane == 0) {
                 EXPAND_MARK(i, 0);
-                ExTileInfo &inf = ctl.info[s];
+                ExTileInfo &inf = ctl.info[sy];
                 inf.row0 = row0;
                 inf.rows = rows;
                 inf.col0 = nt * kTileN;
                 inf.ncols = min(kTileN, p.o - nt * kTileN);
                 inf.vb = vb;
                 inf.scale = sc;
-                uint8_t *st = ring + s * kExStageBytes;
-                const uint32_t fb = smem_u32(&ctl.full[s]);
-                mbar_arrive_expect_tx(fb, kExStageBytes);
-                // test-only stall: the first tile's stage is armed but never loaded
-                if (!((p.inject & 4) && i == 0)) {
-                    tma_load_2d(smem_u32(st), p.tm_B + (size_t)a * 128, 0, nt * kTileN, fb);
+                uint8_t *yst = yring + sy * kExYBytes;
+                const uint32_t yb = smem_u32(&ctl.yfull[sy]), bb = smem_u32(&ctl.bfull[sb]);
+                mbar_arrive_expect_tx(yb, kExYBytes);
+                mbar_arrive_expect_tx(bb, kExBBytes);
+                if (load) {
+                    tma_load_2d(smem_u32(bring + sb * kExBBytes), p.tm_B + (size_t)a * 128, 0, nt * kTileN, bb);
                     if (!p.perm) {
-                        tma_load_2d(smem_u32(st + 16384), &p.tmap_io, nt * kTileN, row0, fb);
-                        tma_load_2d(smem_u32(st + 32768), &p.tmap_io, nt * kTileN + 64, row0, fb);
+                        tma_load_2d(smem_u32(yst), &p.tmap_io, nt * kTileN, row0, yb);
+                        tma_load_2d(smem_u32(yst + 16384), &p.tmap_io, nt * kTileN + 64, row0, yb);
                     }
                 }
             }
             __syncwarp();
-            if (p.perm && !((p.inject & 4) && i == 0)) {   // the y tile's rows, four per lane
-                const uint32_t st = smem_u32(ring + s * kExStageBytes);
-                const uint32_t fb = smem_u32(&ctl.full[s]);
-                tma_gather4(st + 16384 + lane * 512, &p.tmap_g, nt * kTileN, tk[0], tk[1], tk[2], tk[3], fb);
-                tma_gather4(st + 32768 + lane * 512, &p.tmap_g, nt * kTileN + 64, tk[0], tk[1], tk[2], tk[3], fb);
+            if (p.perm && load) {   // the y tile's rows, four per lane
+                const uint32_t yst = smem_u32(yring + sy * kExYBytes);
+                const uint32_t yb = smem_u32(&ctl.yfull[sy]);
+                tma_gather4(yst + lane * 512, &p.tmap_g, nt * kTileN, tk[0], tk[1], tk[2], tk[3], yb);
+                tma_gather4(yst + 16384 + lane * 512, &p.tmap_g, nt * kTileN + 64, tk[0], tk[1], tk[2], tk[3], yb);
             }
             ++nissued;
             __syncwarp();
         }
         // drain: every TMA issued by this CTA has landed before shared memory is released (the
-        // stages of the last kExStages tiles armed; earlier ones were consumed before reuse)
+        // stages of the last tiles armed; earlier ones were consumed before reuse)
         const int n = nissued;
         if (lane == 0) {
-            for (int i = max(0, n - kExStages); i < n; ++i)
-                mbar_wait(smem_u32(&ctl.full[i % kExStages]), (i / kExStages) & 1, p.status, p.wait_ns);
+            for (int i = max(0, n - kExYStages); i < n; ++i)
+                mbar_wait(smem_u32(&ctl.yfull[i % kExYStages]), (i / kExYStages) & 1, p.status, p.wait_ns);
+            for (int i = max(0, n - kExBStages); i < n; ++i)
+                mbar_wait(smem_u32(&ctl.bfull[i % kExBStages]), (i / kExBStages) & 1, p.status, p.wait_ns);
             for (int c = max(0, vcount - 2); c < vcount; ++c)
                 mbar_wait(smem_u32(&ctl.vfull[c & 1]), (c >> 1) & 1, p.status, p.wait_ns);
         }
@@ -562,29 +591,28 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             const uint32_t idesc = idesc_bf16(kTileM, kTileN);
             int vuse = 0, prev_vb = -1;
             for (int t = t0; t < t1; ++t) {
-                const int i = t - t0, s = i % kExStages, ab = i & 1;
-                if (!mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status, p.wait_ns)) break;
-                const int vb = ctl.info[s].vb;
+                const int i = t - t0, sy = i % kExYStages, sb = i % kExBStages, ab = i & 1;
+                if (!mbar_wait(smem_u32(&ctl.bfull[sb]), (i / kExBStages) & 1, p.status, p.wait_ns)) break;
+                EXPAND_MARK(i, 1);
+                const int vb = ctl.info[sy].vb;
                 if (vb != prev_vb) {
                     if (prev_vb >= 0) umma_commit(smem_u32(&ctl.vempty[prev_vb]));   // old tile may be rebuilt
                     if (!mbar_wait(smem_u32(&ctl.vfull[vb]), (vuse >> 1) & 1, p.status, p.wait_ns)) break;
                     ++vuse;
                     prev_vb = vb;
                 }
-                EXPAND_MARK(i, 1);
                 if (i >= 2 && !mbar_wait(smem_u32(&ctl.accempty[ab]), ((i >> 1) - 1) & 1, p.status, p.wait_ns)) break;
                 tc_fence_after();
-                const uint8_t *st = ring + s * kExStageBytes;
                 const uint64_t dh = sw128_desc(smem_u32(vbuf + vb * kExVBytes));
                 const uint64_t dl = sw128_desc(smem_u32(vbuf + vb * kExVBytes + 16384));
-                const uint64_t db = sw128_desc(smem_u32(st));
+                const uint64_t db = sw128_desc(smem_u32(bring + sb * kExBBytes));
                 const uint32_t acc = tmem + (uint32_t)(ab * kTileN);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) umma_bf16(acc, dh + 2 * k, db + 2 * k, idesc, k != 0 ? 1u : 0u);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) umma_bf16(acc, dl + 2 * k, db + 2 * k, idesc, 1u);
                 umma_commit(smem_u32(&ctl.accfull[ab]));
-                umma_commit(smem_u32(&ctl.empty[s]));
+                umma_commit(smem_u32(&ctl.bempty[sb]));
             }
             // every MMA of this CTA has completed before tensor memory is released
             umma_commit(smem_u32(&ctl.mma_done));
@@ -597,50 +625,54 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         const int half = (warp - 2) >> 2;       // column half of the tile
         const int m = q * 32 + lane;            // row of the tile
         const int ew = warp - 2;                // epilogue warp 0..7
+        int pending = -1;                       // ew 0: y stage whose TMA store is still reading it
         for (int t = t0; t < t1; ++t) {
-            const int i = t - t0, s = i % kExStages, ab = i & 1;
+            const int i = t - t0, sy = i % kExYStages, ab = i & 1;
             // every epilogue warp leaves together if any lane ran out of time (the tensor-memory
             // loads below are warp-collective and the warps meet at a named barrier)
             const bool oka = mbar_wait(smem_u32(&ctl.accfull[ab]), (i >> 1) & 1, p.status, p.wait_ns);
-            const bool okf = mbar_wait(smem_u32(&ctl.full[s]), (i / kExStages) & 1, p.status, p.wait_ns);
+            const bool okf = mbar_wait(smem_u32(&ctl.yfull[sy]), (i / kExYStages) & 1, p.status, p.wait_ns);
             if (!named_bar_and(3, kEpiWarps * 32, oka && okf)) break;
             tc_fence_after();
             if (ew == 0 && lane == 0) EXPAND_MARK(i, 2);
-            const ExTileInfo inf = ctl.info[s];
-            uint8_t *yt = ring + s * kExStageBytes + 16384 + half * 16384;   // this half's 64-column box
-#pragma unroll 1
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                float acc[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kTileN + half * 64 + c0), acc);
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    uint4 *pw = reinterpret_cast<uint4 *>(yt + sw128_off(m, (c0 >> 3) + qq));
-                    uint4 w = *pw;
-                    uint32_t *wv = reinterpret_cast<uint32_t *>(&w);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float y0 = fmaf(inf.scale, acc[qq * 8 + 2 * e], bf16_lo(wv[e]));
-                        const float y1 = fmaf(inf.scale, acc[qq * 8 + 2 * e + 1], bf16_hi(wv[e]));
-                        wv[e] = pack_bf16x2(y0, y1);
-                    }
-                    *pw = w;
-                }
-            }
+            const ExTileInfo inf = ctl.info[sy];
+            uint8_t *yt = yring + sy * kExYBytes + half * 16384;   // this half's 64-column box
+            float acc[64];
+            tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kTileN + half * 64), acc);
             tc_fence_before();
-            fence_proxy_async_smem();            // the updated tile is read by the TMA unit below
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl.accempty[ab]));
+            if (lane == 0) mbar_arrive(smem_u32(&ctl.accempty[ab]));   // the accumulator is in registers
+            uint4 w[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) w[c] = *reinterpret_cast<const uint4 *>(yt + sw128_off(m, c));
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t *wv = reinterpret_cast<uint32_t *>(&w[c]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float y0 = fmaf(inf.scale, acc[c * 8 + 2 * e], bf16_lo(wv[e]));
+                    const float y1 = fmaf(inf.scale, acc[c * 8 + 2 * e + 1], bf16_hi(wv[e]));
+                    wv[e] = pack_bf16x2(y0, y1);
+                }
+                *reinterpret_cast<uint4 *>(yt + sw128_off(m, c)) = w[c];
+            }
+            fence_proxy_async_smem();            // the updated tile is read by the TMA unit below
             named_bar_sync(2, kEpiWarps * 32);   // the whole tile is updated in shared memory
             const bool full_tile = !p.perm && inf.rows == kTileM && inf.ncols == kTileN;
             if (full_tile) {
-                // a full tile lies inside one segment: two TMA stores write it back
                 if (ew == 0 && lane == 0) {
-                    const uint32_t yt0 = smem_u32(ring + s * kExStageBytes + 16384);
+                    const uint32_t yt0 = smem_u32(yring + sy * kExYBytes);
                     tma_store_2d(&p.tmap_io, yt0, inf.col0, inf.row0);
                     tma_store_2d(&p.tmap_io, yt0 + 16384, inf.col0 + 64, inf.row0);
                     bulk_commit_group();
-                    bulk_wait_group_read0();     // the stage is reused only after this warp arrives
+                    // the previous tile's store has read its stage: release that stage now
+                    if (pending >= 0) {
+                        bulk_wait_group_read1();
+                        mbar_arrive(smem_u32(&ctl.yempty[pending]));
+                    }
+                    EXPAND_MARK(i, 3);
                 }
+                if (ew == 0) pending = sy;
             } else {
                 // coalesced stores masked to the segment's rows and to o: epilogue warp ew stores
                 // rows 16 ew .. 16 ew + 15, two per step
@@ -652,28 +684,41 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                     if (rr < inf.rows && chunk * 8 < inf.ncols) {
                         const int tok = p.perm ? p.perm[inf.row0 + rr] : inf.row0 + rr;
                         if (tok < 0 || tok >= p.T) continue;   // latched when the rows were gathered
-                        const uint8_t *box = ring + s * kExStageBytes + 16384 + (chunk >= 8 ? 16384 : 0);
-                        const uint4 w = *reinterpret_cast<const uint4 *>(box + sw128_off(rr, chunk & 7));
+                        const uint8_t *box = yring + sy * kExYBytes + (chunk >= 8 ? 16384 : 0);
+                        const uint4 wv = *reinterpret_cast<const uint4 *>(box + sw128_off(rr, chunk & 7));
                         *reinterpret_cast<uint4 *>(
-                            yg + ((int64_t)tok * p.ldy + p.y_off + inf.col0 + chunk * 8) * 2) = w;
+                            yg + ((int64_t)tok * p.ldy + p.y_off + inf.col0 + chunk * 8) * 2) = wv;
                     }
                 }
+                if (ew == 0 && lane == 0 && pending >= 0) {   // no store group of this tile to keep
+                    bulk_wait_group_read0();
+                    mbar_arrive(smem_u32(&ctl.yempty[pending]));
+                }
+                if (ew == 0) pending = -1;
             }
             __syncwarp();
-            if (ew == 0 && lane == 0) EXPAND_MARK(i, 3);
-            if (lane == 0) mbar_arrive(smem_u32(&ctl.empty[s]));
+            // warps 1..7, and warp 0 for a tile without a TMA store, release the stage now
+            if (lane == 0 && !(ew == 0 && pending == sy)) mbar_arrive(smem_u32(&ctl.yempty[sy]));
         }
-        if (ew == 0 && lane == 0) bulk_wait_group0();   // this CTA's tile stores are complete
+        if (ew == 0 && lane == 0) {
+            if (pending >= 0) {
+                bulk_wait_group_read0();
+                mbar_arrive(smem_u32(&ctl.yempty[pending]));
+            }
+            bulk_wait_group0();   // this CTA's tile stores are complete
+        }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, 256);
+    if (tid == 0) EXPAND_GMARK(3);
 }
 
 // ------------------------------------------------------------------- host side
 
 constexpr int shrink_smem(int ks) { return shrink_stages(ks) * (kTileM * 128 + kMaxRankPF * 128) + 256 + 1024; }
-constexpr int kExpandSmem = 2 * kExVBytes + kExStages * kExStageBytes + (int)sizeof(ExpandCtl) + 1024;
+constexpr int kExpandSmem = 2 * kExVBytes + kExYStages * kExYBytes + kExBStages * kExBBytes + (int)sizeof(ExpandCtl) + 1024;
+static_assert(kExpandSmem <= 227 * 1024, "expand shared memory");
 static_assert(shrink_stages(8) * (kTileM * 128 + kMaxRankPF * 128) >= kTileM * (kMaxRankPF + 4) * 4, "partial fits ring");
 static_assert(shrink_smem(4) <= 227 * 1024, "shrink shared memory");
 
