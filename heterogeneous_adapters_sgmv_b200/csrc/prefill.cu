@@ -202,6 +202,19 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     const int g = (int)cluster_id_x();
 
     if (tid == 0) SHRINK_MARK(0);
+    // set-up that touches no global memory runs before the wait on the previous kernel
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(smem_u32(&ctl.full[i]), 1);
+            mbar_init(smem_u32(&ctl.empty[i]), 1);
+        }
+        mbar_init(smem_u32(&ctl.done), 1);
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(&ctl.tmem_base), 64);
+        tmem_relinquish();
+    }
     pdl_wait();
     pdl_launch_dependents();
     if (tid == 0) SHRINK_MARK(1);
@@ -218,17 +231,7 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
             ctl.info[3] = a;
             ctl.info[4] = good ? p.desc[a].rank : 0;
             ctl.scale = (good && p.fold_scale) ? p.desc[a].scale : 1.f;
-            for (int i = 0; i < kStages; ++i) {
-                mbar_init(smem_u32(&ctl.full[i]), 1);
-                mbar_init(smem_u32(&ctl.empty[i]), 1);
-            }
-            mbar_init(smem_u32(&ctl.done), 1);
-            fence_mbar_init_cluster();
         }
-    }
-    if (warp == 1) {
-        tmem_alloc(smem_u32(&ctl.tmem_base), 64);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
