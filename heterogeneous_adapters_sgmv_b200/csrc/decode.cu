@@ -58,6 +58,10 @@ constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers + 32;   // + one producer warp
 constexpr int kTokChunk = 16;               // tokens per work unit
+// Cost-balanced split of segment-table units over the clusters: a unit's estimated work is a
+// fixed part plus tokens x rank, in the proportion measured on this kernel (about 2.5 us per
+// unit plus 21 ns per token-rank at 4096 -> 4096).
+constexpr int kUnitFixedCost = 120;
 constexpr int kRowBytes = 1024;             // h-subtile row (shrink) / o-subtile span (expand);
                                             // 512 for ranks above 64 (smaller stages)
 constexpr int kBoxBytes = 512;              // one TMA box row of A
@@ -357,6 +361,43 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         }
         __syncthreads();
     }
+    // Segment tables: every thread helps stage each segment's length and rank for the
+    // producer's cost-balanced split of the units (below).  The stage ring is free until the
+    // producer's first tile, so it holds them (8 bytes per segment; larger tables keep the
+    // fixed stride).
+    int2 *segw = reinterpret_cast<int2 *>(stage_base);
+    const int nseg_sc = (SRC == kSrcSegments) ? min(*p.num_segs, p.max_segs) : 0;
+    const bool use_part = SRC == kSrcSegments && p.balance &&
+                          (int64_t)nseg_sc * (int64_t)sizeof(int2) <= (int64_t)p.stages * p.stage_bytes;
+    if (use_part) {
+        bool bad = false;
+        for (int s0 = tid; s0 < nseg_sc; s0 += 2 * kThreads) {
+            int av[2], q0[2], q1[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int sg = s0 + u * kThreads;
+                av[u] = -1;
+                q0[u] = q1[u] = 0;
+                if (sg < nseg_sc) {
+                    av[u] = p.seg_adapter[sg];
+                    q0[u] = p.seg_ptr[sg];
+                    q1[u] = p.seg_ptr[sg + 1];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int sg = s0 + u * kThreads;
+                if (sg < nseg_sc) {
+                    const bool okseg = av[u] >= 0 && av[u] < p.n && q0[u] >= 0 && q1[u] >= q0[u] && q1[u] <= p.T;
+                    bad |= !okseg;
+                    int len = okseg ? q1[u] - q0[u] : 0;
+                    if (p.long_len != 0 && len >= p.long_len) len = 0;   // served by the tensor-core kernels
+                    segw[sg] = make_int2(len, len > 0 ? p.pj[0].desc[av[u]].rank : 0);
+                }
+            }
+        }
+        if (__syncthreads_or(bad) && tid == 0 && crank == 0 && cid == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+    }
     if (tid == 0) LORA_TRACE_MARK(1);
 
     if (warp == kConsumerWarps) {
@@ -392,18 +433,108 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         }
         // Walk this cluster's units; each yields (adapter, descriptor, tokens in lanes 0..L-1).
         // Segment tables: units are the 16-token chunks of the segments, numbered segment by
-        // segment, and cluster c takes units c, c + G, ... so a long segment spreads over many
-        // clusters.  The warp holds a window of 32 segments (lane l: segment sb + l) with the
-        // inclusive prefix count of their units and slides it forward as units are taken.
+        // segment.  The units are cut into G contiguous runs of about equal estimated work and
+        // cluster c takes run c (with the segments staged), else units c, c + G, ...; a long
+        // segment spreads over many clusters either way.  A fixed stride can stack several heavy
+        // units (many tokens of a high-rank adapter) on one cluster; the runs keep each
+        // cluster's work within one unit of the average.  The warp holds a window of 32 segments
+        // (lane l: segment sb + l) with the inclusive prefix count of their units and slides it
+        // forward as units are taken.
         const int nseg = (SRC == kSrcSegments) ? min(*p.num_segs, p.max_segs) : 0;
         int sb = -32, ubase = 0, w_p0 = 0, w_p1 = 0, w_sa = -1, w_nu = 0, w_incl = 0, w_total = 0;
-        int un = cid;
+        int un = cid, un_end = INT_MAX, un_step = G;
+        if (use_part) {
+            // lane l sums the segments [l B, l B + B): estimated work and units, then scans
+            const int B = (nseg + 31) / 32;
+            const int s_lo = min(nseg, lane * B), s_hi = min(nseg, s_lo + B);
+            long long C = 0;
+            int U = 0;
+            for (int sg = s_lo; sg < s_hi; ++sg) {
+                const int2 e = segw[sg];
+                const int nu = (e.x + kTokChunk - 1) / kTokChunk;
+                C += (long long)kUnitFixedCost * nu + (long long)e.x * e.y;
+                U += nu;
+            }
+            long long Ci = C;
+            int Ui = U;
+#pragma unroll
+            for (int dl = 1; dl < 32; dl <<= 1) {
+                const long long vc = __shfl_up_sync(0xffffffffu, Ci, dl);
+                const int vu = __shfl_up_sync(0xffffffffu, Ui, dl);
+                if (lane >= dl) {
+                    Ci += vc;
+                    Ui += vu;
+                }
+            }
+            const long long tot = __shfl_sync(0xffffffffu, Ci, 31);
+            const long long Gl = G;
+            // units whose doubled midpoint m (twice the work before them plus their own) has
+            // m G < X: per segment in closed form (its units cost cf but the last, cl)
+            int cnt_lo = 0, cnt_hi = 0;
+            {
+                long long P = Ci - C;
+                const long long Xlo = 2 * tot * cid, Xhi = 2 * tot * (cid + 1);
+                for (int sg = s_lo; sg < s_hi; ++sg) {
+                    const int2 e = segw[sg];
+                    const int nu = (e.x + kTokChunk - 1) / kTokChunk;
+                    if (nu == 0) continue;
+                    const long long cf = kUnitFixedCost + (long long)kTokChunk * e.y;
+                    const long long cl = kUnitFixedCost + (long long)(e.x - kTokChunk * (nu - 1)) * e.y;
+                    const long long mlast = 2 * P + 2 * (long long)(nu - 1) * cf + cl;
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        const long long X = w == 0 ? Xlo : Xhi;
+                        int c = 0;
+                        const long long Y = X - 2 * P * Gl;
+                        if (nu > 1 && Y > 0) {
+                            const long long q = (Y + cf * Gl - 1) / (cf * Gl);
+                            c = (int)min((long long)(nu - 1), q / 2);
+                        }
+                        if (mlast * Gl < X) c = nu;
+                        if (w == 0) cnt_lo += c;
+                        else cnt_hi += c;
+                    }
+                    P += (long long)kUnitFixedCost * nu + (long long)e.x * e.y;
+                }
+            }
+#pragma unroll
+            for (int dl = 16; dl >= 1; dl >>= 1) {
+                cnt_lo += __shfl_xor_sync(0xffffffffu, cnt_lo, dl);
+                cnt_hi += __shfl_xor_sync(0xffffffffu, cnt_hi, dl);
+            }
+            un = cnt_lo;
+            un_end = cnt_hi;
+            un_step = 1;
+            if (un < un_end) {
+                // start the window at the window of 32 segments that holds unit `un`
+                const int ub = Ui - U;   // units before this lane's segments
+                int hs = -1;
+                if (un >= ub && un < Ui) {
+                    int acc = ub;
+                    for (int sg = s_lo; sg < s_hi; ++sg) {
+                        acc += (segw[sg].x + kTokChunk - 1) / kTokChunk;
+                        if (un < acc) {
+                            hs = sg;
+                            break;
+                        }
+                    }
+                }
+                const int hsw = __reduce_max_sync(0xffffffffu, hs);
+                const int s0w = hsw / 32 * 32;
+                int before = 0;
+                for (int sg = s_lo; sg < min(s_hi, s0w); ++sg) before += (segw[sg].x + kTokChunk - 1) / kTokChunk;
+                before = __reduce_add_sync(0xffffffffu, before);
+                sb = s0w - 32;
+                ubase = before;
+            }
+        }
         int g = cid, base = -1, cnt = 0, gi = 0;
         for (;;) {
             int a = -1, my_tok = 0, L = 0;
             AdapterDesc d = {};
             if (SRC == kSrcSegments) {
                 while (L == 0) {
+                    if (un >= un_end) break;   // this cluster's run is done
                     while (un >= ubase + w_total && sb + 32 < nseg) {
                         ubase += w_total;
                         sb += 32;
@@ -437,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     const int p1 = __shfl_sync(0xffffffffu, w_p1, hl);
                     const int first_unit = ubase + __shfl_sync(0xffffffffu, w_incl - w_nu, hl);
                     const int start = __shfl_sync(0xffffffffu, w_p0, hl) + (un - first_unit) * kTokChunk;
-                    un += G;
+                    un += un_step;
                     d = p.pj[0].desc[sa];
                     const int L0 = min(kTokChunk, p1 - start);
                     int t = -1;

@@ -44,6 +44,7 @@ Options &options()
         o.split = env_or("LORA_SPLIT", o.split);
         o.tc_min_seg_len = env_or("LORA_TC_MIN_SEG_LEN", o.tc_min_seg_len);
         o.tc_min_tokens = env_or("LORA_TC_MIN_TOKENS", o.tc_min_tokens);
+        o.decode_balance = env_or("LORA_DECODE_BALANCE", o.decode_balance);
     });
     return o;
 }
@@ -131,6 +132,16 @@ int check_segments(const lora_segments *seg)
     return LORA_OK;
 }
 
+// Whether the decode kernel cuts segment-table units into cost-balanced runs per cluster: it
+// pays when unit costs differ widely, i.e. when the ranks do (measured: multi-rank 57.7 -> 45.3
+// us per step; with one rank the staging of the table costs more than the balance gains).
+int32_t balance_for(int min_rank, int max_rank)
+{
+    const int64_t o = options().decode_balance;
+    if (o >= 0) return o ? 1 : 0;
+    return max_rank >= 2 * min_rank ? 1 : 0;
+}
+
 DecodeParams base_params(const lora_table *t)
 {
     DecodeParams p;
@@ -145,6 +156,7 @@ DecodeParams base_params(const lora_table *t)
     p.w_stride = 1;
     p.n = t->n;
     p.R = t->max_rank;
+    p.balance = balance_for(t->min_rank, t->max_rank);
     p.status = t->d_status;
     p.wait_ns = wait_limit_ns();
     p.inject = (int32_t)(options().inject_stall & 1);
@@ -174,13 +186,14 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
     if (n < 1 || h < 1 || o < 1) return LORA_ERR_INVALID_ARG;
     if (dtype != LORA_BF16 && dtype != LORA_F32) return LORA_ERR_UNSUPPORTED;
     if (h % epc(dtype) || o % epc(dtype)) return LORA_ERR_UNSUPPORTED;
-    int max_rank = 0;
+    int max_rank = 0, min_rank = LORA_MAX_RANK;
     for (int i = 0; i < n; ++i) {
         if (!A[i] || !B[i]) return LORA_ERR_INVALID_ARG;
         if (ranks[i] < 1) return LORA_ERR_INVALID_ARG;
         if (ranks[i] > LORA_MAX_RANK) return LORA_ERR_UNSUPPORTED;
         if (!al16(A[i]) || !al16(B[i])) return LORA_ERR_UNSUPPORTED;
         if (ranks[i] > max_rank) max_rank = ranks[i];
+        if (ranks[i] < min_rank) min_rank = ranks[i];
     }
     lora_table *t = new (std::nothrow) lora_table();
     if (!t) return LORA_ERR_INVALID_ARG;
@@ -189,6 +202,7 @@ int lora_table_create(lora_table **out, int32_t n, int32_t h, int32_t o, int32_t
     t->o = o;
     t->dtype = dtype;
     t->max_rank = max_rank;
+    t->min_rank = min_rank;
     t->d_desc = nullptr;
     t->d_status = nullptr;
     t->d_tmaps = nullptr;
@@ -478,6 +492,7 @@ int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_seg
         pj.y_off = y_off[i];
         pj.sigma_kind = t->sigma_kind;
         if (t->max_rank > p.R) p.R = t->max_rank;
+        p.balance |= balance_for(t->min_rank, t->max_rank);
     }
     return launch_decode(kModeFused, kSrcSegments, p, tables[0]->dtype, static_cast<cudaStream_t>(stream));
 }
@@ -630,6 +645,7 @@ int lora_set_option(const char *key, int64_t value)
     else if (!std::strcmp(key, "inject_stall")) o.inject_stall = value;
     else if (!std::strcmp(key, "tc_min_seg_len")) o.tc_min_seg_len = value;
     else if (!std::strcmp(key, "tc_min_tokens")) o.tc_min_tokens = value;
+    else if (!std::strcmp(key, "decode_balance")) o.decode_balance = value;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }
@@ -650,6 +666,7 @@ int lora_get_option(const char *key, int64_t *value)
     else if (!std::strcmp(key, "inject_stall")) *value = o.inject_stall;
     else if (!std::strcmp(key, "tc_min_seg_len")) *value = o.tc_min_seg_len;
     else if (!std::strcmp(key, "tc_min_tokens")) *value = o.tc_min_tokens;
+    else if (!std::strcmp(key, "decode_balance")) *value = o.decode_balance;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }

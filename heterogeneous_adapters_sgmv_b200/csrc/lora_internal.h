@@ -50,6 +50,7 @@ struct DecodeParams {
     uint64_t wait_ns;      // bound of every device-side wait (option "wait_limit_ns")
     int32_t inject;        // test-only stall injection (option "inject_stall"), 0 in normal use
     int32_t long_len;      // segments of at least this many tokens are served elsewhere (0: none)
+    int32_t balance;       // segment tables: cost-balanced runs of units per cluster (1) or a fixed stride (0)
     int32_t stages;        // pipeline depth
     int32_t stage_bytes;   // bytes of one stage (header + data)
     int32_t ids_smem;      // kSrcIds: bytes of the id / leader scratch in shared memory
@@ -68,6 +69,7 @@ struct Options {
     int64_t inject_stall = 0;        // test-only: bit 0 decode, bit 1 prefill shrink, bit 2 prefill expand
     int64_t tc_min_seg_len = 64;     // mixed batches: segments this long take the tcgen05 kernels (0: never)
     int64_t tc_min_tokens = 1024;    // ... in batches of at least this many tokens
+    int64_t decode_balance = -1;     // segment units: -1 by the tables' rank spread, 0 fixed stride, 1 balanced runs
 };
 // Bound of the device-side waits for the next launch.
 uint64_t wait_limit_ns();
@@ -103,7 +105,7 @@ int encode_tmap_A(void *out128, const void *A, int dtype, int h, int rank);
 }  // namespace lora
 
 struct lora_table {
-    int32_t n, h, o, dtype, max_rank;
+    int32_t n, h, o, dtype, max_rank, min_rank;
     int device;
     lora::AdapterDesc *d_desc;
     uint32_t *d_status;

@@ -274,7 +274,10 @@ const char *lora_status_string(int code);
  * out, LORA_STATUS_TIMEOUT is latched and the kernel drains its copies, releases tensor
  * memory and returns; results are then invalid), "tc_min_seg_len" (segments at least this
  * long take the tcgen05 kernels in mixed batches; 0 disables that split), "tc_min_tokens"
- * (smallest batch that considers the split).  Returns LORA_ERR_INVALID_ARG for an unknown
+ * (smallest batch that considers the split), "decode_balance" (segment tables on the cluster
+ * kernel: -1, the default, cuts the units into runs of about equal estimated work per cluster
+ * when the table's ranks differ by 2x or more, else deals them with a fixed stride; 0 always the
+ * stride, 1 always the runs; results are bit-identical either way).  Returns LORA_ERR_INVALID_ARG for an unknown
  * key. */
 int lora_set_option(const char *key, int64_t value);
 int lora_get_option(const char *key, int64_t *value);

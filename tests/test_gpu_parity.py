@@ -225,6 +225,25 @@ def test_paths_agree_bit_for_bit(cluster):
     assert_close(dp.to_np(y_b), ref, wl.dtype, "small multirank")
 
 
+@pytest.mark.parametrize("name", ["multirank_decode", "many_adapter_qkvo"])
+def test_balanced_runs_and_stride_agree_bit_for_bit(name):
+    """Segment-table units dealt to the clusters as runs of about equal estimated work or with a
+    fixed stride: a unit is computed the same way on whichever cluster takes it, so y is
+    bit-identical, and both match the oracle."""
+    wl = workload(name)
+    ref = reference(name)
+    dp = DeviceProj(wl)
+    seg, _keep = dp.segments()
+    ys = {}
+    for b in (1, 0):
+        with option("decode_balance", b):
+            ys[b] = dp.sgmv(dp.y(), seg)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1])
+    assert_close(dp.to_np(ys[1]), ref, wl.dtype, name + " (balanced runs)")
+    assert dp.status() == (0, 0)
+
+
 def test_token_permutation_permutes_output_exactly():
     wl = _small("multirank_decode")
     dp = DeviceProj(wl)
