@@ -646,54 +646,74 @@ def run_ours(args, rank, world, local_rank):
     if args.base:
         roofline = tensor_roofline(flops_step, ms_step, launches_per_step, kname)
 
-    # end to end through the C ABI with host buffers: H2D inputs, the call, D2H of y
+    # end to end through the C ABI with host buffers: H2D inputs, the call, D2H of y.  Two
+    # device buffer sets and three streams, as a serving loop would run it: step i + 1's inputs
+    # go in (copy engine, host to device) while step i computes and step i - 1's output comes
+    # out (the other copy engine); every step still copies all of its inputs in and its result out.
     e2e = None
     if args.e2e_steps != 0:
-        c = copies[0]
-        hx = [torch.empty_like(p.x, device="cpu").pin_memory() for p in c.projs]
-        hy = [torch.empty_like(p.y0, device="cpu").pin_memory() for p in c.projs]
-        hout = [torch.empty_like(p.y0, device="cpu").pin_memory() for p in c.projs]
+        nb = 2 if len(copies) >= 2 else 1
+        bufs = copies[:nb]
+        hx = [torch.empty_like(p.x, device="cpu").pin_memory() for p in bufs[0].projs]
+        hy = [torch.empty_like(p.y0, device="cpu").pin_memory() for p in bufs[0].projs]
+        hout = [[torch.empty_like(p.y0, device="cpu").pin_memory() for p in bufs[0].projs] for _ in range(nb)]
         hids = torch.from_numpy(wl.ids).pin_memory()
-        for i, p in enumerate(c.projs):
+        for i, p in enumerate(bufs[0].projs):
             hx[i].copy_(p.x)
             hy[i].copy_(p.y0)
         h2d = sum(t.numel() * t.element_size() for t in hx + hy) + hids.numel() * 4
-        d2h = sum(t.numel() * t.element_size() for t in hout)
-        stream = tm.stream
+        d2h = sum(t.numel() * t.element_size() for t in hout[0])
+        s_in, s_run, s_out = torch.cuda.Stream(), tm.stream, torch.cuda.Stream()
         sh = tm.sh
+        out_done = [None] * nb
 
-        def e2e_step():
-            c.ids.copy_(hids, non_blocking=True)
-            for i, p in enumerate(c.projs):
-                p.x.copy_(hx[i], non_blocking=True)
-                p.y0.copy_(hy[i], non_blocking=True)
-            step(c, sh)
-            for i, p in enumerate(c.projs):
-                hout[i].copy_(p.y0, non_blocking=True)
+        def e2e_step(k):
+            b = k % nb
+            c = bufs[b]
+            with torch.cuda.stream(s_in):
+                if out_done[b] is not None:
+                    s_in.wait_event(out_done[b])   # this buffer's previous result is out
+                c.ids.copy_(hids, non_blocking=True)
+                for i, p in enumerate(c.projs):
+                    p.x.copy_(hx[i], non_blocking=True)
+                    p.y0.copy_(hy[i], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(ev_in)
+                step(c, sh)
+                ev_run = torch.cuda.Event()
+                ev_run.record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_run)
+                for i, p in enumerate(c.projs):
+                    hout[b][i].copy_(p.y0, non_blocking=True)
+                out_done[b] = torch.cuda.Event()
+                out_done[b].record(s_out)
 
-        with torch.cuda.stream(stream):
-            for _ in range(W):
-                e2e_step()
+        for k in range(W):
+            e2e_step(k)
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        with torch.cuda.stream(stream):
-            e2e_step()
+        e2e_step(0)
         torch.cuda.synchronize()
         Ke = args.e2e_steps if args.e2e_steps > 0 else int(max(20, min(5000, 1.5 / max(time.perf_counter() - t0, 1e-5))))
         if dist:
             dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(Ke):
-                e2e_step()
-            e1.record(stream)
+        e0.record(s_in)
+        for k in range(Ke):
+            e2e_step(k)
+        s_in.wait_stream(s_out)
+        e1.record(s_in)
         torch.cuda.synchronize()
         ems = max_over_ranks(float(e0.elapsed_time(e1)), dist, "cuda")
         e2e = {"value": round(job_throughput(world, T, Ke, ems), 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": Ke, "ms_per_step": round(ems / Ke, 6),
-               "path": "pinned host -> cudaMemcpyAsync -> C-ABI call -> cudaMemcpyAsync -> pinned host"}
+               "path": "pinned host -> cudaMemcpyAsync (copy stream) -> C-ABI call (compute stream) -> "
+                       "cudaMemcpyAsync (second copy stream) -> pinned host; %d device buffer sets" % nb}
     pdl = bool(L.lora_get_option("pdl"))
     free_copies(torch, copies)
 
