@@ -58,7 +58,7 @@ uint64_t wait_limit_ns()
 // prefill.cu
 bool prefill_supported(const lora_table *t);
 int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y,
-                   int64_t ldy, int32_t y_off, void *v, int32_t min_len, cudaStream_t s);
+                   int64_t ldy, int32_t y_off, void *v, int32_t *tile_ctr, int32_t min_len, cudaStream_t s);
 
 }  // namespace lora
 
@@ -78,7 +78,7 @@ inline size_t up256(size_t b) { return (b + 255) & ~size_t(255); }
 inline int ldv_of(const lora_table *t) { return (t->max_rank + 3) & ~3; }
 
 struct WsLayout {
-    size_t v, perm, seg_ptr, seg_adapter, num_segs, total;
+    size_t v, perm, seg_ptr, seg_adapter, num_segs, tile_ctr, total;
 };
 
 WsLayout ws_layout(const lora_table *t, int32_t T)
@@ -97,6 +97,7 @@ WsLayout ws_layout(const lora_table *t, int32_t T)
     w.seg_adapter = off;
     off += up256((size_t)t->n * sizeof(int32_t));
     w.num_segs = off;
+    w.tile_ctr = off + 128;   // the tcgen05 expand's tile counter, in the same 256-byte block
     off += 256;
     w.total = off;
     return w;
@@ -385,7 +386,8 @@ int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int6
         if (!ws || ws_bytes < w.total) return LORA_ERR_WORKSPACE;
         if (!al16(ws)) return LORA_ERR_UNSUPPORTED;
         float *v = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + w.v);
-        if (prefill) return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, 0, s);
+        int32_t *ctr = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.tile_ctr);
+        if (prefill) return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, ctr, 0, s);
         if ((rc = lora_shrink(t, seg, x, ldx, v, ldv_of(t), stream))) return rc;
         return lora_expand(t, seg, v, ldv_of(t), y, ldy, y_off, stream);
     }
@@ -404,8 +406,10 @@ int lora_sgmv(const lora_table *t, const lora_segments *seg, const void *x, int6
                        ws_bytes >= ws_layout(t, seg->T).total && al16(ws);
     if (mixed) p.long_len = (int32_t)opt.tc_min_seg_len;
     if ((rc = launch_decode(kModeFused, kSrcSegments, p, t->dtype, s)) != LORA_OK || !mixed) return rc;
-    float *v = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_layout(t, seg->T).v);
-    return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, (int32_t)opt.tc_min_seg_len, s);
+    const WsLayout w = ws_layout(t, seg->T);
+    float *v = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + w.v);
+    int32_t *ctr = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.tile_ctr);
+    return launch_prefill(t, seg, x, ldx, y, ldy, y_off, v, ctr, (int32_t)opt.tc_min_seg_len, s);
 }
 
 int lora_sgmv_base(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, const void *W,

@@ -92,6 +92,7 @@ struct PrefillParams {
     const int32_t *perm;          // token of each sorted position, or null (tokens contiguous)
     int32_t min_len;              // only segments of at least this many tokens (0: all)
     CUtensorMap tmap_g;           // perm: x [T, h] (shrink) or the y slice (expand), box 64 x 1
+    int32_t *tile_ctr;            // expand: next tile of the shared pool (zeroed by the shrink), or null
 };
 
 // 4-row gather (TMA tile::gather4, one-row box, 128-byte swizzle) of columns [c0, c0 + 64) of
@@ -218,6 +219,9 @@ __global__ void __launch_bounds__(kThreadsPF, 1) prefill_shrink_kernel(const __g
     pdl_wait();
     pdl_launch_dependents();
     if (tid == 0) SHRINK_MARK(1);
+    // the expand that follows deals the last tiles from a shared counter; the wait above means
+    // the previous expand on this workspace has finished with it
+    if (blockIdx.x == 0 && tid == 0 && p.tile_ctr) *p.tile_ctr = 0;
 
     if (warp == 0) {
         int s, row0 = 0, rows = 0, a = 0;
@@ -403,6 +407,7 @@ constexpr int kExBStages = 2;
 constexpr int kExYBytes = 32768;                       // y tile: two 64-column boxes of 128 rows
 constexpr int kExBBytes = 16384;                       // B_i tile: 128 rows of o x 64 ranks
 constexpr int kExVBytes = 32768;                       // hi + lo intermediate tile
+constexpr int kExPoolPerCta = 3;                       // tiles per CTA dealt from the shared pool
 
 struct ExTileInfo {
     int32_t row0, rows, col0, ncols, vb;
@@ -492,8 +497,15 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
     if (tid == 0) EXPAND_MARK(64, 1);
     const uint32_t tmem = ctl.tmem_base;
     const int total = ctl.total_m * NT;
-    const int t0 = (int)((int64_t)blockIdx.x * total / gridDim.x);
-    const int t1 = (int)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
+    // Each CTA first takes a contiguous share of the tiles (consecutive tiles share the
+    // intermediate tile); the last ~kExPoolPerCta per CTA form a pool dealt one at a time
+    // from a counter, so CTAs that started late or ran slow take fewer of them.  Without a
+    // counter every tile is in the contiguous shares.
+    const int G = (int)gridDim.x, b = (int)blockIdx.x;
+    const int S = p.tile_ctr ? max(0, total / G - kExPoolPerCta) : 0;
+    const int t0 = p.tile_ctr ? b * S : (int)((int64_t)b * total / G);
+    const int t1 = p.tile_ctr ? t0 + S : (int)((int64_t)(b + 1) * total / G);
+    const int pool0 = G * S;   // first pool tile (with a counter)
     bool ok = true;
 
     if (warp == 0) {
@@ -501,8 +513,25 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         int cur_g = -1, vcount = 0, row0 = 0, rows = 0, a = 0, vb = 0, nissued = 0;
         int tk[4] = {0, 0, 0, 0};   // with a permutation: tokens of rows 4 lane .. 4 lane + 3
         float sc = 0.f;
-        for (int t = t0; t < t1 && ok; ++t) {
-            const int i = t - t0, sy = i % kExYStages, sb = i % kExBStages;
+        int grab = 0;   // lane 0: pool index taken ahead of its use
+        for (int i = 0; ok; ++i) {
+            // the tile of stage i: the share, then pool tiles (the next index is taken one tile
+            // ahead, so the counter's round trip overlaps the tile before)
+            int t;
+            if (!p.tile_ctr) {
+                t = t0 + i;
+                if (t >= t1) break;
+            } else {
+                if (lane == 0 && i == max(S - 1, 0)) grab = atomicAdd(p.tile_ctr, 1);
+                if (i < S) {
+                    t = t0 + i;
+                } else {
+                    t = pool0 + __shfl_sync(0xffffffffu, grab, 0);
+                    if (t >= total) break;
+                    if (lane == 0) grab = atomicAdd(p.tile_ctr, 1);
+                }
+            }
+            const int sy = i % kExYStages, sb = i % kExBStages;
             const int g = t / NT, nt = t - g * NT;
             if (g != cur_g) {
                 int sg;
@@ -577,13 +606,34 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             ++nissued;
             __syncwarp();
         }
-        // drain: every TMA issued by this CTA has landed before shared memory is released (the
-        // stages of the last tiles armed; earlier ones were consumed before reuse)
+        // end of the tiles: a stage whose info has rows = -1, with its barriers completed by
+        // plain arrivals, tells the MMA issuer and the epilogue to stop
+        int sentinel = 0;
+        if (ok) {
+            const int i = nissued, sy = i % kExYStages, sb = i % kExBStages;
+            const bool oky = i < kExYStages || __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.yempty[sy]),
+                                                                                   ((i / kExYStages) - 1) & 1,
+                                                                                   p.status, p.wait_ns));
+            const bool okb = i < kExBStages || __all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.bempty[sb]),
+                                                                                   ((i / kExBStages) - 1) & 1,
+                                                                                   p.status, p.wait_ns));
+            if (oky && okb && lane == 0) {
+                ctl.info[sy].rows = -1;
+                mbar_arrive(smem_u32(&ctl.yfull[sy]));
+                mbar_arrive(smem_u32(&ctl.bfull[sb]));
+            }
+            sentinel = (oky && okb) ? 1 : 0;
+            __syncwarp();
+        }
+        // drain: every TMA issued by this CTA has landed before shared memory is released.  The
+        // stages of the last tiles armed hold the loads still in flight; earlier tiles' stages
+        // were consumed before reuse (the end-of-tiles stage reused one more of each ring, and
+        // waiting on that stage's older phase would never succeed).
         const int n = nissued;
         if (lane == 0) {
-            for (int i = max(0, n - kExYStages); i < n; ++i)
+            for (int i = max(0, n + sentinel - kExYStages); i < n; ++i)
                 mbar_wait(smem_u32(&ctl.yfull[i % kExYStages]), (i / kExYStages) & 1, p.status, p.wait_ns);
-            for (int i = max(0, n - kExBStages); i < n; ++i)
+            for (int i = max(0, n + sentinel - kExBStages); i < n; ++i)
                 mbar_wait(smem_u32(&ctl.bfull[i % kExBStages]), (i / kExBStages) & 1, p.status, p.wait_ns);
             for (int c = max(0, vcount - 2); c < vcount; ++c)
                 mbar_wait(smem_u32(&ctl.vfull[c & 1]), (c >> 1) & 1, p.status, p.wait_ns);
@@ -593,10 +643,17 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(kTileM, kTileN);
             int vuse = 0, prev_vb = -1;
-            for (int t = t0; t < t1; ++t) {
-                const int i = t - t0, sy = i % kExYStages, sb = i % kExBStages, ab = i & 1;
+            for (int i = 0;; ++i) {
+                const int sy = i % kExYStages, sb = i % kExBStages, ab = i & 1;
                 if (!mbar_wait(smem_u32(&ctl.bfull[sb]), (i / kExBStages) & 1, p.status, p.wait_ns)) break;
                 EXPAND_MARK(i, 1);
+                if (ctl.info[sy].rows < 0) {
+                    // end of the tiles: complete the accumulator barrier the epilogue waits on
+                    // next (once it is done with this accumulator's previous tile)
+                    if (i < 2 || mbar_wait(smem_u32(&ctl.accempty[ab]), ((i >> 1) - 1) & 1, p.status, p.wait_ns))
+                        umma_commit(smem_u32(&ctl.accfull[ab]));
+                    break;
+                }
                 const int vb = ctl.info[sy].vb;
                 if (vb != prev_vb) {
                     if (prev_vb >= 0) umma_commit(smem_u32(&ctl.vempty[prev_vb]));   // old tile may be rebuilt
@@ -629,8 +686,8 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         const int m = q * 32 + lane;            // row of the tile
         const int ew = warp - 2;                // epilogue warp 0..7
         int pending = -1;                       // ew 0: y stage whose TMA store is still reading it
-        for (int t = t0; t < t1; ++t) {
-            const int i = t - t0, sy = i % kExYStages, ab = i & 1;
+        for (int i = 0;; ++i) {
+            const int sy = i % kExYStages, ab = i & 1;
             // every epilogue warp leaves together if any lane ran out of time (the tensor-memory
             // loads below are warp-collective and the warps meet at a named barrier)
             const bool oka = mbar_wait(smem_u32(&ctl.accfull[ab]), (i >> 1) & 1, p.status, p.wait_ns);
@@ -639,6 +696,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             tc_fence_after();
             if (ew == 0 && lane == 0) EXPAND_MARK(i, 2);
             const ExTileInfo inf = ctl.info[sy];
+            if (inf.rows < 0) break;   // end of the tiles (the same for every thread)
             uint8_t *yt = yring + sy * kExYBytes + half * 16384;   // this half's 64-column box
             float acc[64];
             tmem_ld64(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(ab * kTileN + half * 64), acc);
@@ -859,7 +917,7 @@ int launch_prefill_shrink(const lora_table *t, const lora_segments *seg, const v
 }
 
 int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, void *y, int64_t ldy,
-                   int32_t y_off, void *v, int32_t min_len, cudaStream_t s)
+                   int32_t y_off, void *v, int32_t *tile_ctr, int32_t min_len, cudaStream_t s)
 {
     if (!prefill_supported(t)) return LORA_ERR_UNSUPPORTED;
     int rc = set_prefill_attributes();
@@ -869,6 +927,7 @@ int launch_prefill(const lora_table *t, const lora_segments *seg, const void *x,
     p.ldy = ldy;
     p.y_off = y_off;
     p.min_len = min_len;
+    p.tile_ctr = tile_ctr;
     const int mt_bound = tile_bound(seg, min_len);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return LORA_ERR_CUDA;
