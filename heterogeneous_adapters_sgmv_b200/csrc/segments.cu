@@ -214,23 +214,24 @@ count_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int
         seg_ptr[segs] = valid;
         *num_segs = segs;
     }
-    __syncthreads();   // every thread has read cnt[] before warp 0 advances it
-    if (warp == 0) {
-        for (int t0 = 0; t0 < T; t0 += 32) {
-            const int t = t0 + lane;
-            const bool ok = t < T;
-            const int32_t key = ok ? key_s[t] : -1;
-            const uint32_t peers = __match_any_sync(0xffffffffu, key);
-            const int leader = __ffs(peers) - 1;
-            int32_t base = 0;
-            if (ok && lane == leader && key < n) {
-                base = cnt[key];
-                cnt[key] = base + __popc(peers);
-            }
-            base = __shfl_sync(0xffffffffu, base, leader);
-            if (ok && key < n) perm[base + __popc(peers & ((1u << lane) - 1u))] = t;
-            __syncwarp();
+    // Place every token at its adapter's first position plus the number of earlier tokens with
+    // the same adapter (the stable order), all tokens at once: a thread counts the matches
+    // among the keys before its token, read from shared memory in step by its warp's lanes
+    // (one broadcast per key), 32 keys per step.
+    for (int t0 = warp * 32; t0 < T; t0 += kSegThreads) {
+        const int t = t0 + lane;
+        const bool ok = t < T;
+        const int32_t key = ok ? key_s[t] : -1;
+        int rank = 0;
+        for (int u0 = 0; u0 < t0; u0 += 32) {
+            const int32_t ku = key_s[u0 + lane];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) rank += __shfl_sync(0xffffffffu, ku, j) == key;
         }
+        // the warp's own earlier lanes
+        const uint32_t peers = __match_any_sync(0xffffffffu, key);
+        rank += __popc(peers & ((1u << lane) - 1u));
+        if (ok && key < n) perm[cnt[key] + rank] = t;
     }
 }
 
