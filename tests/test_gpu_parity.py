@@ -504,6 +504,23 @@ def test_prefill_tcgen05_zero_B_leaves_y_bit_identical():
     assert torch.equal(y, dp.d.y0)
 
 
+def test_prefill_tcgen05_reuses_one_workspace():
+    """Calls on one workspace back to back (the expand deals its last tiles from a counter in the
+    workspace, which each call's shrink resets): every call matches the oracle and the first."""
+    wl, dp, seg, _keep = _prefill_case([512, 384, 200], 4096, 2048, (64,))
+    ref = oracle.workload_reference(wl)
+    ws = dp.workspace()
+    ys = []
+    for _ in range(3):
+        y = dp.y()
+        L.lora_sgmv(dp.table.handle, seg, dp.d.x, dp.d.x.shape[1], y, y.shape[1], 0, ws, ws.numel())
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+    assert_close(dp.to_np(ys[2]), ref, wl.dtype, "tcgen05 prefill, reused workspace")
+    assert dp.status() == (0, 0)
+
+
 def test_prefill_tcgen05_deterministic():
     wl, dp, seg, _keep = _prefill_case([512, 384], 4096, 2048, (64,))
     y1 = dp.sgmv(dp.y(), seg)
