@@ -37,7 +37,7 @@ LORA_SIGMA_NONE = 0
 LORA_SIGMA_FULL = 1
 LORA_SIGMA_DIAG = 2
 LORA_MAX_MERGE = 8
-LORA_KERNEL_KINDS = 6
+LORA_KERNEL_KINDS = 7
 
 EXPORTS = (
     "lora_table_create", "lora_table_destroy", "lora_table_info", "lora_workspace_bytes",

@@ -717,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         if (pi > 0 || j >= skip) issue_tile(g, pi, j, a, d, s);
                     }
                     // L2 hints for the rows the consumers load for this tile (lane l: row l)
-                    if (lane < L) {
+                    if (lane < L && (shrink || !p.yacc)) {
                         const uint8_t *row =
                             shrink ? static_cast<const uint8_t *>(pj.x) + ((int64_t)my_tok * pj.ldx + off) * ESZ
                                    : static_cast<const uint8_t *>(pj.y) + ((int64_t)my_tok * pj.ldy + pj.y_off + off) * ESZ;
@@ -773,7 +773,9 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             const int e = tid + kConsumers * i;
             const int l = e >> lgC, c = e & (CHUNKS - 1);
             ld[i] = make_uint4(0, 0, 0, 0);
-            if (l < L && c < nch) ld[i] = *reinterpret_cast<const uint4 *>(src + h.tok[l] * ld_row + c * 16);
+            // with an fp32 sum (merged ensembles) the expand never reads y
+            if (l < L && c < nch && (xr || !p.yacc))
+                ld[i] = *reinterpret_cast<const uint4 *>(src + h.tok[l] * ld_row + c * 16);
         }
     };
     bool live = named_bar_and(1, kConsumers, mbar_wait(smem_u32(&ctl.meta[0]), 0, p.status, p.wait_ns));
@@ -1111,7 +1113,13 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         const float sl = sc * hdr.tw[l + q];   // exact when the weight is 1
                         const uint8_t *yr = ys + (l + q) * rowb + c * ESZ;
                         const int64_t gofs = (int64_t)hdr.tok[l + q] * pj.ldy + pj.y_off + off + c;
-                        if constexpr (CPT == 2) {
+                        if (p.yacc) {
+                            // merged ensembles: the slot's term goes into the fp32 sum, rounded
+                            // into y once after the last slot
+                            float *ya = p.yacc + (int64_t)hdr.tok[l + q] * p.ldacc + off + c;
+#pragma unroll
+                            for (int j = 0; j < CPT; ++j) ya[j] = fmaf(sl, acc[j], ya[j]);
+                        } else if constexpr (CPT == 2) {
                             const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
                             const float y0 = fmaf(sl, acc[0], bf16_lo(w));
                             const float y1 = fmaf(sl, acc[1], bf16_hi(w));

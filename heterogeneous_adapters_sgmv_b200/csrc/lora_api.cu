@@ -24,7 +24,7 @@ static int64_t env_or(const char *name, int64_t dflt)
 static std::atomic<int64_t> g_launches[kKernKinds];
 static const char *const kKernelNames[kKernKinds] = {
     "lora_decode_kernel", "count_segments_kernel", "build_segments_kernel", "prefill_shrink_kernel",
-    "prefill_expand_kernel", "base_gemm_kernel",
+    "prefill_expand_kernel", "base_gemm_kernel", "merge_finish_kernel",
 };
 
 void note_launch(KernelKind k) { g_launches[k].fetch_add(1, std::memory_order_relaxed); }
@@ -560,7 +560,15 @@ int lora_bgmv_merged(const lora_table *t, const int32_t *d_ids, const float *d_w
     if (!direct && (!ws || ws_bytes < w.total)) return LORA_ERR_WORKSPACE;
     if (!direct && !al16(ws)) return LORA_ERR_UNSUPPORTED;
     // One pass per slot, in slot order: each pass is the BGMV update of that slot's adapters
-    // with the per-token weight folded into the scale; y is rounded after each pass.
+    // with the per-token weight folded into the scale.  With room for an fp32 [T, o] sum after
+    // the workspace's own areas the passes add into that sum (zeroed first) and one last launch
+    // rounds y + sum once; otherwise y is rounded after each pass.
+    const size_t acc_off = (w.total + 255) / 256 * 256;
+    const size_t acc_bytes = (size_t)T * t->o * sizeof(float);
+    float *yacc = (ws && al16(ws) && ws_bytes >= acc_off + acc_bytes)
+                      ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + acc_off)
+                      : nullptr;
+    if (yacc && cudaMemsetAsync(yacc, 0, acc_bytes, s) != cudaSuccess) return LORA_ERR_CUDA;
     for (int k = 0; k < K; ++k) {
         DecodeParams p = base_params(t);
         p.pj[0].x = x;
@@ -570,6 +578,8 @@ int lora_bgmv_merged(const lora_table *t, const int32_t *d_ids, const float *d_w
         p.pj[0].y_off = y_off;
         p.tok_w = d_w + k;
         p.w_stride = K;
+        p.yacc = yacc;
+        p.ldacc = t->o;
         if (direct) {
             p.ids = d_ids + k;
             p.ids_stride = K;
@@ -600,6 +610,7 @@ int lora_bgmv_merged(const lora_table *t, const int32_t *d_ids, const float *d_w
         }
         if (rc) return rc;
     }
+    if (yacc) return launch_merge_finish(y, ldy, y_off, yacc, t->o, T, t->o, t->dtype, s);
     return LORA_OK;
 }
 

@@ -51,6 +51,8 @@ struct DecodeParams {
     int32_t inject;        // test-only stall injection (option "inject_stall"), 0 in normal use
     int32_t long_len;      // segments of at least this many tokens are served elsewhere (0: none)
     int32_t balance;       // segment tables: cost-balanced runs of units per cluster (1) or a fixed stride (0)
+    float *yacc;           // fused / expand: add the scaled delta to this fp32 [T, ldacc] array instead of
+    int64_t ldacc;         // rounding it into y (merged ensembles summed before their one rounding), or null
     int32_t stages;        // pipeline depth
     int32_t stage_bytes;   // bytes of one stage (header + data)
     int32_t ids_smem;      // kSrcIds: bytes of the id / leader scratch in shared memory
@@ -78,7 +80,7 @@ Options &options();
 // Host-side count of accepted launches per kernel (lora_kernel_launches).
 enum KernelKind {
     kKernDecode = 0, kKernCountSegments, kKernBuildSegments, kKernPrefillShrink, kKernPrefillExpand,
-    kKernBaseGemm, kKernKinds
+    kKernBaseGemm, kKernMergeFinish, kKernKinds
 };
 void note_launch(KernelKind k);
 
@@ -99,6 +101,9 @@ int launch_prefill_shrink(const lora_table *t, const lora_segments *seg, const v
 int launch_base_gemm(const lora_table *t, const lora_segments *seg, const void *x, int64_t ldx, const void *W,
                      int64_t ldw, void *y, int64_t ldy, int32_t y_off, int accumulate, const void *v, bool after_shrink,
                      cudaStream_t s);
+// y[t, y_off + n] = round(y[t, y_off + n] + yacc[t, n]) for t < T, n < o (merge.cu).
+int launch_merge_finish(void *y, int64_t ldy, int32_t y_off, const float *yacc, int64_t ldacc, int32_t T, int32_t o,
+                        int dtype, cudaStream_t s);
 // Encode the TMA tensor map of A_i [rank, h] used by the decode shrink (host side).
 int encode_tmap_A(void *out128, const void *A, int dtype, int h, int rank);
 

@@ -222,10 +222,13 @@ int lora_bgmv(const lora_table *table, const int32_t *d_ids, int32_t T, const vo
  *   y[t, y_offset + n] += sum_{j < K, ids[t, j] >= 0} w[t, j] * s_i * (B_i (A_i x[t]))[n]
  * d_ids and d_w are [T, K] row-major DEVICE arrays (int32 ids, -1 = empty slot; fp32
  * weights), 1 <= K <= LORA_MAX_MERGE.  Runs one BGMV pass per slot, in slot order, with the
- * weight folded into the scale, so y is rounded to its type after each slot (K roundings
- * instead of one).  Batches above 1024 tokens or 4096 adapters sort each slot into the
- * workspace (ws_bytes >= lora_workspace_bytes(table, T)); otherwise ws may be NULL.  The
- * "split" option does not apply. */
+ * weight folded into the scale.  With a workspace of at least
+ *   W + T * h_out * 4 bytes,   W = lora_workspace_bytes(table, T) rounded up to 256,
+ * (16-byte aligned) the passes add into an fp32 sum held after the first W bytes (zeroed
+ * first) and a last launch rounds y + sum once, as one weighted update; with less (or no)
+ * workspace y is rounded to its type after each slot (K roundings).  Batches above 1024 tokens
+ * or 4096 adapters sort each slot into the workspace (ws_bytes >= lora_workspace_bytes(table,
+ * T)); otherwise ws may be NULL.  The "split" option does not apply. */
 #define LORA_MAX_MERGE 8
 int lora_bgmv_merged(const lora_table *table, const int32_t *d_ids, const float *d_w, int32_t T,
                      int32_t K, const void *x, int64_t ldx, void *y, int64_t ldy, int32_t y_offset,
@@ -285,12 +288,13 @@ int lora_get_option(const char *key, int64_t *value);
 /* Launch counters (diagnostics, process-wide): the number of launches of each of the library's
  * kernels that the CUDA runtime has accepted since the library was loaded.  kind runs from 0 to
  * LORA_KERNEL_KINDS - 1 (0 the decode kernel, 1 and 2 the two segment-building kernels, 3 and
- * 4 the tcgen05 shrink and expand, 5 the fused base GEMM).  lora_kernel_name returns the
+ * 4 the tcgen05 shrink and expand, 5 the fused base GEMM, 6 the merged ensembles' final
+ * rounding).  lora_kernel_name returns the
  * kernel's name (static text; NULL outside that range) and lora_kernel_launches its count (-1
  * outside that range).  A count says that a launch was enqueued, not that it has finished;
  * lora_get_status reports what the device found.  Tests read them to see which path a call
  * took. */
-#define LORA_KERNEL_KINDS 6
+#define LORA_KERNEL_KINDS 7
 const char *lora_kernel_name(int32_t kind);
 int64_t lora_kernel_launches(int32_t kind);
 
