@@ -43,6 +43,7 @@
 
 #include <climits>
 #include <mutex>
+#include <type_traits>
 
 #include "lora_common.cuh"
 #include "lora_internal.h"
@@ -1058,79 +1059,87 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     krot = ((tid >> sh) & (nchk - 1)) * EPC;
                 }
             }
-            if (c < len) {
-                // Two tokens per pass share each load of this thread's B rows; per output the
-                // products are added in one fixed order (the thread's rotated chunk order).
+            // TG tokens per pass share each load (and unpacking) of this thread's B rows: two
+            // for the 1-2 token units of wide batches, four for larger units.  Per
+            // output the products are added in one fixed order (the thread's rotated chunk
+            // order) whatever TG is.  Rows of vsum past L hold stale values; their sums are
+            // formed but never stored.
+            auto expand_pass = [&](auto tg, int l0) {
+                constexpr int TG = decltype(tg)::value;
                 const uint8_t *brow = data + (size_t)c * r * ESZ;   // CPT consecutive rows of B
-                for (int l = 0; l < L; l += 2) {
-                    const bool l2 = l + 1 < L;   // row l + 1 of vsum exists even when unused
-                    const float *vr0 = vsum + l * RP, *vr1 = vr0 + RP;
-                    float acc0[CPT], acc1[CPT];
+                float acc[TG][CPT];
 #pragma unroll
-                    for (int j = 0; j < CPT; ++j) acc0[j] = acc1[j] = 0.f;
-                    if ((r % EPC) == 0) {
-                        // Each thread starts its walk over the 16-byte chunks of its B rows at
-                        // a rotated chunk, so the lanes of a quarter warp read different bank
-                        // groups (rows of 2 r bytes would otherwise put them on one group).
-                        for (int kk = 0; kk < r; kk += EPC) {
-                            int k = kk + krot;
-                            if (k >= r) k -= r;
-                            float v0[EPC], v1[EPC];
+                for (int q = 0; q < TG; ++q)
+#pragma unroll
+                    for (int j = 0; j < CPT; ++j) acc[q][j] = 0.f;
+                if ((r % EPC) == 0) {
+                    // Each thread starts its walk over the 16-byte chunks of its B rows at a
+                    // rotated chunk, so the lanes of a quarter warp read different bank groups
+                    // (rows of 2 r bytes would otherwise put them on one group).
+                    for (int kk = 0; kk < r; kk += EPC) {
+                        int k = kk + krot;
+                        if (k >= r) k -= r;
+                        float b[CPT][EPC];
+#pragma unroll
+                        for (int j = 0; j < CPT; ++j)
+                            cvt16(*reinterpret_cast<const uint4 *>(brow + ((size_t)j * r + k) * ESZ), b[j],
+                                  (E *)nullptr);
+#pragma unroll
+                        for (int q = 0; q < TG; ++q) {
+                            const float *vr = vsum + (l0 + q) * RP + k;
+                            float v[EPC];
 #pragma unroll
                             for (int e = 0; e < EPC; e += 4) {
-                                const float4 a4 = *reinterpret_cast<const float4 *>(vr0 + k + e);
-                                const float4 b4 = *reinterpret_cast<const float4 *>(vr1 + k + e);
-                                v0[e] = a4.x; v0[e + 1] = a4.y; v0[e + 2] = a4.z; v0[e + 3] = a4.w;
-                                v1[e] = b4.x; v1[e + 1] = b4.y; v1[e + 2] = b4.z; v1[e + 3] = b4.w;
+                                const float4 a4 = *reinterpret_cast<const float4 *>(vr + e);
+                                v[e] = a4.x; v[e + 1] = a4.y; v[e + 2] = a4.z; v[e + 3] = a4.w;
                             }
 #pragma unroll
-                            for (int j = 0; j < CPT; ++j) {
-                                float b[EPC];
-                                cvt16(*reinterpret_cast<const uint4 *>(brow + ((size_t)j * r + k) * ESZ), b,
-                                      (E *)nullptr);
+                            for (int j = 0; j < CPT; ++j)
 #pragma unroll
-                                for (int e = 0; e < EPC; ++e) {
-                                    acc0[j] = fmaf(v0[e], b[e], acc0[j]);
-                                    acc1[j] = fmaf(v1[e], b[e], acc1[j]);
-                                }
-                            }
-                        }
-                    } else {
-                        for (int k = 0; k < r; ++k) {
-#pragma unroll
-                            for (int j = 0; j < CPT; ++j) {
-                                const float b = (float)reinterpret_cast<const E *>(brow)[j * r + k];
-                                acc0[j] = fmaf(vr0[k], b, acc0[j]);
-                                acc1[j] = fmaf(vr1[k], b, acc1[j]);
-                            }
+                                for (int e = 0; e < EPC; ++e) acc[q][j] = fmaf(v[e], b[j][e], acc[q][j]);
                         }
                     }
-                    if (tid == 0 && l == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(32 + 2 * (it - kTraceTile0));
+                } else {
+                    for (int k = 0; k < r; ++k) {
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        if (q == 1 && !l2) break;
-                        const float *acc = q == 0 ? acc0 : acc1;
-                        const float sl = sc * hdr.tw[l + q];   // exact when the weight is 1
-                        const uint8_t *yr = ys + (l + q) * rowb + c * ESZ;
-                        const int64_t gofs = (int64_t)hdr.tok[l + q] * pj.ldy + pj.y_off + off + c;
-                        if (p.yacc) {
-                            // merged ensembles: the slot's term goes into the fp32 sum, rounded
-                            // into y once after the last slot
-                            float *ya = p.yacc + (int64_t)hdr.tok[l + q] * p.ldacc + off + c;
+                        for (int j = 0; j < CPT; ++j) {
+                            const float b = (float)reinterpret_cast<const E *>(brow)[j * r + k];
 #pragma unroll
-                            for (int j = 0; j < CPT; ++j) ya[j] = fmaf(sl, acc[j], ya[j]);
-                        } else if constexpr (CPT == 2) {
-                            const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
-                            const float y0 = fmaf(sl, acc[0], bf16_lo(w));
-                            const float y1 = fmaf(sl, acc[1], bf16_hi(w));
-                            *reinterpret_cast<uint32_t *>(static_cast<E *>(pj.y) + gofs) = pack_bf16x2(y0, y1);
-                        } else {
-                            const float w = *reinterpret_cast<const float *>(yr);
-                            static_cast<float *>(pj.y)[gofs] = fmaf(sl, acc[0], w);
+                            for (int q = 0; q < TG; ++q) acc[q][j] = fmaf(vsum[(l0 + q) * RP + k], b, acc[q][j]);
                         }
                     }
-                    if (tid == 0 && l == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(33 + 2 * (it - kTraceTile0));
                 }
+                if (tid == 0 && l0 == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(32 + 2 * (it - kTraceTile0));
+#pragma unroll
+                for (int q = 0; q < TG; ++q) {
+                    const int l = l0 + q;
+                    if (l >= L) break;
+                    const float sl = sc * hdr.tw[l];   // exact when the weight is 1
+                    const uint8_t *yr = ys + l * rowb + c * ESZ;
+                    const int64_t gofs = (int64_t)hdr.tok[l] * pj.ldy + pj.y_off + off + c;
+                    if (p.yacc) {
+                        // merged ensembles: the slot's term goes into the fp32 sum, rounded
+                        // into y once after the last slot
+                        float *ya = p.yacc + (int64_t)hdr.tok[l] * p.ldacc + off + c;
+#pragma unroll
+                        for (int j = 0; j < CPT; ++j) ya[j] = fmaf(sl, acc[q][j], ya[j]);
+                    } else if constexpr (CPT == 2) {
+                        const uint32_t w = *reinterpret_cast<const uint32_t *>(yr);
+                        const float y0 = fmaf(sl, acc[q][0], bf16_lo(w));
+                        const float y1 = fmaf(sl, acc[q][1], bf16_hi(w));
+                        *reinterpret_cast<uint32_t *>(static_cast<E *>(pj.y) + gofs) = pack_bf16x2(y0, y1);
+                    } else {
+                        const float w = *reinterpret_cast<const float *>(yr);
+                        static_cast<float *>(pj.y)[gofs] = fmaf(sl, acc[q][0], w);
+                    }
+                }
+                if (tid == 0 && l0 == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(33 + 2 * (it - kTraceTile0));
+            };
+            if (c < len) {
+                if (L <= 2)
+                    expand_pass(std::integral_constant<int, 2>(), 0);
+                else
+                    for (int l0 = 0; l0 < L; l0 += 4) expand_pass(std::integral_constant<int, 4>(), l0);
             }
         }
         if (tid == 0 && (unsigned)(it - kTraceTile0) < 2u) LORA_TRACE_MARK(9 + 5 * (it - kTraceTile0));

@@ -4,11 +4,12 @@
 //
 // Two single-CTA (1024-thread) kernels, both giving the unique stable order, bit-identical
 // run to run:
-//  * counting sort, for decode-sized batches (T <= 2048, n < 8192): one histogram of the
+//  * counting sort, for decode-sized batches (T <= 512, n < 8192): one histogram of the
 //    adapter ids in shared memory (warp-aggregated atomics: counts only, not positions), one
 //    exclusive scan giving each adapter's first position and one giving segment indices,
-//    then one warp walks the tokens in batch order and places them (ties inside a warp
-//    broken by lane order), so positions never depend on timing;
+//    then every token is placed at its adapter's first position plus the number of earlier
+//    tokens with the same adapter, so positions never depend on timing (that count costs
+//    O(T^2) compares over the block, which is why larger batches take the radix sort);
 //  * least-significant-digit radix sort for the rest (8-bit digits, as many passes as the
 //    adapter count needs).  Every pass is stable: each warp owns a contiguous run of the
 //    input, counts its digits into a private histogram row, the rows are scanned digit-major
@@ -235,7 +236,7 @@ count_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int
     }
 }
 
-constexpr int kCountMaxT = 2048;
+constexpr int kCountMaxT = 512;   // above this the radix sort is faster (measured)
 constexpr int kCountMaxN = 8191;
 
 }  // namespace

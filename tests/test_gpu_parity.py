@@ -113,20 +113,21 @@ def test_std_reading_of_the_weight_law(name):
 @pytest.mark.parametrize("case", ["decode_bgmv", "multirank_decode", "many_adapter_qkvo", "prefill_sgmv",
                                   "edge_empty", "edge_one", "edge_all_none", "edge_max_T", "edge_large_n",
                                   "edge_single_adapter", "edge_count_max", "edge_sort_T", "edge_sort_n",
-                                  "edge_heavy"])
+                                  "edge_heavy", "edge_count_max_T", "edge_radix_T", "edge_heavy_2048"])
 def test_build_segments_bit_exact(case):
-    """Both bookkeeping kernels (counting sort up to 2048 tokens and 8191 adapters, radix sort
+    """Both bookkeeping kernels (counting sort up to 512 tokens and 8191 adapters, radix sort
     beyond) against the oracle's stable counting sort, including both sides of the switch."""
     rng = np.random.default_rng(17)
     if case.startswith("edge"):
         n, T = {"edge_empty": (5, 0), "edge_one": (5, 1), "edge_all_none": (7, 300),
                 "edge_max_T": (1000, L.LORA_MAX_SEGMENT_TOKENS), "edge_large_n": (70000, 3000),
                 "edge_single_adapter": (1, 777), "edge_count_max": (8191, 2048), "edge_sort_T": (100, 2049),
-                "edge_sort_n": (8192, 2048), "edge_heavy": (5, 2048)}[case]
+                "edge_sort_n": (8192, 2048), "edge_heavy": (5, 512), "edge_count_max_T": (8191, 512),
+                "edge_radix_T": (100, 513), "edge_heavy_2048": (5, 2048)}[case]
         ids = rng.integers(-1, n, size=T).astype(np.int32)
         if case == "edge_all_none":
             ids[:] = -1
-        if case == "edge_heavy":   # one adapter carries most tokens: long runs of equal ids
+        if case.startswith("edge_heavy"):   # one adapter carries most tokens: long runs of equal ids
             ids[rng.random(T) < 0.9] = 2
         wl = workload("tiny_sgmv")
         dp = DeviceProj(wl)
