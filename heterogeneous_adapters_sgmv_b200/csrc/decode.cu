@@ -116,24 +116,30 @@ struct Layout {
 
 __host__ __device__ inline int row_bytes_for(int R) { return R > 64 ? kRowBytes / 2 : kRowBytes; }
 
-__host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int stages, int stage_bytes, int CL)
+// VP: projections whose intermediates share one exchange (a grouped launch with one exchange
+// per unit), else 1.  A token's row of the partial / intermediate holds VP slices of RP floats.
+__host__ __device__ inline Layout make_layout(int src, int R, int n, int T, int stages, int stage_bytes, int CL,
+                                              int VP)
 {
     Layout l;
     const int rowb = row_bytes_for(R);
     l.RP = round_up(R, 8);
+    const int VS = VP * l.RP;
     l.ids_off = kCtlBytes;
     // ids, first member and count per adapter, leaders, weights, chunk offsets per group
     const int ids_bytes = (src == kSrcIds) ? round_up(4 * (4 * T + n + 1), 128) : 0;
+    // x rows (shrink tiles) and y rows (expand tiles) share one buffer: a tile stages only one
+    // of them, after every consumer is done with the previous tile's
     l.xs_off = l.ids_off + ids_bytes;
-    l.ys_off = l.xs_off + kTokChunk * rowb;
+    l.ys_off = l.xs_off;
     l.vpart_off = l.ys_off + kTokChunk * rowb;
-    l.recv_off = l.vpart_off + round_up(kTokChunk * l.RP * 4, 128);
+    l.recv_off = l.vpart_off + round_up(kTokChunk * VS * 4, 128);
     if (CL > 1) {
-        l.vsum_off = l.recv_off + CL * kTokChunk * l.RP * 4;
-        l.stage_off = l.vsum_off + round_up(kTokChunk * l.RP * 4, 128);
+        l.vsum_off = l.recv_off + CL * kTokChunk * VS * 4;
+        l.stage_off = l.vsum_off + round_up(kTokChunk * VS * 4, 128);
     } else {   // no exchange: the CTA's own partial is the unit's intermediate
         l.recv_off = l.vsum_off = l.vpart_off;
-        l.stage_off = l.vpart_off + round_up(kTokChunk * l.RP * 4, 128);
+        l.stage_off = l.vpart_off + round_up(kTokChunk * VS * 4, 128);
     }
     l.total = l.stage_off + stages * stage_bytes;
     return l;
@@ -179,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
 
     extern __shared__ __align__(128) uint8_t smem[];
     SmemCtl &ctl = *reinterpret_cast<SmemCtl *>(smem);
-    const Layout lay = make_layout(SRC, p.R, p.n, p.T, p.stages, p.stage_bytes, CL);
+    const int VP = p.mx ? p.P : 1;   // projections sharing one exchange per unit
+    const Layout lay = make_layout(SRC, p.R, p.n, p.T, p.stages, p.stage_bytes, CL, VP);
     uint8_t *xs = smem + lay.xs_off;
     uint8_t *ys = smem + lay.ys_off;
     float *vpart = reinterpret_cast<float *>(smem + lay.vpart_off);   // [kTokChunk][RP] this CTA's partial
@@ -188,6 +195,8 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
     uint8_t *stage_base = smem + lay.stage_off;
     const int RP = lay.RP;
     const int lgRP = ceil_log2(RP);
+    const int VS = VP * RP;                // floats per token row of vpart / recv / vsum
+    const int lgVS = ceil_log2(VS);
     const int S = p.stages;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -669,18 +678,25 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             if (lane == 0) LORA_TRACE_MARK(2);
             const int skip = npre;
             npre = 0;
-            for (int pi = 0; pi < p.P && alive; ++pi) {
+            // With a shared exchange (grouped launch, option decode_shared_exchange) the unit's
+            // shrink tiles of every projection come first, then all its expand tiles: the
+            // consumers exchange the projections' partials once, after the last shrink tile.
+            const int npass = p.mx ? 2 : 1;
+            for (int step = 0; step < npass * p.P && alive; ++step) {
+                const int pass = step / p.P, pi = step - pass * p.P;
                 const ProjParams &pj = p.pj[pi];
-                if (pi > 0) d = pj.desc[a];
+                const AdapterDesc dd = pi == 0 ? d : pj.desc[a];
                 const Geo g = pi == 0 ? geo0 : geo_of(pi);
-                const int r = d.rank;
+                const int r = dd.rank;
                 const int ntiles = g.n_shrink + g.n_expand;
+                const int j0 = (p.mx && pass == 1) ? g.n_shrink : 0;
+                const int j1 = (p.mx && pass == 0) ? g.n_shrink : ntiles;
                 if (pj.sigma_kind != LORA_SIGMA_NONE) {   // the consumers read Sigma_i after the shrink
                     const int sbytes = (pj.sigma_kind == LORA_SIGMA_FULL ? r * r : r) * 4;
                     for (int c = lane * 128; c < sbytes; c += 32 * 128)
-                        prefetch_l2(reinterpret_cast<const uint8_t *>(d.sigma) + c);
+                        prefetch_l2(reinterpret_cast<const uint8_t *>(dd.sigma) + c);
                 }
-                for (int j = 0; j < ntiles; ++j) {
+                for (int j = j0; j < j1; ++j) {
                     const int s = ps, m = pround;
                     if (m >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status,
                                                                       p.wait_ns))) {
@@ -701,21 +717,23 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         hdr->kind = shrink ? kTileShrink : kTileExpand;
                         const int first_j = shrink ? 0 : g.n_shrink;
                         const int last_j = shrink ? g.n_shrink - 1 : ntiles - 1;
-                        hdr->flags = (j == first_j ? kFlagFirst : 0) | (j == last_j ? kFlagLast : 0);
+                        // the exchange follows the last shrink tile (of the last projection when shared)
+                        const bool last = j == last_j && !(shrink && p.mx && pi != p.P - 1);
+                        hdr->flags = (j == first_j ? kFlagFirst : 0) | (last ? kFlagLast : 0);
                         hdr->adapter = a;
                         hdr->rank = r;
-                        hdr->scale = d.scale;
+                        hdr->scale = dd.scale;
                         hdr->L = L;
                         hdr->off = off;
                         hdr->len = len;
                         hdr->proj = pi;
                         hdr->skind = pj.sigma_kind;
-                        hdr->sigma = d.sigma;
+                        hdr->sigma = dd.sigma;
                     }
                     __syncwarp();
                     if (lane == 0) {
                         mbar_arrive(smem_u32(&ctl.meta[s]));
-                        if (pi > 0 || j >= skip) issue_tile(g, pi, j, a, d, s);
+                        if (pi > 0 || j >= skip) issue_tile(g, pi, j, a, dd, s);
                     }
                     // L2 hints for the rows the consumers load for this tile (lane l: row l)
                     if (lane < L && (shrink || !p.yacc)) {
@@ -791,6 +809,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
         const int kind = hdr.kind;
         if (kind == kTileEnd) break;
         const int r = hdr.rank, L = hdr.L, flags = hdr.flags, len = hdr.len, off = hdr.off;
+        const int po = p.mx ? hdr.proj * RP : 0;   // this projection's slice of a token row
         const uint8_t *data = stage_base + (size_t)s * p.stage_bytes + kHeaderBytes;
         const int nch = len / EPC;   // 16-byte chunks per staged row
         if (tid == 0 && u < 6 && kind == kTileShrink && (flags & kFlagFirst)) LORA_TRACE_MARK(40 + 4 * u);
@@ -866,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         tot += __shfl_xor_sync(0xffffffffu, tot, 2);
                         tot += __shfl_xor_sync(0xffffffffu, tot, 1);
                         if ((lane & 7) == 0 && (!hi16 || l2) && (!hi8 || k2)) {
-                            float *dst = vpart + (l + (hi16 ? 1 : 0)) * RP + k + (hi8 ? kConsumerWarps : 0);
+                            float *dst = vpart + (l + (hi16 ? 1 : 0)) * VS + po + k + (hi8 ? kConsumerWarps : 0);
                             *dst = first ? tot : *dst + tot;
                         }
                     }
@@ -917,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         tot += __shfl_xor_sync(0xffffffffu, tot, 2);
                         tot += __shfl_xor_sync(0xffffffffu, tot, 1);
                         if ((lane & 7) == 0 && (!hi16 || l2) && (!hi8 || k2)) {
-                            float *dst = vpart + (l + (hi16 ? 1 : 0)) * RP + k + (hi8 ? kConsumerWarps : 0);
+                            float *dst = vpart + (l + (hi16 ? 1 : 0)) * VS + po + k + (hi8 ? kConsumerWarps : 0);
                             *dst = first ? tot : *dst + tot;
                         }
                         if (tid == 0 && l == 0 && k == warp && (unsigned)(it - kTraceTile0) < 2u)
@@ -941,9 +960,9 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     const bool okF =
                         u < 1 || mbar_wait_cluster(smem_u32(&ctl.freed), (u - 1) & 1, p.status, p.wait_ns);
                     if (tid == 0) LORA_TRACE_MARK(17);
-                    const int nq = L * RP / 4;            // float4 quads of the partial
+                    const int nq = L * VS / 4;            // float4 quads of the partial
                     const int lgq = ceil_log2(nq);
-                    const uint32_t my_slot = smem_u32(recv + crank * kTokChunk * RP);
+                    const uint32_t my_slot = smem_u32(recv + crank * kTokChunk * VS);
                     const uint32_t rbar = smem_u32(&ctl.recv);
                     for (int e = tid; e < (CL << lgq); e += kConsumers) {
                         const int peer = e >> lgq, qd = e & ((1 << lgq) - 1);
@@ -956,14 +975,16 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                     if (tid == 0) LORA_TRACE_MARK(18);
                     const bool okR = mbar_wait_cluster(rbar, u & 1, p.status, p.wait_ns);
                     if (tid == 0) LORA_TRACE_MARK(19);
-                    // ---- sum the CL partials in CTA order (entries k >= r are never read)
-                    for (int e = tid; e < (L << lgRP); e += kConsumers) {
-                        const int l = e >> lgRP, k = e & ((1 << lgRP) - 1);
-                        if (k < r) {
+                    // ---- sum the CL partials in CTA order (entries k >= r are never read; with a
+                    // shared exchange each projection's slice is summed whole)
+                    const int kmax = p.mx ? VS : r;
+                    for (int e = tid; e < (L << lgVS); e += kConsumers) {
+                        const int l = e >> lgVS, k = e & ((1 << lgVS) - 1);
+                        if (k < kmax) {
                             float acc = 0.f;
 #pragma unroll
-                            for (int j = 0; j < CL; ++j) acc += recv[(j * kTokChunk + l) * RP + k];
-                            vsum[l * RP + k] = acc;
+                            for (int j = 0; j < CL; ++j) acc += recv[(j * kTokChunk + l) * VS + k];
+                            vsum[l * VS + k] = acc;
                         }
                     }
                     if (tid == 0) LORA_TRACE_MARK(20);
@@ -1086,7 +1107,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                                   (E *)nullptr);
 #pragma unroll
                         for (int q = 0; q < TG; ++q) {
-                            const float *vr = vsum + (l0 + q) * RP + k;
+                            const float *vr = vsum + (l0 + q) * VS + po + k;
                             float v[EPC];
 #pragma unroll
                             for (int e = 0; e < EPC; e += 4) {
@@ -1105,7 +1126,7 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
                         for (int j = 0; j < CPT; ++j) {
                             const float b = (float)reinterpret_cast<const E *>(brow)[j * r + k];
 #pragma unroll
-                            for (int q = 0; q < TG; ++q) acc[q][j] = fmaf(vsum[(l0 + q) * RP + k], b, acc[q][j]);
+                            for (int q = 0; q < TG; ++q) acc[q][j] = fmaf(vsum[(l0 + q) * VS + po + k], b, acc[q][j]);
                         }
                     }
                 }
@@ -1178,7 +1199,8 @@ int launch_shape(const DecodeParams &p, LaunchShape &ls)
     });
     // Pipeline depth: aim for two CTAs per SM unless told otherwise.
     const int stage_bytes = kHeaderBytes + p.R * row_bytes_for(p.R);
-    const int fixed = make_layout(SRC, p.R, p.n, p.T, 0, stage_bytes, CL).total;
+    const int VP = p.mx ? p.P : 1;
+    const int fixed = make_layout(SRC, p.R, p.n, p.T, 0, stage_bytes, CL, VP).total;
     const int ctas_per_sm = opt.decode_ctas_per_sm > 0 ? (int)opt.decode_ctas_per_sm : 2;
     int stages = (int)opt.decode_stages;
     if (stages <= 0) {
@@ -1187,8 +1209,9 @@ int launch_shape(const DecodeParams &p, LaunchShape &ls)
     }
     // at least two stages: consumers read the next tile's header before releasing this one
     stages = max(2, min(kMaxStages, stages));
-    while (stages > 2 && make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes, CL).total > max_optin[dev]) --stages;
-    const Layout lay = make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes, CL);
+    while (stages > 2 && make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes, CL, VP).total > max_optin[dev])
+        --stages;
+    const Layout lay = make_layout(SRC, p.R, p.n, p.T, stages, stage_bytes, CL, VP);
     if (lay.total > max_optin[dev]) return LORA_ERR_UNSUPPORTED;
     static int smem_set[64];
     if (smem_set[dev] < lay.total) {
@@ -1270,21 +1293,30 @@ int launch_mode(const DecodeParams &p, cudaStream_t s)
     const int64_t forced = options().decode_cluster;
     int CL = (forced == 1 || forced == 2 || forced == 4) ? (int)forced : kMaxCluster;
     // The widest width whose pipeline fits in shared memory (the partial-exchange buffers grow
-    // with the width).
+    // with the width).  A shared exchange (grouped launch) multiplies those buffers by the
+    // projection count; it is dropped where it would not fit at a width, or would leave fewer
+    // than three pipeline stages, so that it never costs cluster width or depth.
+    DecodeParams q = p;
+    auto shape = [&](int cl, LaunchShape &ls) {
+        if (cl == 8) return launch_shape<E, MODE, SRC, 8>(q, ls);
+        if (cl == 4) return launch_shape<E, MODE, SRC, 4>(q, ls);
+        if (cl == 2) return launch_shape<E, MODE, SRC, 2>(q, ls);
+        return launch_shape<E, MODE, SRC, 1>(q, ls);
+    };
     for (;; CL >>= 1) {
         LaunchShape ls;
-        int rc = LORA_OK;
-        if (CL == 8) rc = launch_shape<E, MODE, SRC, 8>(p, ls);
-        else if (CL == 4) rc = launch_shape<E, MODE, SRC, 4>(p, ls);
-        else if (CL == 2) rc = launch_shape<E, MODE, SRC, 2>(p, ls);
-        else rc = launch_shape<E, MODE, SRC, 1>(p, ls);
+        int rc = shape(CL, ls);
+        if (q.mx && (rc == LORA_ERR_UNSUPPORTED || (rc == LORA_OK && ls.stages < 3))) {
+            q.mx = 0;
+            rc = shape(CL, ls);
+        }
         if (rc == LORA_OK || CL == 1 || rc != LORA_ERR_UNSUPPORTED) break;
     }
     switch (CL) {
-    case 8: return launch_one<E, MODE, SRC, 8>(p, units, s);
-    case 4: return launch_one<E, MODE, SRC, 4>(p, units, s);
-    case 2: return launch_one<E, MODE, SRC, 2>(p, units, s);
-    default: return launch_one<E, MODE, SRC, 1>(p, units, s);
+    case 8: return launch_one<E, MODE, SRC, 8>(q, units, s);
+    case 4: return launch_one<E, MODE, SRC, 4>(q, units, s);
+    case 2: return launch_one<E, MODE, SRC, 2>(q, units, s);
+    default: return launch_one<E, MODE, SRC, 1>(q, units, s);
     }
 }
 

@@ -45,6 +45,7 @@ Options &options()
         o.tc_min_seg_len = env_or("LORA_TC_MIN_SEG_LEN", o.tc_min_seg_len);
         o.tc_min_tokens = env_or("LORA_TC_MIN_TOKENS", o.tc_min_tokens);
         o.decode_balance = env_or("LORA_DECODE_BALANCE", o.decode_balance);
+        o.decode_shared_exchange = env_or("LORA_DECODE_SHARED_EXCHANGE", o.decode_shared_exchange);
     });
     return o;
 }
@@ -498,6 +499,11 @@ int lora_sgmv_grouped(const lora_table *const *tables, int32_t P, const lora_seg
         if (t->max_rank > p.R) p.R = t->max_rank;
         p.balance |= balance_for(t->min_rank, t->max_rank);
     }
+    // one exchange per unit for all projections, unless a projection applies Sigma_i after its
+    // own exchange
+    p.mx = (P > 1 && opt.decode_shared_exchange) ? 1 : 0;
+    for (int i = 0; i < P; ++i)
+        if (tables[i]->sigma_kind != LORA_SIGMA_NONE) p.mx = 0;
     return launch_decode(kModeFused, kSrcSegments, p, tables[0]->dtype, static_cast<cudaStream_t>(stream));
 }
 
@@ -661,6 +667,7 @@ int lora_set_option(const char *key, int64_t value)
     else if (!std::strcmp(key, "tc_min_seg_len")) o.tc_min_seg_len = value;
     else if (!std::strcmp(key, "tc_min_tokens")) o.tc_min_tokens = value;
     else if (!std::strcmp(key, "decode_balance")) o.decode_balance = value;
+    else if (!std::strcmp(key, "decode_shared_exchange")) o.decode_shared_exchange = value;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }
@@ -682,6 +689,7 @@ int lora_get_option(const char *key, int64_t *value)
     else if (!std::strcmp(key, "tc_min_seg_len")) *value = o.tc_min_seg_len;
     else if (!std::strcmp(key, "tc_min_tokens")) *value = o.tc_min_tokens;
     else if (!std::strcmp(key, "decode_balance")) *value = o.decode_balance;
+    else if (!std::strcmp(key, "decode_shared_exchange")) *value = o.decode_shared_exchange;
     else return LORA_ERR_INVALID_ARG;
     return LORA_OK;
 }

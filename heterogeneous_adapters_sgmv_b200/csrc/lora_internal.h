@@ -51,6 +51,7 @@ struct DecodeParams {
     int32_t inject;        // test-only stall injection (option "inject_stall"), 0 in normal use
     int32_t long_len;      // segments of at least this many tokens are served elsewhere (0: none)
     int32_t balance;       // segment tables: cost-balanced runs of units per cluster (1) or a fixed stride (0)
+    int32_t mx;            // grouped launch: one exchange per unit for all projections' shrinks (no Sigma)
     float *yacc;           // fused / expand: add the scaled delta to this fp32 [T, ldacc] array instead of
     int64_t ldacc;         // rounding it into y (merged ensembles summed before their one rounding), or null
     int32_t stages;        // pipeline depth
@@ -72,6 +73,7 @@ struct Options {
     int64_t tc_min_seg_len = 64;     // mixed batches: segments this long take the tcgen05 kernels (0: never)
     int64_t tc_min_tokens = 1024;    // ... in batches of at least this many tokens
     int64_t decode_balance = -1;     // segment units: -1 by the tables' rank spread, 0 fixed stride, 1 balanced runs
+    int64_t decode_shared_exchange = 1;  // grouped launches: one cluster exchange per unit for all projections
 };
 // Bound of the device-side waits for the next launch.
 uint64_t wait_limit_ns();

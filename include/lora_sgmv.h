@@ -280,8 +280,11 @@ const char *lora_status_string(int code);
  * (smallest batch that considers the split), "decode_balance" (segment tables on the cluster
  * kernel: -1, the default, cuts the units into runs of about equal estimated work per cluster
  * when the table's ranks differ by 2x or more, else deals them with a fixed stride; 0 always the
- * stride, 1 always the runs; results are bit-identical either way).  Returns LORA_ERR_INVALID_ARG for an unknown
- * key. */
+ * stride, 1 always the runs; results are bit-identical either way), "decode_shared_exchange"
+ * (lora_sgmv_grouped on the cluster kernel: 1, the default, runs each unit's shrink tiles of
+ * every projection first and exchanges their partials across the cluster once, then the
+ * expand tiles; 0 exchanges once per projection; tables with Sigma_i always take the latter;
+ * results are bit-identical either way).  Returns LORA_ERR_INVALID_ARG for an unknown key. */
 int lora_set_option(const char *key, int64_t value);
 int lora_get_option(const char *key, int64_t *value);
 

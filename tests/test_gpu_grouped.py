@@ -132,3 +132,35 @@ def test_grouped_split_option_runs_separate_calls():
         _grouped(dps, seg, [d.d.x for d in dps], ys, [0, 0])
     for pi, d in enumerate(dps):
         assert_close(d.to_np(ys[pi]), reference(name, proj=pi), wl.dtype, "split proj %d" % pi)
+
+
+@pytest.mark.parametrize("cluster", [8, 4, 1])
+def test_shared_exchange_is_bit_identical(cluster):
+    """One cluster exchange per unit for all projections (the default) against one per
+    projection: the same sums in the same order, so bit-identical outputs, here with three
+    projections (a token row of 3 x 16 partial slots) and with four of different ranks."""
+    wl = workload("many_adapter_qkvo")
+    dps = [DeviceProj(wl, pi) for pi in range(3)]
+    seg, _k = dps[0].segments()
+    x = dps[0].d.x
+    mixed = workloads.generate("multirank_decode", T=150, n=23, ranks=(8, 16, 32, 64),
+                               shapes=(("a", 1024, 1032, 0), ("b", 1032, 2048, 1), ("c", 1024, 512, 0),
+                                       ("d", 2048, 1024, 2)))
+    dpm = [DeviceProj(mixed, pi) for pi in range(4)]
+    segm, _km = dpm[0].segments()
+    with option("decode_cluster", cluster):
+        outs = {}
+        for shared in (1, 0):
+            with option("decode_shared_exchange", shared):
+                ys = [d.y() for d in dps]
+                _grouped(dps, seg, [x, x, x], ys, [0, 0, 0])
+                ym = [d.y() for d in dpm]
+                _grouped(dpm, segm, [d.d.x for d in dpm], ym, [0, 0, 0, 0])
+                torch.cuda.synchronize()
+                outs[shared] = ys + ym
+        for a, b in zip(outs[1], outs[0]):
+            assert torch.equal(a, b)
+        for pi, d in enumerate(dpm):
+            assert_close(d.to_np(outs[1][3 + pi]), oracle.workload_reference(mixed, pi), mixed.dtype,
+                         "shared exchange, mixed proj %d" % pi)
+    assert dps[0].status() == (0, 0) and dpm[0].status() == (0, 0)
