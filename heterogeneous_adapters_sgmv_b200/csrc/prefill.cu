@@ -408,6 +408,8 @@ constexpr int kExYBytes = 32768;                       // y tile: two 64-column 
 constexpr int kExBBytes = 16384;                       // B_i tile: 128 rows of o x 64 ranks
 constexpr int kExVBytes = 32768;                       // hi + lo intermediate tile
 constexpr int kExPoolPerCta = 3;                       // tiles per CTA dealt from the shared pool
+constexpr int kExPreTiles = 1;                         // tiles loaded before the wait on the shrink
+                                                       // (<= kExBStages; 2 measured 0.3 us slower)
 
 struct ExTileInfo {
     int32_t row0, rows, col0, ncols, vb;
@@ -485,7 +487,10 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         tmem_alloc(smem_u32(&ctl.tmem_base), 256);
         tmem_relinquish();
     }
-    pdl_wait();
+    // The shrink that precedes this kernel writes only the intermediate and the tile counter,
+    // and it lets this grid launch only after its own wait on everything before it: the
+    // segment table, y and the weights are final already.  Only the producer's intermediate
+    // loads and counter grabs wait for the shrink (below).
     pdl_launch_dependents();
     if (warp == 0) {
         const int tm = count_m_tiles(p);
@@ -514,6 +519,56 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
         int tk[4] = {0, 0, 0, 0};   // with a permutation: tokens of rows 4 lane .. 4 lane + 3
         float sc = 0.f;
         int grab = 0;   // lane 0: pool index taken ahead of its use
+        // The first tiles of the share (kExPreTiles, within one token tile): their y and B_i
+        // tiles are loaded before the wait on the shrink (tile info included); the loop then
+        // adds the intermediate load.
+        int npre = 0;
+        if ((p.tile_ctr ? S >= 1 : t0 < t1) && !(p.inject & 4)) {
+            const int g = t0 / NT;
+            int sg;
+            if (!find_tile(p, g, &sg, &row0, &rows, &a) || a < 0 || a >= p.n) {
+                if (lane == 0 && t0 - g * NT == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
+                row0 = 0;
+                rows = 0;
+                a = 0;
+            }
+            sc = p.desc[a].scale;
+            cur_g = g;
+            if (p.perm && rows > 0) tile_tokens(p, row0, rows, tk);
+            const int avail = p.tile_ctr ? S : t1 - t0;
+            for (int i = 0; i < kExPreTiles && i < avail && (t0 + i) / NT == g; ++i) {
+                const int nt = t0 + i - g * NT;
+                if (lane == 0) {
+                    EXPAND_MARK(i, 0);
+                    ExTileInfo &inf = ctl.info[i];
+                    inf.row0 = row0;
+                    inf.rows = rows;
+                    inf.col0 = nt * kTileN;
+                    inf.ncols = min(kTileN, p.o - nt * kTileN);
+                    inf.vb = 0;
+                    inf.scale = sc;
+                    uint8_t *yst = yring + i * kExYBytes;
+                    const uint32_t yb = smem_u32(&ctl.yfull[i]), bb = smem_u32(&ctl.bfull[i]);
+                    mbar_arrive_expect_tx(yb, kExYBytes);
+                    mbar_arrive_expect_tx(bb, kExBBytes);
+                    tma_load_2d(smem_u32(bring + i * kExBBytes), p.tm_B + (size_t)a * 128, 0, nt * kTileN, bb);
+                    if (!p.perm) {
+                        tma_load_2d(smem_u32(yst), &p.tmap_io, nt * kTileN, row0, yb);
+                        tma_load_2d(smem_u32(yst + 16384), &p.tmap_io, nt * kTileN + 64, row0, yb);
+                    }
+                }
+                __syncwarp();
+                if (p.perm) {
+                    const uint32_t yst = smem_u32(yring + i * kExYBytes), yb = smem_u32(&ctl.yfull[i]);
+                    tma_gather4(yst + lane * 512, &p.tmap_g, nt * kTileN, tk[0], tk[1], tk[2], tk[3], yb);
+                    tma_gather4(yst + 16384 + lane * 512, &p.tmap_g, nt * kTileN + 64, tk[0], tk[1], tk[2], tk[3],
+                                yb);
+                }
+                __syncwarp();
+                ++npre;
+            }
+        }
+        pdl_wait();
         for (int i = 0; ok; ++i) {
             // the tile of stage i: the share, then pool tiles (the next index is taken one tile
             // ahead, so the counter's round trip overlaps the tile before)
@@ -533,18 +588,24 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             }
             const int sy = i % kExYStages, sb = i % kExBStages;
             const int g = t / NT, nt = t - g * NT;
-            if (g != cur_g) {
+            const bool pre_i = i < npre;   // this tile's y and B_i are loaded already
+            const bool pre_v = i == 0 && npre > 0;   // its token tile was found above
+            if (g != cur_g || pre_v) {
                 int sg;
-                if (!find_tile(p, g, &sg, &row0, &rows, &a) || a < 0 || a >= p.n) {
+                if (pre_v) {
+                    // (tile found above)
+                } else if (!find_tile(p, g, &sg, &row0, &rows, &a) || a < 0 || a >= p.n) {
                     // a bad segment entry: keep the pipeline fed, store nothing for this tile
                     if (lane == 0 && nt == 0) atomicOr(p.status, LORA_STATUS_BAD_SEGMENT);
                     row0 = 0;
                     rows = 0;
                     a = 0;
                 }
-                sc = p.desc[a].scale;
-                cur_g = g;
-                if (p.perm && rows > 0) tile_tokens(p, row0, rows, tk);
+                if (!pre_v) {
+                    sc = p.desc[a].scale;
+                    cur_g = g;
+                    if (p.perm && rows > 0) tile_tokens(p, row0, rows, tk);
+                }
                 vb = vcount & 1;
                 if (vcount >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.vempty[vb]),
                                                                      ((vcount >> 1) - 1) & 1, p.status, p.wait_ns))) {
@@ -575,7 +636,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
             }
             // test-only stall: the first tile's stages are armed but never loaded
             const bool load = !((p.inject & 4) && i == 0);
-            if (lane == 0) {
+            if (lane == 0 && !pre_i) {
                 EXPAND_MARK(i, 0);
                 ExTileInfo &inf = ctl.info[sy];
                 inf.row0 = row0;
@@ -597,7 +658,7 @@ __global__ void __launch_bounds__(kThreadsEX, 1) prefill_expand_kernel(const __g
                 }
             }
             __syncwarp();
-            if (p.perm && load) {   // the y tile's rows, four per lane
+            if (p.perm && load && !pre_i) {   // the y tile's rows, four per lane
                 const uint32_t yst = smem_u32(yring + sy * kExYBytes);
                 const uint32_t yb = smem_u32(&ctl.yfull[sy]);
                 tma_gather4(yst + lane * 512, &p.tmap_g, nt * kTileN, tk[0], tk[1], tk[2], tk[3], yb);
