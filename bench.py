@@ -468,7 +468,7 @@ def secondary_lines(args, L, torch, dist, world):
         wl = workloads.generate(name, seed=rank_seed(name, int(os.environ.get("RANK", "0"))))
         ms, launches, kname, C, per, K, reps = timed_workload(args, L, torch, wl, grouped, 0.4, dist)
         b = accounting.workload_bytes(wl, shared_x=grouped)
-        traffic = profile_traffic(name) if not grouped else None
+        traffic = profile_traffic(name + ("_grouped" if grouped else ""))
         out.append({"workload": "%s: %s" % (name, workload_description(name, grouped)),
                     "tokens_per_step": wl.T, "value": round(job_throughput(world, wl.T, 1, ms), 1),
                     "unit": UNIT, "ms_per_step": round(ms, 6), "steps": K, "repetitions": reps,
@@ -640,8 +640,8 @@ def run_ours(args, rank, world, local_rank):
     value = job_throughput(world, T, K, ms)
     tm.release()
 
-    traffic = profile_traffic(args.workload) if not (args.grouped or args.sigma != "none" or args.merge > 1
-                                                     or args.base) else None
+    traffic = profile_traffic(args.workload + ("_grouped" if args.grouped else "")) if not (
+        args.sigma != "none" or args.merge > 1 or args.base) else None
     roofline = roofline_of(bytes_step, ms_step, launches_per_step, kname, traffic)
     if args.base:
         roofline = tensor_roofline(flops_step, ms_step, launches_per_step, kname)
