@@ -10,7 +10,8 @@
 //    the per-token BGMV form).  CTA j of the cluster streams the j-th CL-th of h for the shrink
 //    and the j-th CL-th of o for the expand, so each adapter's A_i and B_i are read once per
 //    unit and every token of the unit reuses that read.  Segment chunks are dealt to clusters
-//    round-robin, so a long segment spreads over many clusters.
+//    round-robin (or, when the table's ranks differ, in runs of about equal estimated work),
+//    so a long segment spreads over many clusters.
 //  * One producer warp per CTA runs ahead across units: it stages this CTA's slice of A_i with
 //    2-D tensor-map TMA loads (one or two instructions per unit) and its slice of B_i with one
 //    bulk copy, into a ring of shared-memory stages guarded by mbarriers, and hints the unit's
@@ -25,13 +26,14 @@
 //    in fixed CTA order.  No atomics, no grid barrier: bit-identical run to run.  A cluster of
 //    one keeps its own sum and exchanges nothing.  The three-stage form applies the adapter's
 //    Sigma_i (full or diagonal) to the summed intermediate here.
-//  * Expand: a thread owns two output columns (bf16) and takes the unit's tokens two at a time,
-//    sharing each B_i load; it walks its B rows from a rotated 16-byte chunk so a quarter warp
-//    hits distinct shared-memory banks; one rounding (nearest-even) per output, coalesced
-//    32-bit stores.  A per-token weight (merged ensembles) multiplies the
-//    scale.
-//  * A grouped launch carries up to four projections (tables, x, y slices); each unit then
-//    runs once per projection, back to back on the same cluster.
+//  * Expand: a thread owns two output columns (bf16) and takes the unit's tokens two or four
+//    at a time, sharing each B_i load; it walks its B rows from a rotated 16-byte chunk so a
+//    quarter warp hits distinct shared-memory banks; one rounding (nearest-even) per output,
+//    coalesced 32-bit stores.  A per-token weight (merged ensembles) multiplies the scale; with
+//    an fp32 sum (merged ensembles rounded once) the term is added there instead of into y.
+//  * A grouped launch carries up to four projections (tables, x, y slices); each unit runs
+//    the shrink tiles of every projection, one cluster exchange of all their partials, then
+//    the expand tiles, back to back on the same cluster.
 //  * Short kernels like this one are dominated by instruction fetch and dependent latency, so
 //    the per-unit code is kept to a few compact loops (no run-time integer division), and
 //    work that reads no input (barrier set-up; in the direct BGMV mode the adapter descriptor
