@@ -191,3 +191,30 @@ def test_merged_fp32_sum_f32_outputs():
     assert ran(names, "merge_finish_kernel")
     assert_close(dp.to_np(y), _ref(wl, dp, ids2, w2), wl.dtype, "merged fp32 sum, f32")
     assert dp.status() == (0, 0)
+
+
+@pytest.mark.parametrize("fp32_sum", [False, True])
+def test_merged_with_sigma_tables(fp32_sum):
+    """Merged ensembles over a table in the three-stage form (full Sigma_i), K = 2, in both
+    rounding modes, against the oracle: the three-stage oracle's delta of each slot (y0 = 0),
+    weighted per token and added to y0 in fp64 (the update is linear in each slot's term)."""
+    wl = workload("decode_bgmv")
+    dp = DeviceProj(wl)
+    p = dp.p
+    sig = workloads.draw_sigma(p.ranks, "full", 53)
+    dev = [torch.from_numpy(s).cuda() for s in sig]
+    dp.table.set_sigma(L.LORA_SIGMA_FULL, dev)
+    ids2, w2 = workloads.draw_merge(wl.ids, wl.n, 2, seed=55, empty=0.25)
+    A = [p.A(i) for i in range(wl.n)]
+    B = [p.B(i) for i in range(wl.n)]
+    zeros = np.zeros_like(p.y0)
+    ref = workloads.to_float64(p.y0, wl.dtype).copy()
+    for j in range(2):
+        dj = oracle.lora_delta_sigma(wl.dtype, p.x, zeros, ids2[:, j].copy(), A, B, p.scales, oracle.SIGMA_FULL, sig)
+        ref += w2[:, j:j + 1].astype(np.float64) * dj
+    ws = _sum_workspace(dp, wl.T) if fp32_sum else None
+    y = dp.y()
+    names = kernels_launched(lambda: _merged(dp, ids2, w2, y, ws))
+    assert ran(names, "merge_finish_kernel") == fp32_sum
+    assert_close(dp.to_np(y), ref, wl.dtype, "merged sigma, fp32 sum %s" % fp32_sum)
+    assert dp.status() == (0, 0)
