@@ -6,8 +6,8 @@
 // run to run:
 //  * counting sort, for decode-sized batches (T <= 512, n < 8192): one histogram of the
 //    adapter ids in shared memory (warp-aggregated atomics: counts only, not positions), one
-//    exclusive scan giving each adapter's first position and one giving segment indices,
-//    then every token is placed at its adapter's first position plus the number of earlier
+//    exclusive scan of packed (count, non-empty) pairs giving each adapter's first position
+//    and its segment index at once, then every token is placed at its adapter's first position plus the number of earlier
 //    tokens with the same adapter, so positions never depend on timing (that count costs
 //    O(T^2) compares over the block, which is why larger batches take the radix sort);
 //  * least-significant-digit radix sort for the rest (8-bit digits, as many passes as the
@@ -164,7 +164,10 @@ build_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int
     }
 }
 
-// Counting sort (see above).  Shared memory: cnt[n + 1], flag[n], key[T].
+// Counting sort (see above).  Shared memory: cnt[n + 1], key[T].  One scan gives both the first
+// position of each adapter and its segment index: entry i holds (count_i << 16) | (count_i > 0)
+// before the scan, so after it the high half is the position and the low half the number of
+// non-empty adapters before i (T <= 512 and n <= 8191 keep both halves below 2^16).
 __global__ void __launch_bounds__(kSegThreads, 1)
 count_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int32_t *__restrict__ perm,
                       int32_t *__restrict__ seg_ptr, int32_t *__restrict__ seg_adapter,
@@ -174,9 +177,9 @@ count_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int
     pdl_launch_dependents();
 
     extern __shared__ __align__(16) int32_t sm[];
-    int32_t *cnt = sm, *flag = sm + (n + 1), *key_s = flag + n;
+    int32_t *cnt = sm, *key_s = sm + (n + 1);
     __shared__ int32_t warp_sums[kSegWarps];
-    __shared__ int32_t total, segs;
+    __shared__ int32_t total;
     __shared__ uint32_t bad;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) bad = 0;
@@ -200,15 +203,19 @@ count_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int
     }
     __syncthreads();
     if (tid == 0 && bad) atomicOr(status, LORA_STATUS_BAD_ID);
-    for (int i = tid; i < n; i += kSegThreads) flag[i] = cnt[i] > 0 ? 1 : 0;
+    for (int i = tid; i <= n; i += kSegThreads) {
+        const int32_t c = cnt[i];
+        cnt[i] = (c << 16) | (i < n && c > 0 ? 1 : 0);
+    }
     __syncthreads();
-    block_exclusive_scan(cnt, n + 1, warp_sums, &total);   // cnt[i]: first position of adapter i
-    block_exclusive_scan(flag, n, warp_sums, &segs);       // flag[i]: segment index of adapter i
-    const int32_t valid = cnt[n];
+    block_exclusive_scan(cnt, n + 1, warp_sums, &total);   // cnt[i]: (first position << 16) | segment
+    const int32_t valid = cnt[n] >> 16;
+    const int32_t segs = cnt[n] & 0xFFFF;
     for (int i = tid; i < n; i += kSegThreads) {
-        if (cnt[i + 1] > cnt[i]) {
-            seg_ptr[flag[i]] = cnt[i];
-            seg_adapter[flag[i]] = i;
+        const int32_t e = cnt[i];
+        if ((cnt[i + 1] >> 16) > (e >> 16)) {
+            seg_ptr[e & 0xFFFF] = e >> 16;
+            seg_adapter[e & 0xFFFF] = i;
         }
     }
     if (tid == 0) {
@@ -232,12 +239,13 @@ count_segments_kernel(const int32_t *__restrict__ ids, int32_t T, int32_t n, int
         // the warp's own earlier lanes
         const uint32_t peers = __match_any_sync(0xffffffffu, key);
         rank += __popc(peers & ((1u << lane) - 1u));
-        if (ok && key < n) perm[cnt[key] + rank] = t;
+        if (ok && key < n) perm[(cnt[key] >> 16) + rank] = t;
     }
 }
 
 constexpr int kCountMaxT = 512;   // above this the radix sort is faster (measured)
 constexpr int kCountMaxN = 8191;
+static_assert(kCountMaxT < 32768 && kCountMaxN < 65536, "packed (position, segment) scan");
 
 }  // namespace
 
@@ -245,12 +253,12 @@ int launch_build_segments(const int32_t *ids, int32_t T, int32_t n, int32_t *per
                           int32_t *seg_adapter, int32_t *num_segs, uint32_t *status, cudaStream_t s)
 {
     const bool counting = T <= kCountMaxT && n <= kCountMaxN;
-    const size_t smem = counting ? (size_t)(2 * n + 1 + T) * sizeof(int32_t)
+    const size_t smem = counting ? (size_t)(n + 1 + T) * sizeof(int32_t)
                                  : (size_t)(4 * T + kHistEntries) * sizeof(int32_t);
     static bool attr_set = false;
     if (!attr_set) {
         const int max_smem = (4 * LORA_MAX_SEGMENT_TOKENS + kHistEntries) * (int)sizeof(int32_t);
-        const int max_count = (2 * kCountMaxN + 1 + kCountMaxT) * (int)sizeof(int32_t);
+        const int max_count = (kCountMaxN + 1 + kCountMaxT) * (int)sizeof(int32_t);
         if (cudaFuncSetAttribute(build_segments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  max_smem) != cudaSuccess ||
             cudaFuncSetAttribute(count_segments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
