@@ -684,74 +684,72 @@ __global__ void __launch_bounds__(kThreads, 2) lora_decode_kernel(const __grid_c
             // shrink tiles of every projection come first, then all its expand tiles: the
             // consumers exchange the projections' partials once, after the last shrink tile.
             const int npass = p.mx ? 2 : 1;
-            for (int pass = 0; pass < npass && alive; ++pass) {
-                for (int pi = 0; pi < p.P && alive; ++pi) {
-                    const ProjParams &pj = p.pj[pi];
-                    const AdapterDesc dd = pi == 0 ? d : pj.desc[a];
-                    const Geo g = pi == 0 ? geo0 : geo_of(pi);
-                    const int r = dd.rank;
-                    const int ntiles = g.n_shrink + g.n_expand;
-                    const int j0 = (p.mx && pass == 1) ? g.n_shrink : 0;
-                    const int j1 = (p.mx && pass == 0) ? g.n_shrink : ntiles;
-                    if (pj.sigma_kind != LORA_SIGMA_NONE) {   // the consumers read Sigma_i after the shrink
-                        const int sbytes = (pj.sigma_kind == LORA_SIGMA_FULL ? r * r : r) * 4;
-                        for (int c = lane * 128; c < sbytes; c += 32 * 128)
-                            prefetch_l2(reinterpret_cast<const uint8_t *>(dd.sigma) + c);
+            for (int step = 0; step < npass * p.P && alive; ++step) {
+                const int pass = step / p.P, pi = step - pass * p.P;
+                const ProjParams &pj = p.pj[pi];
+                const AdapterDesc dd = pi == 0 ? d : pj.desc[a];
+                const Geo g = pi == 0 ? geo0 : geo_of(pi);
+                const int r = dd.rank;
+                const int ntiles = g.n_shrink + g.n_expand;
+                const int j0 = (p.mx && pass == 1) ? g.n_shrink : 0;
+                const int j1 = (p.mx && pass == 0) ? g.n_shrink : ntiles;
+                if (pj.sigma_kind != LORA_SIGMA_NONE) {   // the consumers read Sigma_i after the shrink
+                    const int sbytes = (pj.sigma_kind == LORA_SIGMA_FULL ? r * r : r) * 4;
+                    for (int c = lane * 128; c < sbytes; c += 32 * 128)
+                        prefetch_l2(reinterpret_cast<const uint8_t *>(dd.sigma) + c);
+                }
+                for (int j = j0; j < j1; ++j) {
+                    const int s = ps, m = pround;
+                    if (m >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status,
+                                                                      p.wait_ns))) {
+                        alive = false;
+                        break;
                     }
-                    for (int j = j0; j < j1; ++j) {
-                        const int s = ps, m = pround;
-                        if (m >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&ctl.empty[s]), (m - 1) & 1, p.status,
-                                                                          p.wait_ns))) {
-                            alive = false;
-                            break;
-                        }
-                        StageHeader *hdr = reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
-                        const bool shrink = j < g.n_shrink;
-                        int off, len, nbox;
-                        tile_geom(g, j, r, off, len, nbox);
-                        if (lane < L) {
-                            hdr->tok[lane] = my_tok;
-                            hdr->tw[lane] = SRC == kSrcIds ? w_s[my_tok]
-                                            : !p.tok_w ? 1.f
-                                                       : p.tok_w[(int64_t)my_tok * p.w_stride];
-                        }
-                        if (lane == 0) {
-                            hdr->kind = shrink ? kTileShrink : kTileExpand;
-                            const int first_j = shrink ? 0 : g.n_shrink;
-                            const int last_j = shrink ? g.n_shrink - 1 : ntiles - 1;
-                            // the exchange follows the last shrink tile (of the last projection when shared)
-                            const bool last = j == last_j && !(shrink && p.mx && pi != p.P - 1);
-                            hdr->flags = (j == first_j ? kFlagFirst : 0) | (last ? kFlagLast : 0);
-                            hdr->adapter = a;
-                            hdr->rank = r;
-                            hdr->scale = dd.scale;
-                            hdr->L = L;
-                            hdr->off = off;
-                            hdr->len = len;
-                            hdr->proj = pi;
-                            hdr->skind = pj.sigma_kind;
-                            hdr->sigma = dd.sigma;
-                        }
-                        __syncwarp();
-                        if (lane == 0) {
-                            mbar_arrive(smem_u32(&ctl.meta[s]));
-                            if (pi > 0 || j >= skip) issue_tile(g, pi, j, a, dd, s);
-                        }
-                        // L2 hints for the rows the consumers load for this tile (lane l: row l)
-                        if (lane < L && (shrink || !p.yacc)) {
-                            const uint8_t *row =
-                                shrink ? static_cast<const uint8_t *>(pj.x) + ((int64_t)my_tok * pj.ldx + off) * ESZ
-                                       : static_cast<const uint8_t *>(pj.y) +
-                                             ((int64_t)my_tok * pj.ldy + pj.y_off + off) * ESZ;
-                            for (int c = 0; c < len * ESZ; c += 128) prefetch_l2(row + c);
-                        }
-                        ++issued;
-                        if (++ps == S) {
-                            ps = 0;
-                            ++pround;
-                        }
-                        if (lane == 0) LORA_TRACE_MARK(shrink ? 3 : 4);
+                    StageHeader *hdr = reinterpret_cast<StageHeader *>(stage_base + (size_t)s * p.stage_bytes);
+                    const bool shrink = j < g.n_shrink;
+                    int off, len, nbox;
+                    tile_geom(g, j, r, off, len, nbox);
+                    if (lane < L) {
+                        hdr->tok[lane] = my_tok;
+                        hdr->tw[lane] = SRC == kSrcIds ? w_s[my_tok]
+                                        : !p.tok_w ? 1.f
+                                                   : p.tok_w[(int64_t)my_tok * p.w_stride];
                     }
+                    if (lane == 0) {
+                        hdr->kind = shrink ? kTileShrink : kTileExpand;
+                        const int first_j = shrink ? 0 : g.n_shrink;
+                        const int last_j = shrink ? g.n_shrink - 1 : ntiles - 1;
+                        // the exchange follows the last shrink tile (of the last projection when shared)
+                        const bool last = j == last_j && !(shrink && p.mx && pi != p.P - 1);
+                        hdr->flags = (j == first_j ? kFlagFirst : 0) | (last ? kFlagLast : 0);
+                        hdr->adapter = a;
+                        hdr->rank = r;
+                        hdr->scale = dd.scale;
+                        hdr->L = L;
+                        hdr->off = off;
+                        hdr->len = len;
+                        hdr->proj = pi;
+                        hdr->skind = pj.sigma_kind;
+                        hdr->sigma = dd.sigma;
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(smem_u32(&ctl.meta[s]));
+                        if (pi > 0 || j >= skip) issue_tile(g, pi, j, a, dd, s);
+                    }
+                    // L2 hints for the rows the consumers load for this tile (lane l: row l)
+                    if (lane < L && (shrink || !p.yacc)) {
+                        const uint8_t *row =
+                            shrink ? static_cast<const uint8_t *>(pj.x) + ((int64_t)my_tok * pj.ldx + off) * ESZ
+                                   : static_cast<const uint8_t *>(pj.y) + ((int64_t)my_tok * pj.ldy + pj.y_off + off) * ESZ;
+                        for (int c = 0; c < len * ESZ; c += 128) prefetch_l2(row + c);
+                    }
+                    ++issued;
+                    if (++ps == S) {
+                        ps = 0;
+                        ++pround;
+                    }
+                    if (lane == 0) LORA_TRACE_MARK(shrink ? 3 : 4);
                 }
             }
         }
